@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark: OrbitQuant online quantized-linear path on B200.
+
+One step = the whole hot path on one batch: oq_quantize_act (fused RPBH rotate + norm +
+Lloyd-Max codes of the activations) followed by oq_linear (codebook GEMM against weight codes
+quantized offline, before timing).  Default workload: the FLUX-like attention projection
+(T = 4608 tokens, d = 3072 -> 3072, bf16 inputs, h = 128, W4A4).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch of T tokens (weak
+scaling; the path has no exchange step, so no collective touches the data); the timed region
+is bracketed by a barrier + synchronize, and the max over ranks is reported.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (rank 0 only).
+Rank 0 prints one JSON line on stdout; everything else goes to stderr.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from calibration_free_bit_b200 import synth  # noqa: E402
+
+METRIC = ("quantized-linear tokens/s at d=3072; % of HBM (quantize) / BF16 tensor (GEMM) "
+          "peak")
+NSETS = 4            # rotating buffer sets: working set > L2 between reuses
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="flux_attn_w4a4")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profile_traffic(profile_name, kernel_src):
+    """DRAM bytes per launch from a committed ncu summary, or None if absent or stale (the
+    summary records the kernel source hash it was captured from)."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    if not os.path.exists(path):
+        return None, "no profile"
+    text = open(path).read()
+    m = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not h:
+        return None, "profile lacks traffic"
+    if h.group(1) != source_sha(kernel_src):
+        return None, "kernel changed since capture"
+    return float(m.group(1)), "ncu"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.target = str(device_index)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", self.target], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        sm, smax, power, reasons = [], [], [], set()
+        for line in self.out.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.out.name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------
+# oracle (CPU) arm: used for --impl reference and for the cpu_baseline field
+# ------------------------------------------------------------------------------------------
+
+class OracleStep:
+    """The oracle's version of one step on S tokens: fp64 RPBH + Lloyd-Max codes of the
+    activations, then the naive triple-loop linear against all output features."""
+
+    def __init__(self, p):
+        import oracle as O
+        self.O, self.p = O, p
+        self.perm, self.sign = O.build_rpbh(p.d, 0)
+        W = synth.weight(p).double().numpy()
+        self.wc, self.rn = O.quantize_weight(W, p.h, self.perm, self.sign, p.bits_w)
+        self.x = synth.activations(p, rows=np.arange(min(p.T, 2048))).double().numpy()
+        self.cursor = 0
+
+    def run(self, S):
+        rows = (self.cursor + np.arange(S)) % len(self.x)
+        self.cursor = int(rows[-1] + 1)
+        t0 = time.perf_counter()
+        xc, s = self.O.quantize_act(self.x[rows], self.p.h, self.perm, self.sign, self.p.bits_a)
+        self.O.linear(xc, s, self.wc, self.rn, self.p.d, self.p.bits_a, self.p.bits_w)
+        return time.perf_counter() - t0
+
+
+def cores_used():
+    return 1   # the oracle is single-threaded C
+
+
+def run_reference(args, p):
+    step = OracleStep(p)
+    probe = step.run(4) / 4                          # seconds per token, calibration
+    budget = 120.0                                   # seconds for warmup + timed steps
+    S = int(max(1, min(512, budget / max(1, args.steps + args.warmup) / max(probe, 1e-9))))
+    for _ in range(args.warmup):
+        step.run(S)
+    total = 0.0
+    for _ in range(args.steps):
+        total += step.run(S)
+    value = S * args.steps / total
+    sample = (f"{S} tokens per step of the {p.name} workload (d={p.d} -> {p.out}): fp64 "
+              f"rotate+quantize of the S rows, then all {p.out} outputs by the naive loop")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(p, 1),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores_used(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def cpu_baseline(p):
+    step = OracleStep(p)
+    per_tok = step.run(8) / 8
+    S = int(max(8, min(1024, 15.0 / max(per_tok, 1e-9))))
+    t = step.run(S)
+    return {"value": S / t, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+            "sample": f"{S} tokens of {p.name}: fp64 rotate+quantize then all {p.out} outputs "
+                      f"(naive loop), {t:.1f} s on one host core"}
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (the only collective: timing, not data)."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: int, steps: int, ms_max: float) -> float:
+    """Units all ranks processed, divided by the slowest rank's time (weak scaling)."""
+    return world * units_per_rank_step * steps / (ms_max / 1e3)
+
+
+def workload_config(p, world):
+    return {"workload": f"{p.name}: FLUX-like attention projection" if p.name.startswith(
+                "flux_attn") else p.name,
+            "T_per_gpu": p.T, "d": p.d, "out": p.out, "h": p.h, "bits_w": p.bits_w,
+            "bits_a": p.bits_a, "input": "bf16" if p.dtype == torch.bfloat16 else "fp32",
+            "l2": f"{NSETS} rotating buffer sets (x, codes, s, y, W codes) > 126 MB L2",
+            "parallelism": f"dp{world}: independent token batches, no collective"}
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+
+def run_ours(args, p, rank, world, dev):
+    from calibration_free_bit_b200 import build as B
+    B.build()
+    from calibration_free_bit_b200 import oq
+
+    r = oq.oq_build_rpbh(p.d, p.h, 0)
+    ca, cw = oq.oq_lloyd_max(p.d, p.bits_a), oq.oq_lloyd_max(p.d, p.bits_w)
+    x_cpu = synth.activations(p)
+    W = synth.weight(p).to(dev)
+    wc0, rn = oq.oq_quantize_weight(r, cw, W)                # offline, untimed
+    del W
+    sets = []
+    for _ in range(NSETS):
+        x = x_cpu.to(dev)
+        sets.append({
+            "x": x,
+            "xc": torch.empty((p.T, p.d * p.bits_a // 8), dtype=torch.uint8, device=dev),
+            "s": torch.empty(p.T, dtype=torch.float32, device=dev),
+            "y": torch.empty((p.T, p.out), dtype=torch.float32, device=dev),
+            "wc": wc0.clone(),
+        })
+    torch.cuda.synchronize()
+
+    def step(i):
+        b = sets[i % NSETS]
+        oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"])
+        oq.oq_linear(ca, cw, b["xc"], b["s"], b["wc"], rn, b["y"])
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i)
+    oq.oq_check()
+    oq.oq_timing_collect()
+
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    barrier()
+    if clocks:
+        clocks.start()
+    oq.oq_timing_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for i in range(args.steps):
+        step(i)
+    ev1.record()
+    barrier()
+    oq.oq_timing_enable(False)
+    clock_info = clocks.stop() if clocks else None
+    oq.oq_check()
+    ms = ev0.elapsed_time(ev1)
+    recs = oq.oq_timing_collect()
+    per_kernel = {}
+    for name, t in recs:
+        per_kernel.setdefault(name, []).append(t)
+    launches = len(recs)
+
+    ms_max = max_over_ranks(ms, world, dev)
+
+    # end-to-end through the public calls with host buffers (pinned), copies inside timing
+    e2e = None
+    if not args.no_e2e:
+        xh = x_cpu.pin_memory()
+        yh = torch.empty((p.T, p.out), dtype=torch.float32).pin_memory()
+        b = sets[0]
+
+        def e2e_step():
+            b["x"].copy_(xh, non_blocking=True)
+            oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"])
+            oq.oq_linear(ca, cw, b["xc"], b["s"], b["wc"], rn, b["y"])
+            yh.copy_(b["y"], non_blocking=True)
+
+        for _ in range(max(3, min(args.warmup, 20))):
+            e2e_step()
+        n_e2e = max(1, min(args.steps, 500))
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record()
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": whole_job_rate(world, p.T, n_e2e, e_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+               "d2h_bytes_per_step": yh.numel() * yh.element_size(), "steps": n_e2e,
+               "ms_per_step": e_ms / n_e2e}
+
+    if rank != 0:
+        return None
+
+    pk, pk_kind = peaks()
+    gemm_ms = statistics.mean(per_kernel.get("gemm", [float("nan")]))
+    quant_ms = statistics.mean(per_kernel.get("quantize", [float("nan")]))
+    dec_ms = statistics.mean(per_kernel.get("decode", [float("nan")]))
+    flops = 2.0 * p.T * p.d * p.out
+    gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
+    traffic, traffic_src = profile_traffic(f"k2_gemm_{p.name}.md", "calibration_free_bit_b200/"
+                                           "csrc/k2_linear.cu")
+    in_bytes = 2 if p.dtype == torch.bfloat16 else 4
+    q_bytes = p.T * (in_bytes * p.d + p.d * p.bits_a // 8 + 4)
+    q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": whole_job_rate(world, p.T, args.steps, ms_max),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16xf16->f32 (gemm), f32 (quantize)",
+        "data": "synthetic",
+        "config": workload_config(p, world),
+        "kernels_ms_mean": {"quantize": quant_ms, "decode": dec_ms, "gemm": gemm_ms},
+        "roofline": {
+            "kernel": "k2_gemm (tcgen05 kind::f16, 128x256x64 tiles)",
+            "bound": "tensor", "achieved": gemm_tf,
+            "peak": pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+            "peak_note": f"{pk_kind} dense bf16 burst (fp16 kind::f16 runs at the bf16 rate)",
+            "unit": "TFLOP/s",
+            "frac": gemm_tf / pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+            "traffic": traffic, "traffic_source": traffic_src,
+            "algorithmic_per_launch": flops,
+        },
+        "roofline_quantize": {
+            "kernel": "k1_rotquant", "bound": "hbm", "achieved": q_gbs,
+            "peak": pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "unit": "GB/s",
+            "frac": q_gbs / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+            "frac_of_8TBps_nominal": q_gbs / 8000.0,
+            "algorithmic_bytes_per_launch": q_bytes,
+        },
+        "gpu_launches": launches,
+        "clocks": clock_info,
+    }
+    if e2e:
+        out["e2e"] = e2e
+    return out
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    p = synth.get(args.workload)[0]
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, p)), flush=True)
+        return
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        out = run_ours(args, p, rank, world, dev)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(p)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

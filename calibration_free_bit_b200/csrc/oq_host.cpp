@@ -1,0 +1,702 @@
+// oq_host.cpp -- host side of liboq: handles, table builders, validation and launches.
+//
+// Table builders follow rcap.io, "OrbitQuant: Data-Agnostic Quantization for Image and
+// Video": pseudocode build_rpbh(d) (RPBH paragraph: uniform random permutation, random sign
+// flips, block Walsh-Hadamard) and lloyd_max(f_d, b) (change-of-basis paragraph: the standard
+// Lloyd-Max quantizer for the fixed marginal, read as N(0, 1/d)).  The generator and draw
+// order are the ones documented in include/oq.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <limits>
+#include <new>
+
+#include "oq_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int fail_cuda(cudaError_t e, const char *what) {
+    return fail(OQ_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Optional per-kernel timing (oq_timing_enable / oq_timing_collect): events recorded on the
+// caller's stream around every kernel this thread launches through the C ABI.
+struct TimedLaunch {
+    int kernel;
+    cudaEvent_t start, stop;
+};
+thread_local bool g_timing = false;
+thread_local std::vector<TimedLaunch> g_timed;
+thread_local std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess)
+        return nullptr;
+    return e;
+}
+
+// Run `launch` (returning cudaError_t), bracketed by events when timing is on.
+template <class F>
+cudaError_t timed(int kernel, cudaStream_t st, F &&launch) {
+    if (!g_timing)
+        return launch();
+    TimedLaunch t{kernel, take_event(), take_event()};
+    if (t.start)
+        cudaEventRecord(t.start, st);
+    cudaError_t e = launch();
+    if (t.stop)
+        cudaEventRecord(t.stop, st);
+    if (t.start && t.stop)
+        g_timed.push_back(t);
+    return e;
+}
+
+// ---------------------------------------------------------------------------------------
+// RPBH tables.  SplitMix64 (Steele, Lea & Flood 2014), Fisher-Yates (Durstenfeld) with
+// rejection-sampled bounded integers, then one sign per position from the draw's top bit.
+// ---------------------------------------------------------------------------------------
+struct SplitMix64 {
+    uint64_t x;
+    uint64_t next() {
+        uint64_t z = (x += 0x9E3779B97F4A7C15ULL);
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+        return z ^ (z >> 31);
+    }
+    // uniform in [0, n): reject the top 2^64 mod n values
+    uint64_t below(uint64_t n) {
+        const uint64_t cut = (uint64_t)(-n) % n;     // 2^64 mod n
+        for (;;) {
+            const uint64_t r = next();
+            if (cut == 0 || r < (uint64_t)0 - cut)
+                return r % n;
+        }
+    }
+};
+
+// ---------------------------------------------------------------------------------------
+// Lloyd-Max for N(0,1): Lloyd warm-up, then Newton on the centroid conditions
+// c_i = E[X | t_i <= X < t_{i+1}], t_i = (c_{i-1} + c_i)/2, with the tridiagonal Jacobian
+// d mu_i / d t_i = phi(t_i)(mu_i - t_i)/P_i,  d mu_i / d t_{i+1} = phi(t_{i+1})(t_{i+1} - mu_i)/P_i.
+// ---------------------------------------------------------------------------------------
+double npdf(double x) { return std::isinf(x) ? 0.0 : std::exp(-0.5 * x * x) * 0.3989422804014327; }
+double ntail(double x) {   // P(X > x)
+    if (std::isinf(x))
+        return x > 0 ? 0.0 : 1.0;
+    return 0.5 * std::erfc(x * 0.7071067811865476);
+}
+double nprob(double a, double b) {   // P(a <= X < b), a < b
+    if (a >= 0)
+        return ntail(a) - ntail(b);
+    if (b <= 0)
+        return ntail(-b) - ntail(-a);
+    return 1.0 - ntail(-a) - ntail(b);
+}
+
+bool solve_lloyd_max(int L, std::vector<double> &c) {
+    const double inf = std::numeric_limits<double>::infinity();
+    c.assign(L, 0.0);
+    const double span = 1.5 + 0.4 * std::log2((double)L);
+    for (int i = 0; i < L; ++i)
+        c[i] = span * (2.0 * (i + 0.5) / L - 1.0);
+    std::vector<double> t(L + 1), mu(L), da(L), db(L);
+    auto cells = [&]() {
+        t[0] = -inf;
+        t[L] = inf;
+        for (int i = 1; i < L; ++i)
+            t[i] = 0.5 * (c[i - 1] + c[i]);
+        for (int i = 0; i < L; ++i) {
+            const double a = t[i], b = t[i + 1];
+            const double P = nprob(a, b);
+            mu[i] = (npdf(a) - npdf(b)) / P;
+            da[i] = std::isinf(a) ? 0.0 : npdf(a) * (mu[i] - a) / P;
+            db[i] = std::isinf(b) ? 0.0 : npdf(b) * (b - mu[i]) / P;
+        }
+    };
+    // Lloyd iterations bring every cell near the optimum
+    for (int it = 0; it < 400 + 4 * L; ++it) {
+        cells();
+        for (int i = 0; i < L; ++i)
+            c[i] = mu[i];
+    }
+    // Newton with step halving that keeps the centroids ordered
+    std::vector<double> lo(L), di(L), up(L), r(L), step(L), cp(L), dp(L);
+    for (int it = 0; it < 60; ++it) {
+        cells();
+        double rmax = 0.0;
+        for (int i = 0; i < L; ++i) {
+            r[i] = c[i] - mu[i];
+            rmax = std::max(rmax, std::fabs(r[i]));
+            lo[i] = -0.5 * da[i];
+            up[i] = -0.5 * db[i];
+            di[i] = 1.0 - 0.5 * (da[i] + db[i]);
+        }
+        if (rmax < 1e-15)
+            break;
+        // Thomas algorithm (diagonally dominant: da + db < 1 for a log-concave density)
+        cp[0] = up[0] / di[0];
+        dp[0] = r[0] / di[0];
+        for (int i = 1; i < L; ++i) {
+            const double m = di[i] - lo[i] * cp[i - 1];
+            cp[i] = up[i] / m;
+            dp[i] = (r[i] - lo[i] * dp[i - 1]) / m;
+        }
+        step[L - 1] = dp[L - 1];
+        for (int i = L - 2; i >= 0; --i)
+            step[i] = dp[i] - cp[i] * step[i + 1];
+        double lam = 1.0;
+        for (int tries = 0; tries < 30; ++tries, lam *= 0.5) {
+            bool ordered = true;
+            for (int i = 1; i < L && ordered; ++i)
+                ordered = (c[i] - lam * step[i]) > (c[i - 1] - lam * step[i - 1]);
+            if (ordered)
+                break;
+        }
+        for (int i = 0; i < L; ++i)
+            c[i] -= lam * step[i];
+    }
+    // exact symmetry of the N(0,1) problem
+    for (int i = 0; i < L / 2; ++i) {
+        const double m = 0.5 * (c[L - 1 - i] - c[i]);
+        c[i] = -m;
+        c[L - 1 - i] = m;
+    }
+    cells();
+    double rmax = 0.0;
+    for (int i = 0; i < L; ++i)
+        rmax = std::max(rmax, std::fabs(c[i] - mu[i]));
+    return rmax < 1e-12;
+}
+
+// IEEE binary16, round to nearest even (normal range and zero; centroids are in [1e-3, 5]).
+uint16_t to_half_bits(double x) {
+    uint16_t sgn = std::signbit(x) ? 0x8000 : 0;
+    x = std::fabs(x);
+    if (x == 0.0)
+        return sgn;
+    int e;
+    const double m = std::frexp(x, &e);          // x = m 2^e, m in [0.5, 1)
+    int E = e - 1 + 15;                           // x = (2m) 2^(e-1)
+    if (E <= 0)
+        return sgn;                               // not reached for codebook values
+    double frac = (2.0 * m - 1.0) * 1024.0;
+    double fl = std::floor(frac);
+    uint32_t f = (uint32_t)fl;
+    const double rem = frac - fl;
+    if (rem > 0.5 || (rem == 0.5 && (f & 1u)))
+        ++f;
+    if (f == 1024) {
+        f = 0;
+        ++E;
+    }
+    if (E >= 31)
+        return (uint16_t)(sgn | 0x7C00);
+    return (uint16_t)(sgn | (E << 10) | f);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------
+// Handles.
+// ---------------------------------------------------------------------------------------
+struct oq_rpbh {
+    int d = 0, h = 0;
+    uint64_t seed = 0;
+    std::vector<int32_t> perm;
+    std::vector<int8_t> sign;
+    std::vector<uint32_t> packed;                 // perm | (sign < 0) << 31
+    std::mutex mu;
+    uint32_t *dev[oq::kMaxDevices] = {};
+};
+
+struct oq_codebook {
+    int d = 0, bits = 0;
+    std::vector<double> c, t;                     // unit centroids / boundaries
+    uint16_t lut[256] = {};                       // unit centroids, fp16 bits
+    int G = 0, F = 0;
+    double delta = 0.0;
+    std::vector<uint32_t> grid;                   // G + 1 words
+    std::mutex mu;
+    uint32_t *dev_grid[oq::kMaxDevices] = {};
+};
+
+namespace {
+
+// Uniform grid over the unit axis with at most one boundary per cell; see include/oq.h.
+bool build_grid(oq_codebook *cb) {
+    const int L = 1 << cb->bits;
+    double gap = std::numeric_limits<double>::infinity(), tmax = 0.0;
+    for (int j = 0; j + 1 < L - 1; ++j)
+        gap = std::min(gap, cb->t[j + 1] - cb->t[j]);
+    for (double v : cb->t)
+        tmax = std::max(tmax, std::fabs(v));
+    if (L - 1 == 1)
+        gap = 2.0 * tmax > 0 ? 2.0 * tmax : 1.0;
+    for (double shrink = 0.999; shrink > 0.1; shrink *= 0.5) {
+        const double delta = gap * shrink;
+        int G = 8;
+        while (G * delta < 2.0 * tmax * 1.001 + 2.0 * delta)
+            G *= 2;
+        if (G > (1 << 20))
+            return false;
+        int lg = 0;
+        while ((1 << lg) < G)
+            ++lg;
+        const int F = 23 - lg;
+        const double two23 = 8388608.0;
+        std::vector<long long> qthr(L - 1), cell(L - 1);
+        bool ok = true;
+        for (int j = 0; j < L - 1; ++j) {
+            const double A = cb->t[j] / (G * delta) + 0.5;
+            qthr[j] = (long long)std::ceil(A * two23);
+            cell[j] = qthr[j] >> F;
+            if (qthr[j] <= 0 || qthr[j] >= (1LL << 23))
+                ok = false;
+            if (j > 0 && cell[j] == cell[j - 1])
+                ok = false;                       // two boundaries in one cell
+        }
+        if (!ok)
+            continue;
+        cb->G = G;
+        cb->F = F;
+        cb->delta = delta;
+        cb->grid.assign(G + 1, 0);
+        for (int k = 0; k <= G; ++k) {
+            long long base = 0, thr = ((long long)k + 1) << F;   // unreachable by default
+            for (int j = 0; j < L - 1; ++j) {
+                if (cell[j] < k)
+                    ++base;
+                else if (cell[j] == k)
+                    thr = qthr[j];
+            }
+            const uint32_t word = (uint32_t)((uint64_t)(base + 1) << 24) -
+                                  (uint32_t)((uint64_t)(thr + 0x3F800000LL) * (uint64_t)G);
+            cb->grid[k] = word;
+        }
+        return true;
+    }
+    return false;
+}
+
+struct DeviceInfo {
+    int checked = 0;       // 0 unknown, 1 ok, -1 unsupported
+    int sms = 0;
+    cudaMemPool_t pool = nullptr;
+};
+DeviceInfo g_dev[oq::kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device(int *dev_out, DeviceInfo **info_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "cudaGetDevice");
+    if (dev < 0 || dev >= oq::kMaxDevices)
+        return fail(OQ_EUNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &di = g_dev[dev];
+    if (di.checked == 0) {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess)
+            return fail_cuda(e, "cudaDeviceGetAttribute");
+        di.checked = (major == 10 && minor == 0) ? 1 : -1;
+        di.sms = sms;
+    }
+    if (di.checked < 0)
+        return fail(OQ_EUNSUPPORTED, "device %d is not sm_100 (B200 class); liboq is built for "
+                                     "sm_100a only", dev);
+    *dev_out = dev;
+    *info_out = &di;
+    return OQ_OK;
+}
+
+template <class T>
+int upload(std::mutex &mu, uint32_t **slot, const std::vector<T> &host, const char *what) {
+    std::lock_guard<std::mutex> lk(mu);
+    if (*slot)
+        return OQ_OK;
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, host.size() * sizeof(T));
+    if (e != cudaSuccess)
+        return fail_cuda(e, what);
+    e = cudaMemcpy(p, host.data(), host.size() * sizeof(T), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return fail_cuda(e, what);
+    }
+    *slot = static_cast<uint32_t *>(p);
+    return OQ_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(int d, const char *who) {
+    if (d < 128 || d > 16384 || d % 128 != 0)
+        return fail(OQ_EINVAL, "%s: d = %d must be a multiple of 128 in [128, 16384]", who, d);
+    return OQ_OK;
+}
+
+int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dtype, int rows,
+                  int d, uint8_t *codes, float *norms, void *stream, float eps,
+                  const char *who) {
+    if (!r || !cb)
+        return fail(OQ_EINVAL, "%s: null handle", who);
+    if (check_dims(d, who) != OQ_OK)
+        return OQ_EINVAL;
+    if (r->d != d || cb->d != d)
+        return fail(OQ_EINVAL, "%s: d = %d but rotation has d = %d and codebook d = %d", who, d,
+                    r->d, cb->d);
+    if (dtype != OQ_F32 && dtype != OQ_BF16)
+        return fail(OQ_EINVAL, "%s: dtype must be OQ_F32 or OQ_BF16", who);
+    if (rows < 0)
+        return fail(OQ_EINVAL, "%s: negative row count %d", who, rows);
+    if (rows == 0)
+        return OQ_OK;
+    if (!x || !codes || !norms)
+        return fail(OQ_EINVAL, "%s: null data pointer", who);
+    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(norms) & 3u))
+        return fail(OQ_EINVAL, "%s: x and codes must be 16-byte aligned, norms 4-byte", who);
+    int dev;
+    DeviceInfo *di;
+    int rc = current_device(&dev, &di);
+    if (rc != OQ_OK)
+        return rc;
+    oq_rpbh *rw = const_cast<oq_rpbh *>(r);
+    oq_codebook *cw = const_cast<oq_codebook *>(cb);
+    if ((rc = upload(rw->mu, &rw->dev[dev], rw->packed, "upload rotation table")) != OQ_OK)
+        return rc;
+    if ((rc = upload(cw->mu, &cw->dev_grid[dev], cw->grid, "upload quantizer table")) != OQ_OK)
+        return rc;
+    oq::K1Params p{};
+    p.x = x;
+    p.codes = codes;
+    p.norms = norms;
+    p.rp = rw->dev[dev];
+    p.grid = cw->dev_grid[dev];
+    p.T = rows;
+    p.d = d;
+    p.eps = eps;
+    p.K = (float)(std::sqrt((double)d / r->h) / (cb->G * cb->delta));
+    p.G = cb->G;
+    p.F = cb->F;
+    std::string why;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = timed(OQ_KERNEL_QUANTIZE, st, [&] {
+        return oq::launch_k1(p, cb->bits, r->h, dtype == OQ_F32, st, di->sms, &why);
+    });
+    if (e != cudaSuccess)
+        return fail_cuda(e, why.c_str());
+    return OQ_OK;
+}
+
+cudaMemPool_t device_pool(int dev, DeviceInfo *di, int *rc) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (di->pool)
+        return di->pool;
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    cudaError_t e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) {
+        *rc = fail_cuda(e, "cudaMemPoolCreate");
+        return nullptr;
+    }
+    uint64_t keep = std::numeric_limits<uint64_t>::max();
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    di->pool = pool;
+    return pool;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------
+// C ABI.
+// ---------------------------------------------------------------------------------------
+extern "C" {
+
+int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out) {
+    if (!out)
+        return fail(OQ_EINVAL, "oq_build_rpbh: out is NULL");
+    *out = nullptr;
+    if (check_dims(d, "oq_build_rpbh") != OQ_OK)
+        return OQ_EINVAL;
+    if (h < 32 || h > 1024 || (h & (h - 1)) != 0 || d % h != 0)
+        return fail(OQ_EINVAL, "oq_build_rpbh: h = %d must be a power of two in [32, 1024] "
+                               "dividing d = %d", h, d);
+    oq_rpbh *r = new (std::nothrow) oq_rpbh;
+    if (!r)
+        return fail(OQ_ENOMEM, "oq_build_rpbh: out of host memory");
+    r->d = d;
+    r->h = h;
+    r->seed = seed;
+    r->perm.resize(d);
+    r->sign.resize(d);
+    r->packed.resize(d);
+    SplitMix64 g{seed};
+    for (int i = 0; i < d; ++i)
+        r->perm[i] = i;
+    for (int i = d - 1; i > 0; --i) {
+        const int j = (int)g.below((uint64_t)i + 1);
+        std::swap(r->perm[i], r->perm[j]);
+    }
+    for (int k = 0; k < d; ++k)
+        r->sign[k] = (g.next() >> 63) ? -1 : 1;
+    for (int k = 0; k < d; ++k)
+        r->packed[k] = (uint32_t)r->perm[k] | (r->sign[k] < 0 ? 0x80000000u : 0u);
+    *out = r;
+    return OQ_OK;
+}
+
+int oq_rpbh_tables(const oq_rpbh *r, int32_t *perm_out, int8_t *sign_out) {
+    if (!r)
+        return fail(OQ_EINVAL, "oq_rpbh_tables: null handle");
+    if (perm_out)
+        std::memcpy(perm_out, r->perm.data(), sizeof(int32_t) * r->d);
+    if (sign_out)
+        std::memcpy(sign_out, r->sign.data(), r->d);
+    return OQ_OK;
+}
+
+int oq_lloyd_max(int d, int bits, oq_codebook **out) {
+    if (!out)
+        return fail(OQ_EINVAL, "oq_lloyd_max: out is NULL");
+    *out = nullptr;
+    if (d < 1)
+        return fail(OQ_EINVAL, "oq_lloyd_max: d = %d", d);
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
+        return fail(OQ_EINVAL, "oq_lloyd_max: bits = %d not in {2, 3, 4, 8}", bits);
+    oq_codebook *cb = new (std::nothrow) oq_codebook;
+    if (!cb)
+        return fail(OQ_ENOMEM, "oq_lloyd_max: out of host memory");
+    cb->d = d;
+    cb->bits = bits;
+    const int L = 1 << bits;
+    if (!solve_lloyd_max(L, cb->c)) {
+        delete cb;
+        return fail(OQ_EINVAL, "oq_lloyd_max: solver did not converge for %d levels", L);
+    }
+    cb->t.resize(L - 1);
+    for (int j = 0; j < L - 1; ++j)
+        cb->t[j] = 0.5 * (cb->c[j] + cb->c[j + 1]);
+    for (int i = 0; i < L; ++i)
+        cb->lut[i] = to_half_bits(cb->c[i]);
+    if (!build_grid(cb)) {
+        delete cb;
+        return fail(OQ_EINVAL, "oq_lloyd_max: could not build the quantizer grid");
+    }
+    *out = cb;
+    return OQ_OK;
+}
+
+int oq_codebook_values(const oq_codebook *cb, double *centroids, double *bounds) {
+    if (!cb)
+        return fail(OQ_EINVAL, "oq_codebook_values: null handle");
+    const double sigma = 1.0 / std::sqrt((double)cb->d);
+    const int L = 1 << cb->bits;
+    if (centroids)
+        for (int i = 0; i < L; ++i)
+            centroids[i] = sigma * cb->c[i];
+    if (bounds)
+        for (int j = 0; j < L - 1; ++j)
+            bounds[j] = sigma * cb->t[j];
+    return OQ_OK;
+}
+
+int oq_codebook_grid(const oq_codebook *cb, int *grid_cells, double *delta, uint32_t *table) {
+    if (!cb)
+        return fail(OQ_EINVAL, "oq_codebook_grid: null handle");
+    if (grid_cells)
+        *grid_cells = cb->G;
+    if (delta)
+        *delta = cb->delta;
+    if (table)
+        std::memcpy(table, cb->grid.data(), sizeof(uint32_t) * cb->grid.size());
+    return OQ_OK;
+}
+
+int oq_quantize_weight(const oq_rpbh *r, const oq_codebook *cw, const void *W, int dtype,
+                       int out_features, int d, uint8_t *W_codes, float *row_norms,
+                       void *stream) {
+    return quantize_rows(r, cw, W, dtype, out_features, d, W_codes, row_norms, stream, 0.0f,
+                         "oq_quantize_weight");
+}
+
+int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype, int T,
+                    int d, uint8_t *x_codes, float *s, void *stream) {
+    return quantize_rows(r, ca, x, dtype, T, d, x_codes, s, stream, 1e-8f, "oq_quantize_act");
+}
+
+int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
+              const float *s, const uint8_t *W_codes, const float *row_norms, int T, int d,
+              int out_features, void *y, int out_dtype, void *stream) {
+    const char *who = "oq_linear";
+    if (!ca || !cw)
+        return fail(OQ_EINVAL, "%s: null codebook", who);
+    if (check_dims(d, who) != OQ_OK)
+        return OQ_EINVAL;
+    if (ca->d != d || cw->d != d)
+        return fail(OQ_EINVAL, "%s: d = %d but codebooks have d = %d / %d", who, d, ca->d,
+                    cw->d);
+    if (out_dtype != OQ_F32)
+        return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32", who);
+    if (T < 0 || out_features < 1 || out_features % 16 != 0)
+        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
+                               "multiple of 16", who, T, out_features);
+    if (T == 0)
+        return OQ_OK;
+    if (!x_codes || !s || !W_codes || !row_norms || !y)
+        return fail(OQ_EINVAL, "%s: null data pointer", who);
+    if (!aligned16(x_codes) || !aligned16(W_codes) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(s) & 3u) || (reinterpret_cast<uintptr_t>(row_norms) & 3u))
+        return fail(OQ_EINVAL, "%s: codes and y must be 16-byte aligned, s/row_norms 4-byte",
+                    who);
+    int dev;
+    DeviceInfo *di;
+    int rc = current_device(&dev, &di);
+    if (rc != OQ_OK)
+        return rc;
+    cudaMemPool_t pool = device_pool(dev, di, &rc);
+    if (!pool)
+        return rc;
+    const size_t ws_bytes = oq::linear_workspace_bytes(T, d, out_features);
+    void *ws = nullptr;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, ws_bytes, pool, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "oq_linear: workspace allocation");
+    uint16_t *A16 = static_cast<uint16_t *>(ws);
+    uint16_t *B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
+                                                 oq::linear_workspace_b_offset(T, d));
+    std::string why;
+    e = timed(OQ_KERNEL_DECODE, st, [&] {
+        return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
+    });
+    if (e == cudaSuccess)
+        e = timed(OQ_KERNEL_DECODE, st, [&] {
+            return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
+                                     di->sms, &why);
+        });
+    if (e == cudaSuccess)
+        e = timed(OQ_KERNEL_GEMM, st, [&] {
+            return oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T,
+                                   out_features, d, st, &why);
+        });
+    cudaError_t e2 = cudaFreeAsync(ws, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, why.c_str());
+    if (e2 != cudaSuccess)
+        return fail_cuda(e2, "oq_linear: workspace release");
+    return OQ_OK;
+}
+
+int oq_check(void *stream) {
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "oq_check: stream synchronize");
+    unsigned w1 = 0, w2 = 0;
+    if ((e = oq::read_and_clear_k1_error(&w1, st)) != cudaSuccess)
+        return fail_cuda(e, "oq_check: read k1 error word");
+    if ((e = oq::read_and_clear_k2_error(&w2, st)) != cudaSuccess)
+        return fail_cuda(e, "oq_check: read k2 error word");
+    if (w1 || w2)
+        return fail(OQ_EDEVICE, "device error word: quantize=0x%x linear=0x%x (linear bits: "
+                                "1 = TMA stage wait, 2 = slot-release wait, 4 = accumulator "
+                                "wait gave up)", w1, w2);
+    return OQ_OK;
+}
+
+void oq_free_rpbh(oq_rpbh *r) {
+    if (!r)
+        return;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    for (int dev = 0; dev < oq::kMaxDevices; ++dev)
+        if (r->dev[dev]) {
+            cudaSetDevice(dev);
+            cudaFree(r->dev[dev]);
+        }
+    if (cur >= 0)
+        cudaSetDevice(cur);
+    delete r;
+}
+
+void oq_free_codebook(oq_codebook *cb) {
+    if (!cb)
+        return;
+    int cur = -1;
+    cudaGetDevice(&cur);
+    for (int dev = 0; dev < oq::kMaxDevices; ++dev)
+        if (cb->dev_grid[dev]) {
+            cudaSetDevice(dev);
+            cudaFree(cb->dev_grid[dev]);
+        }
+    if (cur >= 0)
+        cudaSetDevice(cur);
+    delete cb;
+}
+
+int oq_timing_enable(int on) {
+    g_timing = on != 0;
+    return OQ_OK;
+}
+
+int oq_timing_collect(oq_timing_record *out, int capacity, int *count) {
+    if (count)
+        *count = 0;
+    if (capacity < 0 || (capacity > 0 && !out))
+        return fail(OQ_EINVAL, "oq_timing_collect: bad output buffer");
+    int n = 0;
+    cudaError_t err = cudaSuccess;
+    for (const TimedLaunch &t : g_timed) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(t.stop);
+        if (e == cudaSuccess)
+            e = cudaEventElapsedTime(&ms, t.start, t.stop);
+        if (e != cudaSuccess && err == cudaSuccess)
+            err = e;
+        if (n < capacity) {
+            out[n].kernel = t.kernel;
+            out[n].ms = ms;
+        }
+        ++n;
+        g_event_pool.push_back(t.start);
+        g_event_pool.push_back(t.stop);
+    }
+    g_timed.clear();
+    if (count)
+        *count = n < capacity ? n : capacity;
+    if (err != cudaSuccess)
+        return fail_cuda(err, "oq_timing_collect");
+    return OQ_OK;
+}
+
+const char *oq_last_error(void) { return g_last_error.c_str(); }
+
+const char *oq_version(void) { return "liboq 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

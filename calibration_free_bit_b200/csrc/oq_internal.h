@@ -1,0 +1,54 @@
+// oq_internal.h -- internal types shared by liboq's host code and its CUDA kernels.
+// Not part of the public ABI (include/oq.h is).
+#pragma once
+
+#include <cstdint>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "oq.h"
+
+namespace oq {
+
+constexpr int kMaxDevices = 32;
+
+// Parameters of the fused rotate + norm + quantize kernel (K1).
+struct K1Params {
+    const void *x;          // [T, d] rows, fp32 or bf16
+    uint8_t *codes;         // [T, d*bits/8]
+    float *norms;           // [T]
+    const uint32_t *rp;     // [d] perm[p] | (sign[p] < 0) << 31
+    const uint32_t *grid;   // [G + 1] quantizer table words
+    int T, d;
+    float eps;              // added to the norm before division (0 for weights)
+    float K;                // sqrt(d/h) / (G * delta): z_unnormalised * K / (s+eps) = u/(G delta)
+    int G, F;               // grid cells (power of two), F = 23 - log2(G)
+    int groups;             // token pairs processed at once per CTA
+};
+
+// Launch K1 for (bits, h, dtype); `num_sms` sizes the grid.
+cudaError_t launch_k1(const K1Params &p, int bits, int h, int in_f32, cudaStream_t st,
+                      int num_sms, std::string *why);
+
+// Codebook linear layer: decode prepass (codes -> fp16 unit centroids) + tcgen05 GEMM.
+// Workspace layout: A16 [T, d] fp16 at offset 0, B16 [N, d] fp16 at linear_workspace_b_offset.
+size_t linear_workspace_bytes(int T, int d, int N);
+size_t linear_workspace_b_offset(int T, int d);
+
+cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long long rows, int d,
+                          const uint16_t *lut, cudaStream_t st, int num_sms, std::string *why);
+
+// y[T, N] = (s_t rn_o / d) * A16[T, d] . B16[N, d]^T   (fp16 x fp16 -> fp32 in TMEM)
+cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s,
+                        const float *rn, float *y, int T, int N, int d, cudaStream_t st,
+                        std::string *why);
+
+// Device error words written by the kernels (bounded waits that gave up etc.):
+// read-and-clear on the current device.
+cudaError_t read_and_clear_k1_error(unsigned *out, cudaStream_t st);
+cudaError_t read_and_clear_k2_error(unsigned *out, cudaStream_t st);
+
+}  // namespace oq

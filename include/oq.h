@@ -1,0 +1,158 @@
+/*
+ * oq.h -- C ABI of liboq, the B200 (sm_100a) OrbitQuant online quantized-linear path.
+ *
+ * The method is the one summarised on rcap.io, "OrbitQuant: Data-Agnostic Quantization for
+ * Image and Video" [RCAP]: rotate every activation row x (dimension d) with a Randomized
+ * Permuted Block-Hadamard (RPBH) rotation R, take its norm s, encode each rotated coordinate
+ * as a b-bit nearest-centroid code of one Lloyd-Max codebook built offline for the fixed
+ * N(0, 1/d) marginal, and multiply against weights stored the same way (row norms times codes
+ * of W R^T).  Since R is orthogonal, W R^T R x = W x and the rotation cancels inside the
+ * layer.
+ *
+ * Conventions shared by every call
+ *   - Return value: OQ_OK (0) or a negative OQ_E* status.  On failure nothing was launched,
+ *     and oq_last_error() returns a thread-local message.
+ *   - Data buffers are owned by the caller.  Pointers named "device" must be CUDA device
+ *     pointers on the current device, 16-byte aligned.  Host pointers are plain memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Launches
+ *     are asynchronous on it; a fault inside a kernel is reported by oq_check() or by the
+ *     next synchronising CUDA call.
+ *   - Handles (oq_rpbh, oq_codebook) are immutable once built, may be shared by several
+ *     streams and threads, and are freed with oq_free_*.  Their first use on a device copies
+ *     small tables to that device synchronously; make that first use outside any CUDA graph
+ *     capture.
+ *   - Sizes: d is a multiple of 128 and of h, 128 <= d <= 16384; h is a power of two,
+ *     32 <= h <= 1024; bits in {2, 3, 4, 8}; 0 <= T < 2^31 rows (T = 0 is a no-op returning
+ *     OQ_OK); the linear layer also needs 1 <= out_features < 2^31.
+ *   - Packed codes: row-major, one row per token (or weight row), row stride d*bits/8 bytes,
+ *     element k of a row in bits [k*bits, k*bits + bits) of the row's byte stream, bit i of
+ *     the stream being bit (i mod 8) of byte i/8 (LSB first).  Code 0 is the most negative
+ *     centroid.
+ */
+#ifndef OQ_H
+#define OQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define OQ_OK 0
+#define OQ_EINVAL (-1)        /* bad argument: size, alignment, null pointer, bit width   */
+#define OQ_EUNSUPPORTED (-2)  /* current device is not sm_100 (B200-class)                 */
+#define OQ_ECUDA (-3)         /* a CUDA runtime/driver call failed                         */
+#define OQ_EDEVICE (-4)       /* a kernel reported an internal error (see oq_check)        */
+#define OQ_ENOMEM (-5)        /* host allocation failed                                    */
+
+#define OQ_F32 0              /* element types for `dtype` / `out_dtype`                  */
+#define OQ_BF16 1
+
+typedef struct oq_rpbh oq_rpbh;
+typedef struct oq_codebook oq_codebook;
+
+/* Build the RPBH rotation of dimension d with Hadamard blocks of size h from `seed`.
+ * [RCAP] RPBH paragraph (uniform random permutation, random sign flips, block-diagonal
+ * Walsh-Hadamard blocks) and pseudocode build_rpbh(d).  Definition used here: SplitMix64
+ * seeded with `seed` draws a Fisher-Yates (Durstenfeld) permutation perm[d] (j = r mod (i+1)
+ * for i = d-1..1, rejecting r >= 2^64 - (2^64 mod (i+1))), then sign[k] for k = 0..d-1 from
+ * the top bit of each next draw (set = -1).  R x = blockdiag(H_h/sqrt(h)) diag(sign) y with
+ * y[i] = x[perm[i]] and Sylvester H_h[i][j] = (-1)^popcount(i & j).
+ * Host-only; no GPU needed.  *out receives a new handle (free with oq_free_rpbh).
+ * Errors: OQ_EINVAL for d, h outside the limits above or out == NULL. */
+int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out);
+
+/* Copy the handle's tables to host memory: perm_out[d] (int32), sign_out[d] (+1/-1).
+ * Either pointer may be NULL.  Host-only. */
+int oq_rpbh_tables(const oq_rpbh *r, int32_t *perm_out, int8_t *sign_out);
+
+/* Build the Lloyd-Max codebook with 2^bits levels for the N(0, 1/d) marginal.
+ * [RCAP] change-of-basis paragraph ("the standard Lloyd-Max quantizer construction" against
+ * the fixed marginal, close to N(0, 1/d) for d > 64) and pseudocode lloyd_max(f_d, b).
+ * The unit (N(0,1)) quantizer is solved in fp64 and scaled by sigma = 1/sqrt(d).
+ * Host-only; no GPU needed.  Errors: OQ_EINVAL for bits not in {2,3,4,8}, d < 1. */
+int oq_lloyd_max(int d, int bits, oq_codebook **out);
+
+/* Copy the codebook to host memory in fp64, sigma-scaled: centroids[2^bits] ascending,
+ * bounds[2^bits - 1] ascending (bounds[j] is the midpoint of centroids j and j+1).
+ * Either pointer may be NULL.  Host-only. */
+int oq_codebook_values(const oq_codebook *cb, double *centroids, double *bounds);
+
+/* Introspection of the fast quantizer table the activation/weight kernel uses (for tests):
+ * grid_cells (G, a power of two), cell width in unit-codebook units (delta), and the G+1
+ * table words (table may be NULL to query G first).  A unit value u maps to
+ * a = sat(u/(G*delta) + 1/2); with q = floor(a * 2^23), word = table[q >> (23 - log2 G)],
+ * code = (word + q*G + 0x3F800000*G) >> 24 in 32-bit unsigned arithmetic.  Host-only. */
+int oq_codebook_grid(const oq_codebook *cb, int *grid_cells, double *delta, uint32_t *table);
+
+/* Offline weight step: [RCAP] pseudocode "W_rot = W @ rotation.T; row_norms = norm(W_rot);
+ * W_hat = diag(row_norms) nearest_centroid(W_rot / row_norms, codebook[d, bw])".
+ * W: device, [out_features, d] row-major of `dtype` (OQ_F32 or OQ_BF16).
+ * W_codes: device, [out_features, d*bw/8] packed codes (bw = cw's bits).
+ * row_norms: device, fp32 [out_features] = ||R w_o|| (fp32 accumulation).
+ * No eps; an all-zero row gives codes 2^bw/2 and norm 0.
+ * Errors: OQ_EINVAL (d mismatch with r/cw, sizes, null or misaligned pointers),
+ * OQ_EUNSUPPORTED, OQ_ECUDA. */
+int oq_quantize_weight(const oq_rpbh *r, const oq_codebook *cw, const void *W, int dtype,
+                       int out_features, int d, uint8_t *W_codes, float *row_norms,
+                       void *stream);
+
+/* Online activation step: [RCAP] pseudocode "x_rot = x @ rotation.T; s = norm(x_rot);
+ * x_hat = s * nearest_centroid(x_rot / (s + eps), codebook[d, ba])", eps = 1e-8.
+ * x: device, [T, d] row-major of `dtype`.  x_codes: device, [T, d*ba/8] packed codes.
+ * s: device, fp32 [T], the per-token norm ("the only input-dependent number at runtime").
+ * A code is the number of sigma-scaled boundaries <= x_rot/(s+eps) (ties go up), decided in
+ * fp32.  An all-zero row gives codes 2^ba/2 and s = 0.
+ * Errors: as oq_quantize_weight. */
+int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype, int T,
+                    int d, uint8_t *x_codes, float *s, void *stream);
+
+/* Codebook linear layer: y[t][o] = s[t] * row_norms[o] * sum_k ca[x_codes[t][k]] *
+ * cw[W_codes[o][k]] with sigma-scaled centroids, i.e. x_hat . w_hat in the rotated basis,
+ * which equals the quantized W x because W R^T R x = W x ([RCAP] rotation-cancellation
+ * paragraph; the fused low-bit GEMM is the speed caveat paragraph's missing piece).
+ * x_codes: device [T, d*ba/8]; s: device fp32 [T]; W_codes: device [out_features, d*bw/8];
+ * row_norms: device fp32 [out_features]; y: device [T, out_features] of out_dtype (OQ_F32).
+ * Centroids enter the tensor cores as fp16 unit-variance values; accumulation is fp32.
+ * Uses stream-ordered temporary device memory (two fp16 operand buffers) from a
+ * library-owned pool.  Errors: as above, plus OQ_ECUDA if the pool allocation fails. */
+int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
+              const float *s, const uint8_t *W_codes, const float *row_norms, int T, int d,
+              int out_features, void *y, int out_dtype, void *stream);
+
+/* Synchronise `stream`, then read and clear the library's device error word.
+ * Returns OQ_OK, OQ_EDEVICE (a kernel gave up a bounded wait or saw an internal
+ * inconsistency; oq_last_error() says which), or OQ_ECUDA. */
+int oq_check(void *stream);
+
+void oq_free_rpbh(oq_rpbh *r);
+void oq_free_codebook(oq_codebook *cb);
+
+/* Per-kernel timing, for profilers and benchmarks (the pages have no counterpart; it only
+ * observes the path).  While enabled on the calling thread, every kernel that oq_quantize_*
+ * and oq_linear launch is bracketed by two CUDA events recorded on the caller's stream.
+ * oq_timing_collect() waits for those events, writes up to `capacity` records in launch
+ * order (kernel id, milliseconds) and forgets all pending records; *count receives the number
+ * written.  Records belong to the device that was current at launch. */
+#define OQ_KERNEL_QUANTIZE 1   /* fused rotate + norm + quantize */
+#define OQ_KERNEL_DECODE 2     /* codes -> fp16 centroid prepass of oq_linear */
+#define OQ_KERNEL_GEMM 3       /* tcgen05 codebook GEMM of oq_linear */
+typedef struct {
+    int kernel;
+    float ms;
+} oq_timing_record;
+int oq_timing_enable(int on);
+int oq_timing_collect(oq_timing_record *out, int capacity, int *count);
+
+/* Thread-local text of the last non-OK status returned on this thread. */
+const char *oq_last_error(void);
+
+/* Library version string. */
+const char *oq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OQ_H */

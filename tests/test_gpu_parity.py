@@ -1,0 +1,281 @@
+"""GPU parity: liboq's sm_100a kernels (through the C ABI) against the fp64 oracle.
+
+Bars (rcap.io OrbitQuant summary, pseudocode block; tolerances from the benchmark spec of
+the method):
+  * packed layout bit-exact (GPU codes re-packed by the oracle reproduce the GPU bytes);
+  * activation / weight codes: >= 99.99% identical, and every mismatch is a neighbour code
+    with the fp64 unit value within 1e-5 sigma of the boundary between them (the kernel decides
+    in fp32; see the design doc for the error budget);
+  * norms s / row_norms: relative error <= 5e-6 (fp32 accumulation over d squares);
+  * oq_linear on identical codes: relative L2 error <= 1e-3 against the fp64 triple loop.
+Inputs are the seeded synthetic workloads of calibration_free_bit_b200.synth; large
+workloads are checked on sampled rows / columns (the oracle computes those one by one) and
+on properties that hold at any size (norm preservation, code range).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from calibration_free_bit_b200 import build as B
+from calibration_free_bit_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+CODE_MATCH = 0.9999
+BOUNDARY_TOL = 1e-5        # in sigma units (unit-codebook units)
+NORM_RTOL = 5e-6
+LINEAR_RTOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def oq(cuda_device):
+    B.build()
+    from calibration_free_bit_b200 import oq as _oq
+    return _oq
+
+
+_HANDLES = {}
+
+
+def handles(oq, d, h, ba, bw, seed=0):
+    key = (d, h, ba, bw, seed)
+    if key not in _HANDLES:
+        _HANDLES[key] = (oq.oq_build_rpbh(d, h, seed), oq.oq_lloyd_max(d, ba),
+                         oq.oq_lloyd_max(d, bw))
+    return _HANDLES[key]
+
+
+def check_codes(gpu_packed, orc_packed, orc_u, d, bits, what):
+    """Code-parity rule on a block of rows; returns the number of mismatches."""
+    gpu_packed = np.ascontiguousarray(gpu_packed)
+    gcodes = O.unpack(gpu_packed, d, bits)
+    # layout: the oracle's packer reproduces the GPU's bytes exactly
+    assert np.array_equal(O.pack(gcodes, bits), gpu_packed), f"{what}: packed layout"
+    ocodes = O.unpack(orc_packed, d, bits)
+    bad = np.argwhere(gcodes != ocodes)
+    n = gcodes.size
+    assert len(bad) <= (1 - CODE_MATCH) * n + 1e-9, f"{what}: {len(bad)} of {n} codes differ"
+    _, t = O.codebook(bits)
+    for r, k in bad:
+        u = orc_u[r, k]
+        j = int(np.argmin(np.abs(t - u)))
+        assert abs(u - t[j]) <= BOUNDARY_TOL, f"{what}: row {r} col {k} u={u} not near a boundary"
+        assert {int(gcodes[r, k]), int(ocodes[r, k])} == {j, j + 1}, f"{what}: non-adjacent"
+    return len(bad)
+
+
+def k1_gpu(oq, r, cb, x_cpu, weight=False):
+    x = x_cpu.cuda()
+    fn = oq.oq_quantize_weight if weight else oq.oq_quantize_act
+    codes, s = fn(r, cb, x)
+    oq.oq_check()
+    return codes.cpu().numpy(), s.cpu().numpy().astype(np.float64)
+
+
+def k1_oracle(x_cpu, h, bits, weight=False, seed=0):
+    d = x_cpu.shape[1]
+    perm, sign = O.build_rpbh(d, seed)
+    x64 = x_cpu.double().numpy()
+    fn = O.quantize_weight if weight else O.quantize_act
+    return fn(x64, h, perm, sign, bits, detail=True)
+
+
+# ----------------------------------------------------------------------------------------
+# K1: rotate + norm + quantize
+# ----------------------------------------------------------------------------------------
+
+def test_k1_toy_fp32_activations_and_weights(oq):
+    p = synth.get("toy_w4a4")[0]
+    r, ca, cw = handles(oq, p.d, p.h, p.bits_a, p.bits_w)
+    x, W = synth.activations(p), synth.weight(p)
+    g, gs = k1_gpu(oq, r, ca, x)
+    o, os_, _, ou = k1_oracle(x, p.h, p.bits_a)
+    check_codes(g, o, ou, p.d, p.bits_a, "toy x")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+    g, gs = k1_gpu(oq, r, cw, W, weight=True)
+    o, os_, _, ou = k1_oracle(W, p.h, p.bits_w, weight=True)
+    check_codes(g, o, ou, p.d, p.bits_w, "toy W")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+
+
+@pytest.mark.parametrize("h", [32, 64, 128, 256, 512, 1024])
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_k1_every_block_size_and_bit_width(oq, h, bits):
+    d = 2048 if h <= 512 else 3072
+    T = 37                                  # odd: the last token pair has one token
+    p = synth.sweep_projection(d, 128, 4, T)
+    x = synth.activations(p)
+    r = oq.oq_build_rpbh(d, h, 0)
+    cb = oq.oq_lloyd_max(d, bits)
+    g, gs = k1_gpu(oq, r, cb, x)
+    o, os_, _, ou = k1_oracle(x, h, bits)
+    check_codes(g, o, ou, d, bits, f"h={h} b={bits}")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+
+
+def test_k1_flux_attention_full_size(oq):
+    """4608 x 3072 bf16, W4A4, h=128: every row against the oracle."""
+    p = synth.get("flux_attn_w4a4")[0]
+    r, ca, cw = handles(oq, p.d, p.h, p.bits_a, p.bits_w)
+    x = synth.activations(p)
+    g, gs = k1_gpu(oq, r, ca, x)
+    o, os_, _, ou = k1_oracle(x, p.h, p.bits_a)
+    check_codes(g, o, ou, p.d, p.bits_a, "flux attn x")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+    W = synth.weight(p)
+    g, gs = k1_gpu(oq, r, cw, W, weight=True)
+    o, os_, _, ou = k1_oracle(W, p.h, p.bits_w, weight=True)
+    check_codes(g, o, ou, p.d, p.bits_w, "flux attn W")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+
+
+def test_k1_edge_rows(oq):
+    """Zero rows, a single huge outlier, a one-hot row, tiny values, T = 1 and T = 0.
+    (Rows below ~1e-17 would underflow fp32 squares; 1e-15 is still exact in fp32.)"""
+    d, h, bits = 1024, 128, 4
+    r = oq.oq_build_rpbh(d, h, 0)
+    cb = oq.oq_lloyd_max(d, bits)
+    x = torch.zeros((7, d), dtype=torch.bfloat16)
+    x[1, 5] = 1.0
+    x[2] = torch.randn(d, generator=torch.Generator().manual_seed(3)).bfloat16()
+    x[2, 17] = 3.0e4
+    x[3] = 1e-15
+    x[5, :] = -2.0
+    g, gs = k1_gpu(oq, r, cb, x)
+    o, os_, _, ou = k1_oracle(x, h, bits)
+    check_codes(g, o, ou, d, bits, "edge rows")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL, atol=0)
+    assert gs[0] == 0.0 and gs[4] == 0.0 and gs[6] == 0.0
+    assert np.all(O.unpack(g[[0, 4, 6]], d, bits) == 8)
+    # T = 1
+    g1, s1 = k1_gpu(oq, r, cb, x[2:3])
+    assert np.array_equal(g1[0], g[2]) and s1[0] == gs[2]
+    # T = 0 is a no-op
+    codes, s = oq.oq_quantize_act(r, cb, torch.empty((0, d), dtype=torch.bfloat16,
+                                                      device="cuda"))
+    assert codes.shape == (0, d // 2) and s.shape == (0,)
+
+
+def test_k1_max_dimension(oq):
+    """d = 16384 (the sweep's largest), h = 256 and 128, bf16 and fp32 inputs."""
+    p = synth.sweep_projection(16384, 256, 8, 64)
+    x = synth.activations(p)
+    for h, bits, xin in [(256, 8, x), (128, 4, x.float()), (256, 3, x.float())]:
+        r = oq.oq_build_rpbh(16384, h, 0)
+        cb = oq.oq_lloyd_max(16384, bits)
+        g, gs = k1_gpu(oq, r, cb, xin)
+        o, os_, _, ou = k1_oracle(xin, h, bits)
+        check_codes(g, o, ou, 16384, bits, f"d=16384 h={h} b={bits}")
+        np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+
+
+def test_k1_video_ffn_full_size_sampled(oq):
+    """65520 x 13824 bf16 (down projection input, W4A8): all rows on the GPU in the launch
+    configuration the benchmark uses; sampled rows against the oracle, every norm against
+    ||x|| (the rotation preserves norms)."""
+    p = synth.get("video_ffn_w4a8")[1]
+    r, ca, _ = handles(oq, p.d, p.h, p.bits_a, p.bits_w)
+    x = synth.activations(p)
+    xg = x.cuda()
+    codes, s = oq.oq_quantize_act(r, ca, xg)
+    oq.oq_check()
+    norm_ref = np.concatenate([torch.linalg.vector_norm(x[i:i + 4096].double(), dim=1).numpy()
+                               for i in range(0, p.T, 4096)])
+    np.testing.assert_allclose(s.cpu().double().numpy(), norm_ref, rtol=NORM_RTOL)
+    rows = np.array([0, 1, 17, 32759, 32760, 40000, 65519])
+    o, os_, _, ou = k1_oracle(x[rows], p.h, p.bits_a)
+    check_codes(codes[rows].cpu().numpy(), o, ou, p.d, p.bits_a, "video ffn sampled")
+
+
+# ----------------------------------------------------------------------------------------
+# K2: codebook linear layer
+# ----------------------------------------------------------------------------------------
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def linear_gpu(oq, ca, cw, xc, s, wc, rn):
+    dev = "cuda"
+    y = oq.oq_linear(ca, cw, torch.from_numpy(np.ascontiguousarray(xc)).to(dev),
+                     torch.from_numpy(np.asarray(s, np.float32)).to(dev),
+                     torch.from_numpy(np.ascontiguousarray(wc)).to(dev),
+                     torch.from_numpy(np.asarray(rn, np.float32)).to(dev))
+    oq.oq_check()
+    return y.cpu().double().numpy()
+
+
+def test_linear_toy_on_oracle_codes(oq):
+    p = synth.get("toy_w4a4")[0]
+    _, ca, cw = handles(oq, p.d, p.h, p.bits_a, p.bits_w)
+    xc, s, _, _ = k1_oracle(synth.activations(p), p.h, p.bits_a)
+    wc, rn, _, _ = k1_oracle(synth.weight(p), p.h, p.bits_w, weight=True)
+    y = linear_gpu(oq, ca, cw, xc, s, wc, rn)
+    ref = O.linear(xc, s, wc, rn, p.d, p.bits_a, p.bits_w)
+    assert rel_l2(y, ref) <= LINEAR_RTOL
+
+
+@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (4, 3), (8, 4), (2, 8), (8, 8)])
+@pytest.mark.parametrize("T,N,d", [(200, 272, 384), (1, 16, 128), (129, 512, 1024)])
+def test_linear_random_codes_ragged(oq, ba, bw, T, N, d):
+    """Uniform random codes (every centroid used), ragged M and N tails."""
+    rng = np.random.default_rng(T * 7 + N + ba * 100 + bw)
+    xc = O.pack(rng.integers(0, 1 << ba, (T, d)).astype(np.uint8), ba)
+    wc = O.pack(rng.integers(0, 1 << bw, (N, d)).astype(np.uint8), bw)
+    s = rng.uniform(0.1, 50.0, T)
+    rn = rng.uniform(0.5, 2.0, N)
+    ca, cw = oq.oq_lloyd_max(d, ba), oq.oq_lloyd_max(d, bw)
+    y = linear_gpu(oq, ca, cw, xc, s, wc, rn)
+    ref = O.linear(xc, s, wc, rn, d, ba, bw)
+    assert rel_l2(y, ref) <= LINEAR_RTOL
+
+
+def _sampled_linear(oq, p, rows, cols):
+    """Full-size GPU path (K1 on all of x and W, then oq_linear), with the sampled rows of
+    x_codes/s and of W_codes/row_norms replaced by the oracle's, so that the compared
+    outputs y[rows, cols] come from identical codes."""
+    r, ca, cw = handles(oq, p.d, p.h, p.bits_a, p.bits_w)
+    x = synth.activations(p)
+    W = synth.weight(p)
+    xc, s = oq.oq_quantize_act(r, ca, x.cuda())
+    wc, rn = oq.oq_quantize_weight(r, cw, W.cuda())
+    oq.oq_check()
+    oxc, os_, _, ou = k1_oracle(x[rows], p.h, p.bits_a)
+    owc, orn, _, wu = k1_oracle(W[cols], p.h, p.bits_w, weight=True)
+    check_codes(xc[rows].cpu().numpy(), oxc, ou, p.d, p.bits_a, p.name + " x")
+    check_codes(wc[cols].cpu().numpy(), owc, wu, p.d, p.bits_w, p.name + " W")
+    ri, ci = torch.from_numpy(rows).cuda(), torch.from_numpy(cols).cuda()
+    xc[ri] = torch.from_numpy(oxc).cuda()
+    s[ri] = torch.from_numpy(os_.astype(np.float32)).cuda()
+    wc[ci] = torch.from_numpy(owc).cuda()
+    rn[ci] = torch.from_numpy(orn.astype(np.float32)).cuda()
+    y = oq.oq_linear(ca, cw, xc, s, wc, rn)
+    oq.oq_check()
+    got = y[ri][:, ci].cpu().double().numpy()
+    ref = O.linear(oxc, os_, owc, orn, p.d, p.bits_a, p.bits_w)
+    assert rel_l2(got, ref) <= LINEAR_RTOL, rel_l2(got, ref)
+    return y
+
+
+def test_linear_flux_attention_full_size(oq):
+    p = synth.get("flux_attn_w4a4")[0]
+    rows = np.unique(np.concatenate([np.arange(0, 4608, 97), [4607, 4095, 4096]]))
+    cols = np.unique(np.concatenate([np.arange(0, 3072, 41), [3071]]))
+    _sampled_linear(oq, p, rows, cols)
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_linear_flux_mlp_full_size(oq, which):
+    p = synth.get("flux_mlp_w2a4")[which]
+    rows = np.arange(0, p.T, 151)
+    cols = np.arange(3, p.out, 389)
+    _sampled_linear(oq, p, rows, cols)
+
+
+@pytest.mark.parametrize("variant", ["video_ffn_w3a4", "video_ffn_w4a8"])
+def test_linear_video_ffn_up_full_size(oq, variant):
+    p = synth.get(variant)[0]
+    rows = np.array([0, 5, 32759, 32760, 50000, 65408, 65519])
+    cols = np.arange(11, p.out, 977)
+    _sampled_linear(oq, p, rows, cols)

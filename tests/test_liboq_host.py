@@ -1,0 +1,130 @@
+"""liboq host logic on the CPU (no GPU calls): the C ABI loads and exports every symbol of
+include/oq.h; its RPBH tables and Lloyd-Max codebooks (independent codings) agree with the
+oracle; the quantizer grid table, evaluated with the kernel's integer recipe, reproduces the
+oracle's boundary count; argument validation rejects bad input before touching a device.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+
+import oracle as O
+from calibration_free_bit_b200 import build as B
+from calibration_free_bit_b200 import oq
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+
+
+def test_library_exports_every_header_symbol():
+    names = oq.header_functions()
+    assert {"oq_build_rpbh", "oq_lloyd_max", "oq_quantize_weight", "oq_quantize_act",
+            "oq_linear"} <= set(names)
+    L = oq.lib()
+    missing = []
+    for n in names:
+        try:
+            getattr(L, n)
+        except AttributeError:
+            missing.append(n)
+    assert not missing, missing
+    assert oq.version().startswith("liboq")
+
+
+@pytest.mark.parametrize("d,h,seed", [(256, 64, 0), (3072, 128, 0), (13824, 128, 7),
+                                      (16384, 256, 12345), (1024, 32, 2**63 + 5)])
+def test_rpbh_tables_bit_exact_vs_oracle(d, h, seed):
+    perm, sign = oq.oq_build_rpbh(d, h, seed).tables()
+    operm, osign = O.build_rpbh(d, seed)
+    assert np.array_equal(perm, operm)
+    assert np.array_equal(sign, osign)
+
+
+@pytest.mark.parametrize("bits,tol", [(2, 1e-11), (3, 1e-11), (4, 1e-11), (8, 1e-8)])
+def test_codebook_matches_oracle(bits, tol):
+    """Two independent solvers (liboq: Lloyd warm-up + Newton to a residual < 1e-15; oracle:
+    plain Lloyd stopped at a step <= 4e-14).  The oracle's distance to the fixed point is
+    step / (1 - contraction): ~1e-12 at 4 bits (contraction ~0.96) and ~1e-10 at 8 bits
+    (contraction ~1 - 2e-4), hence the tolerances (unit-codebook units)."""
+    d = 3072
+    c, t = oq.oq_lloyd_max(d, bits).values()
+    oc, ot = O.codebook(bits)
+    sig = 1.0 / np.sqrt(d)
+    np.testing.assert_allclose(c, sig * oc, rtol=0, atol=tol * sig)
+    np.testing.assert_allclose(t, sig * ot, rtol=0, atol=tol * sig)
+
+
+def emulate_kernel_codes(u, G, delta, table):
+    """The kernel's code recipe in exact integer arithmetic (documented in include/oq.h):
+    a = sat(u/(G delta) + 1/2) in fp32; q = floor(a 2^23); word = table[q >> (23-log2 G)];
+    code = (word + (0x3F800000 + q) G) mod 2^32 >> 24."""
+    a = np.clip((u / (G * delta) + 0.5).astype(np.float32), 0.0, 1.0).astype(np.float64)
+    q = np.floor(a * 2.0**23).astype(np.int64)
+    F = 23 - int(np.log2(G))
+    word = table[q >> F].astype(np.int64)
+    D = (word + (0x3F800000 + q) * G) % (1 << 32)
+    return (D >> 24).astype(np.int64)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_quantizer_grid_matches_boundary_count(bits):
+    cb = oq.oq_lloyd_max(3072, bits)
+    G, delta, table = cb.grid()
+    assert G & (G - 1) == 0 and len(table) == G + 1
+    _, t = O.codebook(bits)
+    rng = np.random.default_rng(bits)
+    u = np.concatenate([rng.standard_normal(400000) * 1.3,
+                        rng.uniform(-60, 60, 20000),
+                        t, t + 1e-7, t - 1e-7, t + 3e-6, t - 3e-6,
+                        [0.0, -0.0, 1e30, -1e30, 55.4, -55.4]])
+    got = emulate_kernel_codes(u, G, delta, table)
+    want = np.searchsorted(t, u, side="right")
+    bad = np.flatnonzero(got != want)
+    # the fixed-point grid moves a boundary by < 2^-23 of the grid span (< 1.2e-6 sigma)
+    for i in bad:
+        j = np.argmin(np.abs(t - u[i]))
+        assert abs(u[i] - t[j]) < 2e-6, (u[i], got[i], want[i])
+        assert {got[i], want[i]} == {j, j + 1}
+    assert len(bad) <= 8 * len(t)
+
+
+def test_validation_rejects_bad_arguments_without_a_gpu():
+    L = oq.lib()
+    h = C.c_void_p()
+    assert L.oq_build_rpbh(100, 64, 0, C.byref(h)) == oq.OQ_EINVAL
+    assert L.oq_build_rpbh(3072, 48, 0, C.byref(h)) == oq.OQ_EINVAL
+    assert L.oq_build_rpbh(3072, 2048, 0, C.byref(h)) == oq.OQ_EINVAL
+    assert L.oq_build_rpbh(3072, 16, 0, C.byref(h)) == oq.OQ_EINVAL
+    assert L.oq_build_rpbh(32768, 128, 0, C.byref(h)) == oq.OQ_EINVAL
+    assert L.oq_lloyd_max(3072, 5, C.byref(h)) == oq.OQ_EINVAL
+    assert b"bits" in L.oq_last_error()
+    r = oq.oq_build_rpbh(3072, 128)
+    ca = oq.oq_lloyd_max(3072, 4)
+    c_other = oq.oq_lloyd_max(1024, 4)
+    fake = 1 << 20        # never dereferenced: validation fails first
+    # d mismatch between rotation and codebook
+    assert L.oq_quantize_act(r.handle, c_other.handle, fake, oq.OQ_BF16, 8, 3072, fake, fake,
+                             None) == oq.OQ_EINVAL
+    # bad dtype, negative T, null pointers, misalignment
+    assert L.oq_quantize_act(r.handle, ca.handle, fake, 7, 8, 3072, fake, fake,
+                             None) == oq.OQ_EINVAL
+    assert L.oq_quantize_act(r.handle, ca.handle, fake, oq.OQ_BF16, -1, 3072, fake, fake,
+                             None) == oq.OQ_EINVAL
+    assert L.oq_quantize_act(r.handle, ca.handle, None, oq.OQ_BF16, 8, 3072, fake, fake,
+                             None) == oq.OQ_EINVAL
+    assert L.oq_quantize_act(r.handle, ca.handle, fake + 2, oq.OQ_BF16, 8, 3072, fake, fake,
+                             None) == oq.OQ_EINVAL
+    # T = 0 is a no-op that succeeds without touching a device
+    assert L.oq_quantize_act(r.handle, ca.handle, None, oq.OQ_BF16, 0, 3072, None, None,
+                             None) == oq.OQ_OK
+    # linear: out_features not a multiple of 16, bf16 output, d mismatch
+    assert L.oq_linear(ca.handle, ca.handle, fake, fake, fake, fake, 8, 3072, 100, fake,
+                       oq.OQ_F32, None) == oq.OQ_EINVAL
+    assert L.oq_linear(ca.handle, ca.handle, fake, fake, fake, fake, 8, 3072, 128, fake,
+                       oq.OQ_BF16, None) == oq.OQ_EINVAL
+    assert L.oq_linear(ca.handle, c_other.handle, fake, fake, fake, fake, 8, 3072, 128, fake,
+                       oq.OQ_F32, None) == oq.OQ_EINVAL
+    assert L.oq_linear(ca.handle, ca.handle, None, None, None, None, 0, 3072, 128, None,
+                       oq.OQ_F32, None) == oq.OQ_OK
