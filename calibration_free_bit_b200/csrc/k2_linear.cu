@@ -26,6 +26,13 @@ namespace {
 
 __device__ unsigned int g_k2_err;
 
+// Fixed workspace for oq_linear_noalloc: the fp16 operand buffers live here instead of in
+// memory the library allocates.  Every GPU that loads the library holds this array until the
+// process exits.  Host code must not use the symbol as an address (it is a host-side stand-in);
+// noalloc_workspace() looks the device address up once per device.
+constexpr size_t kNoAllocWorkspaceBytes = 64ull << 20;
+static __device__ __align__(256) unsigned char g_noalloc_workspace[kNoAllocWorkspaceBytes];
+
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_STAGE_BYTES = BM * BK * 2;               // 16 KB
 constexpr int B_STAGE_BYTES = BN * BK * 2;               // 32 KB
@@ -436,6 +443,29 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s
     if (e != cudaSuccess)
         *why = "k2_gemm launch";
     return e;
+}
+
+size_t noalloc_workspace_bytes() { return kNoAllocWorkspaceBytes; }
+
+cudaError_t noalloc_workspace(void **out) {
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_workspace);   // the current device's copy
+        if (e != cudaSuccess)
+            return e;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
 }
 
 cudaError_t read_and_clear_k2_error(unsigned *out, cudaStream_t st) {

@@ -613,6 +613,63 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     return OQ_OK;
 }
 
+int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
+                      const float *s, const uint8_t *W_codes, const float *row_norms, int T,
+                      int d, int out_features, void *y, int out_dtype, void *stream) {
+    const char *who = "oq_linear_noalloc";
+    if (!ca || !cw)
+        return fail(OQ_EINVAL, "%s: null codebook", who);
+    if (check_dims(d, who) != OQ_OK)
+        return OQ_EINVAL;
+    if (ca->d != d || cw->d != d)
+        return fail(OQ_EINVAL, "%s: d = %d but codebooks have d = %d / %d", who, d, ca->d,
+                    cw->d);
+    if (out_dtype != OQ_F32)
+        return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32", who);
+    if (T < 0 || out_features < 1 || out_features % 16 != 0)
+        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
+                               "multiple of 16", who, T, out_features);
+    const size_t need = oq::linear_workspace_bytes(T, d, out_features);
+    const size_t have = oq::noalloc_workspace_bytes();
+    if (need > have)
+        return fail(OQ_EINVAL, "%s: T = %d, d = %d, out_features = %d need %zu bytes of "
+                               "workspace, more than the fixed %zu bytes "
+                               "(OQ_NOALLOC_WORKSPACE_BYTES); use oq_linear or split T", who,
+                    T, d, out_features, need, have);
+    if (T == 0)
+        return OQ_OK;
+    if (!x_codes || !s || !W_codes || !row_norms || !y)
+        return fail(OQ_EINVAL, "%s: null data pointer", who);
+    if (!aligned16(x_codes) || !aligned16(W_codes) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(s) & 3u) || (reinterpret_cast<uintptr_t>(row_norms) & 3u))
+        return fail(OQ_EINVAL, "%s: codes and y must be 16-byte aligned, s/row_norms 4-byte",
+                    who);
+    int dev;
+    DeviceInfo *di;
+    int rc = current_device(&dev, &di);
+    if (rc != OQ_OK)
+        return rc;
+    void *ws = nullptr;
+    cudaError_t e = oq::noalloc_workspace(&ws);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "oq_linear_noalloc: workspace address lookup");
+    cudaStream_t st = (cudaStream_t)stream;
+    uint16_t *A16 = static_cast<uint16_t *>(ws);
+    uint16_t *B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
+                                                 oq::linear_workspace_b_offset(T, d));
+    std::string why;
+    e = oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
+    if (e == cudaSuccess)
+        e = oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st, di->sms,
+                              &why);
+    if (e == cudaSuccess)
+        e = oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T, out_features,
+                            d, st, &why);
+    if (e != cudaSuccess)
+        return fail_cuda(e, why.c_str());
+    return OQ_OK;
+}
+
 int oq_check(void *stream) {
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaStreamSynchronize(st);

@@ -46,6 +46,11 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s
                         const float *rn, float *y, int T, int N, int d, cudaStream_t st,
                         std::string *why);
 
+// Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
+// its size, and its address on the current device (looked up once per device).
+size_t noalloc_workspace_bytes();
+cudaError_t noalloc_workspace(void **out);
+
 // Device error words written by the kernels (bounded waits that gave up etc.):
 // read-and-clear on the current device.
 cudaError_t read_and_clear_k1_error(unsigned *out, cudaStream_t st);

@@ -52,6 +52,7 @@ def lib():
     L.oq_quantize_weight.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.oq_quantize_act.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.oq_linear.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp]
+    L.oq_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp]
     L.oq_check.argtypes = [vp]
     L.oq_free_rpbh.argtypes = [vp]
     L.oq_free_rpbh.restype = None
@@ -63,7 +64,7 @@ def lib():
     L.oq_version.restype = C.c_char_p
     for name in ("oq_build_rpbh", "oq_rpbh_tables", "oq_lloyd_max", "oq_codebook_values",
                  "oq_codebook_grid", "oq_quantize_weight", "oq_quantize_act", "oq_linear",
-                 "oq_check", "oq_timing_enable", "oq_timing_collect"):
+                 "oq_linear_noalloc", "oq_check", "oq_timing_enable", "oq_timing_collect"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -206,6 +207,17 @@ def oq_linear(ca: Codebook, cw: Codebook, x_codes: torch.Tensor, s: torch.Tensor
         y = torch.empty((T, N), dtype=torch.float32, device=x_codes.device)
     _check(lib().oq_linear(ca.handle, cw.handle, _ptr(x_codes), _ptr(s), _ptr(W_codes),
                            _ptr(row_norms), T, d, N, _ptr(y), OQ_F32, _stream(stream)))
+    return y
+
+
+def oq_linear_noalloc(ca: Codebook, cw: Codebook, x_codes: torch.Tensor, s: torch.Tensor,
+                      W_codes: torch.Tensor, row_norms: torch.Tensor, y: torch.Tensor,
+                      stream=None):
+    """oq_linear with the library's fixed workspace: the caller passes y; nothing is
+    allocated on the device (see include/oq.h for the size limit and sharing rules)."""
+    T, N, d = x_codes.shape[0], W_codes.shape[0], ca.d
+    _check(lib().oq_linear_noalloc(ca.handle, cw.handle, _ptr(x_codes), _ptr(s), _ptr(W_codes),
+                                   _ptr(row_norms), T, d, N, _ptr(y), OQ_F32, _stream(stream)))
     return y
 
 

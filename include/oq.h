@@ -121,6 +121,30 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
               const float *s, const uint8_t *W_codes, const float *row_norms, int T, int d,
               int out_features, void *y, int out_dtype, void *stream);
 
+/* oq_linear for callers that cannot allocate device memory.  The paper has no counterpart;
+ * this is a deployment variant of the same computation, with the same arguments, result and
+ * errors as oq_linear.
+ * Who needs it: code that runs inside a host framework which owns all device memory and gives
+ * plug-ins no allocator (a side cudaMalloc would bypass its accounting or fail under its
+ * memory cap), and latency-critical serving loops that forbid allocation on the request path
+ * because cudaMalloc/cudaFree can synchronise the device and stall other streams.
+ * How: the two fp16 operand buffers live in a fixed array compiled into the library
+ * (OQ_NOALLOC_WORKSPACE_BYTES = 64 MiB), which every GPU that loads the library holds until
+ * the process exits.  The call allocates and frees nothing.
+ * Limit: 2*(T*d + out_features*d) bytes, each part rounded up to 1 KiB, must fit in
+ * OQ_NOALLOC_WORKSPACE_BYTES (e.g. T = 4608, d = out_features = 3072 needs 47 MB); larger
+ * calls return OQ_EINVAL with the sizes in oq_last_error(), before touching the device.
+ * Set-up: the first call on each device looks up the array's device address once (it may
+ * load the library's kernels on that device); make that first call before any stream capture.
+ * Sharing: every call uses the same array and it keeps the last call's contents; nothing in it
+ * needs to start at zero because each call overwrites the parts it reads.  Calls that can run
+ * at the same time on the GPU (different streams, or threads without ordering between them)
+ * race on the array: order them on one stream or with events. */
+#define OQ_NOALLOC_WORKSPACE_BYTES (64u << 20)
+int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
+                      const float *s, const uint8_t *W_codes, const float *row_norms, int T,
+                      int d, int out_features, void *y, int out_dtype, void *stream);
+
 /* Synchronise `stream`, then read and clear the library's device error word.
  * Returns OQ_OK, OQ_EDEVICE (a kernel gave up a bounded wait or saw an internal
  * inconsistency; oq_last_error() says which), or OQ_ECUDA. */
