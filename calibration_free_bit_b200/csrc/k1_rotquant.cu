@@ -7,13 +7,17 @@
 // the RPBH rotation of the summary's RPBH paragraph, applied as an O(d log h) butterfly.
 //
 // B200 design (one HBM-bound pass: read 2d bytes per bf16 row, write d*b/8 + 4):
-//   * A CTA holds `groups` token PAIRS.  Each pair is staged in shared memory interleaved:
-//     32-bit word j = (x_t0[j], x_t1[j]) as two bf16, so one 4-byte gather load serves both
-//     tokens and the butterfly runs on packed fp32x2 (add/sub/fma .f32x2, new on sm_100).
-//   * A group of d/32 threads owns one pair; thread g holds 32 consecutive rotated positions
-//     of one h-block (h/32 threads per block).  The gather offsets and signs (byte offset of
-//     perm[i] in the pair buffer | sign << 31) are converted once per CTA into a shared table
-//     and read back with 16-byte loads.
+//   * Persistent CTAs, each with `groups` thread groups of d/32 threads; a group owns one
+//     token PAIR per round.  The pair's two rows stream into shared memory with bulk copies
+//     (cp.async.bulk, mbarrier completion, no multicast) one round ahead of the compute.
+//   * bf16 rows are interleaved into 32-bit words (x_t0[j], x_t1[j]), so one 4-byte gather
+//     load serves both tokens and the butterfly runs on packed fp32x2 (add/sub/fma .f32x2,
+//     new on sm_100).  The low and high halves of each 8-element chunk go to separate
+//     regions, so the interleave stores of consecutive threads are contiguous.
+//   * Thread g holds the 32 consecutive rotated positions g*32 .. g*32+31 (h/32 threads per
+//     h-block).  Its gather offsets and signs (pair-buffer byte offset of perm[i] | sign<<31)
+//     are converted once per CTA into a shared table, padded to 36 words per thread so the
+//     16-byte entry loads of a warp are bank-conflict free.
 //   * Butterfly: 5 in-register stages, then log2(h/32) shuffle stages across the block's
 //     threads.  The per-token sum of squares is reduced across the group (segmented warp
 //     shuffles + shared memory); s = sqrt(sum z^2 / h) since z is unnormalised.
@@ -22,6 +26,8 @@
 //     round-down, word = table[q >> F], code = (word + q*G) >> 24.  The table words fold the
 //     cell's base code and its boundary, so the decision is exact in the fixed-point q grid
 //     (2^-23 of the grid span, < 1.2e-6 sigma).  Bit widths 2/3/4/8 pack LSB-first.
+//   * Every mbarrier wait is bounded (2 s of %globaltimer); a wait that gives up sets a bit
+//     in the device error word (read by oq_check) and the round's outputs are not written.
 #include <cuda_bf16.h>
 
 #include "oq_internal.h"
@@ -31,8 +37,11 @@ namespace {
 
 __device__ unsigned int g_k1_err;
 
-constexpr int kE = 32;          // rotated positions per thread (per token)
-constexpr int kMaxSeg = 18;     // segment slots per group for the norm reduction
+constexpr int kE = 32;                // rotated positions per thread (per token)
+constexpr int kMaxSeg = 18;           // segment slots per group for the norm reduction
+constexpr int kEntStride = kE + 4;    // padded per-thread entry rows (conflict-free loads)
+
+enum : unsigned { K1_ERR_COPY_WAIT = 1u };
 
 __device__ __forceinline__ float2 f2add(float2 a, float2 b) {
     float2 c;
@@ -78,22 +87,9 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
     return d;
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    return v;
-}
-
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
     return v;
 }
 
@@ -105,6 +101,53 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+// Wait for the phase of the given parity; false after 2 s (the caller records an error).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer();
+    for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+        if (done)
+            return true;
+        if (globaltimer() - t0 > 2000000000ull)
+            return false;
+    }
+}
+
+// One-dimensional bulk copy global -> shared, completion counted on `bar` (no multicast).
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+// Pair-buffer word of source element j (bf16 path): the low and high halves of every
+// 8-element chunk live in separate regions, so the interleave stores of consecutive threads
+// are contiguous 16-byte runs.
+__device__ __forceinline__ uint32_t pair_word(uint32_t j, uint32_t d) {
+    return (j & 4u) ? (d / 2 + (j >> 3) * 4 + (j & 3u)) : ((j >> 3) * 4 + (j & 3u));
 }
 
 // Store `NWORDS` 32-bit words of packed codes; alignment follows from the chunk size.
@@ -125,18 +168,23 @@ __device__ __forceinline__ void store_words(uint8_t *dst, const uint32_t (&w)[NW
     }
 }
 
+// Per CTA: NG groups of d/32 threads, each group owns one token pair per round.  bf16 input:
+// the NEXT round's two rows stream into a raw buffer while the current round computes from
+// the interleaved pair buffer.  fp32 input: rows are gathered straight from `stages` raw
+// buffers (2 when shared memory allows, else 1).
 template <int BITS, bool IN_F32, int H>
 __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
     constexpr int Q = H / kE;                        // threads per h-block
     constexpr bool REPL = (BITS <= 4);               // per-lane table copies (conflict-free)
     constexpr int TSH = REPL ? 7 : 2;                // table row stride: 32 lanes x 4 B, or 4 B
     constexpr int NW = kE * BITS / 32;               // packed code words per token per thread
-    constexpr int PAIR_BYTES = IN_F32 ? 8 : 4;
+    constexpr int IN_BYTES = IN_F32 ? 4 : 2;
 
     extern __shared__ __align__(16) unsigned char smem[];
     const int d = p.d;
     const int GT = d / kE;                           // threads per token pair
     const int NG = p.groups;
+    const int nstage = IN_F32 ? p.stages : 1;        // raw row buffers per group
     const int tid = threadIdx.x;
     const int grp = tid / GT;
     const int g = tid - grp * GT;
@@ -144,105 +192,130 @@ __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
     const int warp_start = tid - lane;
     const int active = min(32, (int)blockDim.x - warp_start);
     const unsigned wmask = active == 32 ? 0xffffffffu : ((1u << active) - 1u);
+    const uint32_t row_in = (uint32_t)d * IN_BYTES;  // bytes of one input row
 
-    // shared memory: [quantizer table][gather entries][segment partials][pair buffers]
+    // shared memory: [table][entries][partials][mbarriers][raw rows][pair buffers (bf16)]
     const int table_words = (p.G + 1) * (REPL ? 32 : 1);
     uint32_t *table = reinterpret_cast<uint32_t *>(smem);
     uint32_t *gent = table + ((table_words + 3) & ~3);
-    float2 *red = reinterpret_cast<float2 *>(gent + d);
-    unsigned char *pairs = reinterpret_cast<unsigned char *>(red + NG * kMaxSeg);
-    unsigned char *mypairs = pairs + (size_t)grp * d * PAIR_BYTES;
+    float2 *red = reinterpret_cast<float2 *>(gent + GT * kEntStride);
+    unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + NG * kMaxSeg);
+    unsigned char *raw = reinterpret_cast<unsigned char *>(bars + 2 * NG);
+    unsigned char *myraw = raw + (size_t)grp * nstage * 2 * row_in;
+    unsigned char *pairs = raw + (size_t)NG * nstage * 2 * row_in;
+    unsigned char *mypairs = pairs + (size_t)grp * d * 4;
 
     for (int i = tid; i < table_words; i += blockDim.x)
         table[i] = p.grid[REPL ? (i >> 5) : i];
     for (int i = tid; i < d; i += blockDim.x) {
         const uint32_t v = p.rp[i];
-        gent[i] = ((v & 0x7fffffffu) * PAIR_BYTES) | (v & 0x80000000u);
+        const uint32_t j = v & 0x7fffffffu;
+        const uint32_t off = IN_F32 ? 4u * j : 4u * pair_word(j, (uint32_t)d);
+        gent[(i >> 5) * kEntStride + (i & 31)] = off | (v & 0x80000000u);
+    }
+    if (g == 0) {
+        for (int s = 0; s < nstage; ++s)
+            mbar_init(smem_u32(&bars[2 * grp + s]), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
 
-    // this thread's 32 rotated positions
+    // this thread's 32 rotated positions: pos0 + e with pos0 = g * 32
     const int blk = g / Q, r = g - blk * Q;
     const int pos0 = blk * H + r * kE;
-    const uint4 *myent = reinterpret_cast<const uint4 *>(gent + pos0);
-    const uint32_t pair_base = smem_u32(mypairs);
+    const uint4 *myent = reinterpret_cast<const uint4 *>(gent + g * kEntStride);
     const uint32_t tbl_lane =
         smem_u32(table) + (REPL ? lane * 4 : 0) - ((0x3F800000u >> p.F) << TSH);
     const uint32_t G = (uint32_t)p.G;
     const int F = p.F;
 
-    // segmented-reduction bookkeeping (a warp may hold the tails of two groups)
     const int seg_end = min(active, lane + (GT - g));
     const bool seg_head = (lane == 0) || (g == 0);
     const int seg_slot = (g == 0) ? 0 : (g + 31) / 32;
     const int nslots = 1 + ((grp * GT + GT - 1) / 32 - (grp * GT) / 32);
     const int row_bytes = d * BITS / 8;
-
     const long long npairs = ((long long)p.T + 1) / 2;
-    for (long long base = (long long)blockIdx.x * NG; base < npairs;
-         base += (long long)gridDim.x * NG) {
-        const long long pr = base + grp;
-        const bool valid = pr < npairs;
-        const long long t0 = 2 * pr, t1 = 2 * pr + 1;
-        const bool has1 = valid && t1 < p.T;
+    const long long stride = (long long)gridDim.x * NG;
+    const unsigned char *xb = static_cast<const unsigned char *>(p.x);
 
-        // ---- stage the pair, interleaved -------------------------------------------------
-        if (valid) {
-            if constexpr (!IN_F32) {
-                const uint4 *x0 = reinterpret_cast<const uint4 *>(
-                    static_cast<const __nv_bfloat16 *>(p.x) + t0 * d);
-                const uint4 *x1 = reinterpret_cast<const uint4 *>(
-                    static_cast<const __nv_bfloat16 *>(p.x) + t1 * d);
+    // the two rows of pair `pr` into raw stage `s` (one thread per group issues)
+    auto issue = [&](long long pr, int s) {
+        if (g != 0 || pr >= npairs)
+            return;
+        const long long t0 = 2 * pr;
+        const bool two = t0 + 1 < p.T;
+        const uint32_t bar = smem_u32(&bars[2 * grp + s]);
+        const uint32_t dst = smem_u32(myraw + (size_t)s * 2 * row_in);
+        mbar_expect_tx(bar, two ? 2 * row_in : row_in);
+        bulk_copy(dst, xb + t0 * row_in, row_in, bar);
+        if (two)
+            bulk_copy(dst + row_in, xb + (t0 + 1) * row_in, row_in, bar);
+    };
+
+    __syncthreads();
+    issue((long long)blockIdx.x * NG + grp, 0);
+
+    int round = 0;
+    for (long long base = (long long)blockIdx.x * NG; base < npairs; base += stride, ++round) {
+        const long long pr = base + grp;
+        bool valid = pr < npairs;
+        const long long t0 = 2 * pr, t1 = 2 * pr + 1;
+        const int stage = round % nstage;
+        const uint32_t parity = (uint32_t)(round / nstage) & 1u;
+
+        if (valid && !mbar_wait(smem_u32(&bars[2 * grp + stage]), parity)) {
+            atomicOr(&g_k1_err, K1_ERR_COPY_WAIT);
+            valid = false;
+        }
+        const bool has1 = valid && t1 < p.T;
+        const unsigned char *cur = myraw + (size_t)stage * 2 * row_in;
+
+        if constexpr (!IN_F32) {
+            // ---- interleave the staged rows into the pair buffer ---------------------------
+            if (valid) {
+                const uint4 *r0 = reinterpret_cast<const uint4 *>(cur);
+                const uint4 *r1 = reinterpret_cast<const uint4 *>(cur + row_in);
+                uint4 *lo = reinterpret_cast<uint4 *>(mypairs);
+                uint4 *hi = reinterpret_cast<uint4 *>(mypairs + 2 * d);
 #pragma unroll
                 for (int k = 0; k < kE / 8; ++k) {
-                    const int c = g + k * GT;            // 16-byte chunk: elements 8c..8c+7
-                    uint4 a = ldg_stream(x0 + c);
-                    uint4 b = has1 ? ldg_stream(x1 + c) : make_uint4(0, 0, 0, 0);
-                    uint4 lo, hi;
-                    lo.x = prmt(a.x, b.x, 0x5410); lo.y = prmt(a.x, b.x, 0x7632);
-                    lo.z = prmt(a.y, b.y, 0x5410); lo.w = prmt(a.y, b.y, 0x7632);
-                    hi.x = prmt(a.z, b.z, 0x5410); hi.y = prmt(a.z, b.z, 0x7632);
-                    hi.z = prmt(a.w, b.w, 0x5410); hi.w = prmt(a.w, b.w, 0x7632);
-                    uint4 *dst = reinterpret_cast<uint4 *>(mypairs) + 2 * c;
-                    dst[0] = lo;
-                    dst[1] = hi;
-                }
-            } else {
-                const uint4 *x0 = reinterpret_cast<const uint4 *>(
-                    static_cast<const float *>(p.x) + t0 * d);
-                const uint4 *x1 = reinterpret_cast<const uint4 *>(
-                    static_cast<const float *>(p.x) + t1 * d);
-#pragma unroll
-                for (int k = 0; k < kE / 4; ++k) {
-                    const int c = g + k * GT;            // elements 4c..4c+3
-                    uint4 a = ldg_stream(x0 + c);
-                    uint4 b = has1 ? ldg_stream(x1 + c) : make_uint4(0, 0, 0, 0);
-                    uint4 *dst = reinterpret_cast<uint4 *>(mypairs) + 2 * c;
-                    dst[0] = make_uint4(a.x, b.x, a.y, b.y);
-                    dst[1] = make_uint4(a.z, b.z, a.w, b.w);
+                    const int c = g + k * GT;              // elements 8c..8c+7
+                    const uint4 a = r0[c], b = r1[c];
+                    lo[c] = make_uint4(prmt(a.x, b.x, 0x5410), prmt(a.x, b.x, 0x7632),
+                                       prmt(a.y, b.y, 0x5410), prmt(a.y, b.y, 0x7632));
+                    hi[c] = make_uint4(prmt(a.z, b.z, 0x5410), prmt(a.z, b.z, 0x7632),
+                                       prmt(a.w, b.w, 0x5410), prmt(a.w, b.w, 0x7632));
                 }
             }
+            __syncthreads();
+            issue(pr + stride, 0);                         // raw is free: fetch next round
+        } else {
+            if (nstage > 1)
+                issue(pr + stride, (round + 1) % nstage);  // the other stage is free
         }
-        __syncthreads();
 
         // ---- gather y[i] = sign[i] * x[perm[i]] for both tokens ------------------------------
         float2 v[kE];
-        uint32_t ent[4];
+        {
+            const uint32_t base0 = IN_F32 ? smem_u32(cur) : smem_u32(mypairs);
 #pragma unroll
-        for (int e = 0; e < kE; ++e) {
-            if ((e & 3) == 0) {
-                const uint4 q4 = myent[e >> 2];
-                ent[0] = q4.x; ent[1] = q4.y; ent[2] = q4.z; ent[3] = q4.w;
-            }
-            const uint32_t en = ent[e & 3];
-            const uint32_t sg = en & 0x80000000u;
-            if constexpr (!IN_F32) {
-                const uint32_t w = lds32(pair_base + (en & 0x7fffffffu));
-                v[e].x = __uint_as_float((w << 16) + sg);
-                v[e].y = __uint_as_float((w ^ en) & 0xffff0000u);
-            } else {
-                const uint2 w = lds64(pair_base + (en & 0x7fffffffu));
-                v[e].x = __uint_as_float(w.x ^ sg);
-                v[e].y = __uint_as_float(w.y ^ sg);
+            for (int e4 = 0; e4 < kE / 4; ++e4) {
+                const uint4 q4 = myent[e4];
+                const uint32_t en4[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int e = 4 * e4 + i;
+                    const uint32_t en = en4[i];
+                    const uint32_t sg = en & 0x80000000u;
+                    const uint32_t off = en & 0x7fffffffu;
+                    if constexpr (!IN_F32) {
+                        const uint32_t w = lds32(base0 + off);
+                        v[e].x = __uint_as_float((w << 16) + sg);
+                        v[e].y = __uint_as_float((w ^ en) & 0xffff0000u);
+                    } else {
+                        v[e].x = __uint_as_float(lds32(base0 + off) ^ sg);
+                        v[e].y = __uint_as_float(lds32(base0 + row_in + off) ^ sg);
+                    }
+                }
             }
         }
 
@@ -289,6 +362,10 @@ __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
         if (seg_head)
             red[grp * kMaxSeg + seg_slot] = acc;
         __syncthreads();
+        if constexpr (IN_F32) {
+            if (nstage == 1)
+                issue(pr + stride, 0);                     // gathers are done: refill
+        }
         float2 ss = red[grp * kMaxSeg];
         for (int i = 1; i < nslots; ++i) {
             const float2 o = red[grp * kMaxSeg + i];
@@ -340,8 +417,8 @@ __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
 }
 
 template <int BITS, bool F32>
-cudaError_t launch_h(const K1Params &p, int h, dim3 grid, int threads, size_t smem,
-                     cudaStream_t st, std::string *why) {
+cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int threads, size_t smem,
+                     int num_sms, cudaStream_t st, std::string *why) {
     auto go = [&](auto kern) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
@@ -349,7 +426,16 @@ cudaError_t launch_h(const K1Params &p, int h, dim3 grid, int threads, size_t sm
             *why = "cudaFuncSetAttribute(k1)";
             return e;
         }
-        kern<<<grid, threads, smem, st>>>(p);
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+        if (e != cudaSuccess || per_sm < 1) {
+            *why = "k1 does not fit on an SM";
+            return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+        }
+        long long grid = (long long)num_sms * per_sm;
+        if (grid > ctas_needed)
+            grid = ctas_needed;
+        kern<<<(unsigned)grid, threads, smem, st>>>(p);
         e = cudaGetLastError();
         if (e != cudaSuccess)
             *why = "k1 launch";
@@ -366,43 +452,55 @@ cudaError_t launch_h(const K1Params &p, int h, dim3 grid, int threads, size_t sm
     }
 }
 
+size_t k1_smem(int d, int G, int bits, int in_f32, int NG, int stages) {
+    const int GT = d / kE;
+    const size_t table_words = (size_t)(G + 1) * (bits <= 4 ? 32 : 1);
+    const size_t row_in = (size_t)d * (in_f32 ? 4 : 2);
+    size_t b = ((table_words + 3) & ~(size_t)3) * 4;       // quantizer table
+    b += (size_t)GT * kEntStride * 4;                      // gather entries
+    b += sizeof(float2) * NG * kMaxSeg;                    // norm partials
+    b += 16 * (size_t)NG;                                  // mbarriers (2 per group)
+    b += (size_t)NG * stages * 2 * row_in;                 // raw rows
+    if (!in_f32)
+        b += (size_t)NG * d * 4;                           // interleaved pairs
+    return b;
+}
+
 }  // namespace
 
 cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStream_t st,
                       int num_sms, std::string *why) {
     K1Params p = p_in;
     const int GT = p.d / kE;
+    const long long npairs = ((long long)p.T + 1) / 2;
+    int stages = in_f32 ? 2 : 1;
+    if (in_f32 && k1_smem(p.d, p.G, bits, in_f32, 1, 2) > 200 * 1024)
+        stages = 1;
     int NG = 256 / GT;
     if (NG < 1)
         NG = 1;
-    const long long npairs = ((long long)p.T + 1) / 2;
     if (NG > npairs)
         NG = (int)npairs;
-    const size_t pair_bytes = (size_t)p.d * (in_f32 ? 8 : 4);
-    while (NG > 1 && NG * pair_bytes > 96 * 1024)
+    while (NG > 1 && k1_smem(p.d, p.G, bits, in_f32, NG, stages) > 100 * 1024)
         --NG;
+    const size_t smem = k1_smem(p.d, p.G, bits, in_f32, NG, stages);
+    if (smem > 227 * 1024) {
+        *why = "k1 shared memory exceeds the per-CTA limit";
+        return cudaErrorInvalidConfiguration;
+    }
     p.groups = NG;
+    p.stages = stages;
     const int threads = NG * GT;
-    const int table_words = (p.G + 1) * (bits <= 4 ? 32 : 1);
-    const size_t smem = (size_t)((table_words + 3) & ~3) * 4 + (size_t)p.d * 4 +
-                        sizeof(float2) * NG * kMaxSeg + NG * pair_bytes;
     const long long ctas_needed = (npairs + NG - 1) / NG;
-    const int resident = (threads <= 256 ? 3 : (threads <= 512 ? 1 : 1));
-    long long grid = (long long)num_sms * resident * 4;
-    if (grid > ctas_needed)
-        grid = ctas_needed;
-    if (grid < 1)
-        grid = 1;
-    const dim3 g((unsigned)grid);
     switch (bits * 2 + (in_f32 ? 1 : 0)) {
-        case 4: return launch_h<2, false>(p, h, g, threads, smem, st, why);
-        case 5: return launch_h<2, true>(p, h, g, threads, smem, st, why);
-        case 6: return launch_h<3, false>(p, h, g, threads, smem, st, why);
-        case 7: return launch_h<3, true>(p, h, g, threads, smem, st, why);
-        case 8: return launch_h<4, false>(p, h, g, threads, smem, st, why);
-        case 9: return launch_h<4, true>(p, h, g, threads, smem, st, why);
-        case 16: return launch_h<8, false>(p, h, g, threads, smem, st, why);
-        case 17: return launch_h<8, true>(p, h, g, threads, smem, st, why);
+        case 4: return launch_h<2, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 5: return launch_h<2, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 6: return launch_h<3, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 7: return launch_h<3, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 8: return launch_h<4, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 9: return launch_h<4, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 16: return launch_h<8, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 17: return launch_h<8, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
         default: *why = "unsupported bit width"; return cudaErrorInvalidValue;
     }
 }

@@ -8,10 +8,10 @@
 //
 // Path: (1) decode prepass: packed codes -> fp16 unit-variance centroids (LUT), for the
 // activation codes and the weight codes, into stream-ordered workspace; (2) a hand-written
-// tcgen05 GEMM: TMA (128B swizzle) brings fp16 K-major tiles into a 4-stage shared-memory
-// ring, one elected thread issues tcgen05.mma kind::f16 (M=128, N=256, K=16) into a TMEM
-// fp32 accumulator (256 columns), and the 4 warps read TMEM back with tcgen05.ld and apply
-// the s_t * rn_o / d scale in the epilogue.  sigma^2 = 1/d is folded into the epilogue so the
+// persistent tcgen05 GEMM: TMA (128B swizzle) brings fp16 K-major tiles into a 4-stage
+// shared-memory ring, one elected thread issues tcgen05.mma kind::f16 (M=128, N=256, K=16)
+// into one of two TMEM fp32 accumulators (2 x 256 columns), and 4 epilogue warps read the
+// other accumulator back with tcgen05.ld and apply the s_t * rn_o / d scale.  sigma^2 = 1/d is folded into the epilogue so the
 // fp16 values are unit-variance (best fp16 precision).  Every mbarrier wait is bounded by
 // wall time (%globaltimer); a wait that gives up sets a bit in the device error word.
 #include <cuda.h>
@@ -198,9 +198,21 @@ struct GemmParams {
     float inv_d;
 };
 
-// One 128 x 256 output tile per CTA; 4 warps (warp 0 lane 0 = TMA producer, warp 1 lane 0 =
-// MMA issuer, warp 2 = TMEM owner; all 4 warps run the epilogue).
-__global__ void __launch_bounds__(128, 1)
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+constexpr int kThreads = 192;        // 6 warps
+constexpr int kEpiWarps = 4;         // warps 2..5
+constexpr int kAccCols = BN;         // one fp32 accumulator: 256 TMEM columns
+constexpr int kTmemCols = 2 * kAccCols;
+
+// Persistent, warp-specialised tcgen05 GEMM.  Warp 0 lane 0: TMA producer over a 4-stage
+// shared-memory ring.  Warp 1: TMEM owner; its lane 0 issues the MMAs.  Warps 2..5: epilogue
+// (TMEM lane quarter = warp % 4).  Two 256-column accumulators alternate between tiles, so the
+// epilogue of one tile overlaps the mainloop of the next.  Tiles are walked n-fastest so
+// consecutive CTAs share the same 128-row A block in L2.
+__global__ void __launch_bounds__(kThreads, 1)
     k2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const GemmParams p) {
     extern __shared__ unsigned char smem_raw[];
@@ -208,16 +220,19 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;                 // 1 KB aligned tiles
     unsigned char *basep = smem_raw + (base - raw);
     const uint32_t sA = base, sB = base + STAGES * A_STAGE_BYTES;
-    const uint32_t bars = sB + STAGES * B_STAGE_BYTES;            // full[S], empty[S], accum
+    const uint32_t bars = sB + STAGES * B_STAGE_BYTES;
     auto full_bar = [&](int s) { return bars + 8u * s; };
     auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
-    const uint32_t accum_bar = bars + 8u * (2 * STAGES);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (accum_bar + 8u - base));
-    float *rn_s = reinterpret_cast<float *>(basep + (accum_bar + 16u - base));
+    auto tfull_bar = [&](int a) { return bars + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bars + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t drain_bar = bars + 8u * (2 * STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain_bar + 8u - base));
+    float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][BN]
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+    const int n_tiles = (p.N + BN - 1) / BN;
+    const int num_tiles = ((p.M + BM - 1) / BM) * n_tiles;
     const int num_kb = p.K / BK;
 
     if (threadIdx.x == 0) {
@@ -225,108 +240,154 @@ __global__ void __launch_bounds__(128, 1)
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(accum_bar, 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), kEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         abort_flag = 0;
     }
-    if (warp == 2) {
+    if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32(tmem_slot)), "r"(TMEM_COLS) : "memory");
+                     ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    for (int i = threadIdx.x; i < BN; i += blockDim.x)
-        rn_s[i] = (n0 + i < p.N) ? p.rn[n0 + i] : 0.f;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
+    auto give_up = [&](unsigned bit) {
+        atomicOr(&g_k2_err, bit);
+        atomicExch(&abort_flag, 1);
+    };
 
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
         // ---------------- TMA producer ----------------
-        int issued = 0;
-        for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % STAGES;
-            if (kb >= STAGES) {
-                if (!mbar_wait(empty_bar(s), ((kb / STAGES) & 1) ^ 1)) {
-                    atomicOr(&g_k2_err, ERR_WAIT_EMPTY);
-                    atomicExch(&abort_flag, 1);
-                    break;
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !aborted(); tile += gridDim.x) {
+                const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (it >= STAGES &&
+                        !mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1)) {
+                        give_up(ERR_WAIT_EMPTY);
+                        break;
+                    }
+                    if (aborted())
+                        break;
+                    mbar_expect_tx(full_bar(s), STAGE_BYTES);
+                    tma_load_2d(sA + s * A_STAGE_BYTES, &tmA, kb * BK, m0, full_bar(s));
+                    tma_load_2d(sB + s * B_STAGE_BYTES, &tmB, kb * BK, n0, full_bar(s));
                 }
             }
-            if (*(volatile int *)&abort_flag)
-                break;
-            mbar_expect_tx(full_bar(s), STAGE_BYTES);
-            tma_load_2d(sA + s * A_STAGE_BYTES, &tmA, kb * BK, m0, full_bar(s));
-            tma_load_2d(sB + s * B_STAGE_BYTES, &tmB, kb * BK, n0, full_bar(s));
-            ++issued;
+            if (aborted()) {
+                // let the loads already issued land before the CTA can exit
+                const uint32_t from = it > (uint32_t)STAGES ? it - STAGES : 0;
+                for (uint32_t j = from; j < it; ++j)
+                    mbar_wait(full_bar(j % STAGES), (j / STAGES) & 1);
+            }
         }
-        if (*(volatile int *)&abort_flag) {
-            // let the loads already issued land before the CTA can exit
-            for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-                mbar_wait(full_bar(kb % STAGES), (kb / STAGES) & 1);
-        }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        // The final commit to accum_bar tracks every MMA issued here, so the epilogue's wait
-        // on it also drains the tensor pipe before TMEM is released, on the error path too.
-        for (int kb = 0; kb < num_kb; ++kb) {
-            const int s = kb % STAGES;
-            if (*(volatile int *)&abort_flag)
-                break;
-            if (!mbar_wait(full_bar(s), (kb / STAGES) & 1)) {
-                atomicOr(&g_k2_err, ERR_WAIT_FULL);
-                atomicExch(&abort_flag, 1);
+        if (lane == 0) {
+            uint32_t it = 0;
+            int i = 0;
+            for (int tile = blockIdx.x; tile < num_tiles && !aborted();
+                 tile += gridDim.x, ++i) {
+                const int acc = i & 1;
+                if (i >= 2 && !mbar_wait(tempty_bar(acc), ((i >> 1) & 1) ^ 1)) {
+                    give_up(ERR_WAIT_EMPTY);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * kAccCols);
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(full_bar(s), (it / STAGES) & 1)) {
+                        give_up(ERR_WAIT_FULL);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = sw128_desc(sA + s * A_STAGE_BYTES);
+                    const uint64_t db = sw128_desc(sB + s * B_STAGE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)   // 16 fp16 = 32 bytes = 2 desc units
+                        mma_f16(d_tmem, da + 2 * kk, db + 2 * kk, (kb | kk) != 0);
+                    mma_commit(empty_bar(s));
+                }
+                if (!ok)
+                    break;
+                mma_commit(tfull_bar(acc));
+            }
+            // every MMA issued above has completed once this barrier flips
+            mma_commit(drain_bar);
+            if (!mbar_wait(drain_bar, 0))
+                atomicOr(&g_k2_err, ERR_WAIT_ACCUM);
+        }
+    } else {
+        // ---------------- epilogue: TMEM -> registers -> scale -> global ----------------
+        // Each epilogue warp keeps its own copy of the tile's row norms (no cross-warp barrier,
+        // so one warp giving up a wait cannot strand the others).
+        const int q = warp & 3;                               // TMEM lane quarter
+        float *rn_t = rn_s + (warp - 2) * BN;
+        int i = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+            const int acc = i & 1;
+            const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+            __syncwarp();                                     // previous tile's reads are done
+            for (int j = lane; j < BN; j += 32)
+                rn_t[j] = (n0 + j < p.N) ? p.rn[n0 + j] : 0.f;
+            __syncwarp();
+            const bool ok = mbar_wait(tfull_bar(acc), (i >> 1) & 1);
+            if (!__all_sync(0xffffffffu, ok && !aborted())) {
+                if (!ok)
+                    give_up(ERR_WAIT_ACCUM);
                 break;
             }
             tc_fence_after();
-            const uint64_t da = sw128_desc(sA + s * A_STAGE_BYTES);
-            const uint64_t db = sw128_desc(sB + s * B_STAGE_BYTES);
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)       // 16 fp16 = 32 bytes = 2 desc units
-                mma_f16(tmem, da + 2 * kk, db + 2 * kk, (kb | kk) != 0);
-            mma_commit(empty_bar(s));
-        }
-        mma_commit(accum_bar);
-    }
-    __syncwarp();
-
-    // ---------------- epilogue: TMEM -> registers -> scale -> global ----------------
-    const bool have_acc = mbar_wait(accum_bar, 0);
-    if (!have_acc)
-        atomicOr(&g_k2_err, ERR_WAIT_ACCUM);
-    tc_fence_after();
-    // tcgen05.ld is warp-collective: decide per warp
-    const bool go = __all_sync(0xffffffffu, have_acc && !*(volatile int *)&abort_flag);
-    if (go) {
-        const int row = m0 + warp * 32 + lane;
-        const float srow = (row < p.M) ? p.s[row] * p.inv_d : 0.f;
-        float *yrow = p.y + (size_t)row * p.N + n0;
+            const int row = m0 + q * 32 + lane;
+            const float srow = (row < p.M) ? p.s[row] * p.inv_d : 0.f;
+            float *yrow = p.y + (size_t)row * p.N + n0;
+            const uint32_t t_base =
+                tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32), r);
-            if (row < p.M) {
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(t_base + (uint32_t)(c * 32), r);
+                if (row < p.M) {
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const int col = c * 32 + j;
-                    if (n0 + col < p.N) {
-                        float4 o;
-                        o.x = __uint_as_float(r[j + 0]) * srow * rn_s[col + 0];
-                        o.y = __uint_as_float(r[j + 1]) * srow * rn_s[col + 1];
-                        o.z = __uint_as_float(r[j + 2]) * srow * rn_s[col + 2];
-                        o.w = __uint_as_float(r[j + 3]) * srow * rn_s[col + 3];
-                        *reinterpret_cast<float4 *>(yrow + col) = o;
+                    for (int j = 0; j < 32; j += 4) {
+                        const int col = c * 32 + j;
+                        if (n0 + col < p.N) {
+                            const float4 rn4 = *reinterpret_cast<const float4 *>(rn_t + col);
+                            float4 o;
+                            o.x = __uint_as_float(r[j + 0]) * srow * rn4.x;
+                            o.y = __uint_as_float(r[j + 1]) * srow * rn4.y;
+                            o.z = __uint_as_float(r[j + 2]) * srow * rn4.z;
+                            o.w = __uint_as_float(r[j + 3]) * srow * rn4.w;
+                            *reinterpret_cast<float4 *>(yrow + col) = o;
+                        }
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(tempty_bar(acc));
         }
     }
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
-                     ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+                     ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
@@ -415,14 +476,14 @@ cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long lo
 
 cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s,
                         const float *rn, float *y, int T, int N, int d, cudaStream_t st,
-                        std::string *why) {
+                        int num_sms, std::string *why) {
     CUtensorMap ma, mb;
     if (!make_map(&ma, A16, T, d, BM) || !make_map(&mb, B16, N, d, BN)) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
-    const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + 8 * (2 * STAGES + 1) + 8 +
-                        BN * sizeof(float) + 64;
+    const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + 8 * (2 * STAGES + 5) + 8 +
+                        kEpiWarps * BN * sizeof(float) + 64;
     cudaError_t e =
         cudaFuncSetAttribute(k2_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) {
@@ -437,8 +498,8 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s
     gp.N = N;
     gp.K = d;
     gp.inv_d = 1.0f / (float)d;
-    dim3 grid((N + BN - 1) / BN, (T + BM - 1) / BM);
-    k2_gemm<<<grid, 128, smem, st>>>(ma, mb, gp);
+    const int tiles = ((N + BN - 1) / BN) * ((T + BM - 1) / BM);
+    k2_gemm<<<tiles < num_sms ? tiles : num_sms, kThreads, smem, st>>>(ma, mb, gp);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         *why = "k2_gemm launch";

@@ -603,7 +603,7 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     if (e == cudaSuccess)
         e = timed(OQ_KERNEL_GEMM, st, [&] {
             return oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T,
-                                   out_features, d, st, &why);
+                                   out_features, d, st, di->sms, &why);
         });
     cudaError_t e2 = cudaFreeAsync(ws, st);
     if (e != cudaSuccess)
@@ -664,7 +664,7 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
                               &why);
     if (e == cudaSuccess)
         e = oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T, out_features,
-                            d, st, &why);
+                            d, st, di->sms, &why);
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());
     return OQ_OK;

@@ -26,7 +26,8 @@ struct K1Params {
     float eps;              // added to the norm before division (0 for weights)
     float K;                // sqrt(d/h) / (G * delta): z_unnormalised * K / (s+eps) = u/(G delta)
     int G, F;               // grid cells (power of two), F = 23 - log2(G)
-    int groups;             // token pairs processed at once per CTA
+    int groups;             // token pairs processed at once per CTA (set by launch_k1)
+    int stages;             // raw row buffers per group, fp32 input only (set by launch_k1)
 };
 
 // Launch K1 for (bits, h, dtype); `num_sms` sizes the grid.
@@ -44,7 +45,7 @@ cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long lo
 // y[T, N] = (s_t rn_o / d) * A16[T, d] . B16[N, d]^T   (fp16 x fp16 -> fp32 in TMEM)
 cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s,
                         const float *rn, float *y, int T, int N, int d, cudaStream_t st,
-                        std::string *why);
+                        int num_sms, std::string *why);
 
 // Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
 // its size, and its address on the current device (looked up once per device).
