@@ -30,6 +30,10 @@
 //     in the device error word (read by oq_check) and the round's outputs are not written.
 #include <cuda_bf16.h>
 
+#include <map>
+#include <set>
+#include <tuple>
+
 #include "oq_internal.h"
 
 namespace oq {
@@ -39,46 +43,24 @@ __device__ unsigned int g_k1_err;
 
 constexpr int kE = 32;                // rotated positions per thread (per token)
 constexpr int kMaxSeg = 18;           // segment slots per group for the norm reduction
-constexpr int kEntStride = kE + 4;    // padded per-thread entry rows (conflict-free loads)
+constexpr int kEntStride = kK1EntStride;   // padded entry rows (conflict-free 16 B loads)
+static_assert(kEntStride == kE + 4, "entry image layout");
 
 enum : unsigned { K1_ERR_COPY_WAIT = 1u };
 
-__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
-    float2 c;
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
-        : "=f"(c.x), "=f"(c.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return c;
-}
+// Packed fp32x2 arithmetic (sm_100 FADD2/FFMA2 through the CUDA builtins).
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
 __device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
-    float2 c;
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "sub.rn.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
-        : "=f"(c.x), "=f"(c.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return c;
+    return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);     // a - b, one rounding
 }
 
-__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // (a + 1.0) rounded toward -inf, for both lanes; returns the fp32 bit patterns.
 __device__ __forceinline__ uint2 f2_add_one_rm_bits(float a0, float a1) {
-    uint2 r;
-    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\t"
-        "add.rm.f32x2 rc, ra, rb;\n\tmov.b64 {%0, %1}, rc;\n\t}"
-        : "=r"(r.x), "=r"(r.y) : "f"(a0), "f"(a1), "f"(1.0f));
-    return r;
+    const float2 r = __fadd2_rd(make_float2(a0, a1), make_float2(1.0f, 1.0f));
+    return make_uint2(__float_as_uint(r.x), __float_as_uint(r.y));
 }
 
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
@@ -143,11 +125,27 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_
         ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
-// Pair-buffer word of source element j (bf16 path): the low and high halves of every
-// 8-element chunk live in separate regions, so the interleave stores of consecutive threads
-// are contiguous 16-byte runs.
-__device__ __forceinline__ uint32_t pair_word(uint32_t j, uint32_t d) {
-    return (j & 4u) ? (d / 2 + (j >> 3) * 4 + (j & 3u)) : ((j >> 3) * 4 + (j & 3u));
+// Top bytes of a, b, c, d as bytes 0..3 of one word.
+__device__ __forceinline__ uint32_t top_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return prmt(prmt(a, b, 0x0073), prmt(c, d, 0x7300), 0x7610);
+}
+
+// 32/BITS codes (each in the top byte of D[k]) -> one LSB-first packed word (BITS = 2, 4, 8).
+template <int BITS>
+__device__ __forceinline__ uint32_t pack_codes(const uint32_t (&D)[32 / BITS]) {
+    if constexpr (BITS == 8) {
+        return top_bytes(D[0], D[1], D[2], D[3]);
+    } else if constexpr (BITS == 4) {
+        const uint32_t even = top_bytes(D[0], D[2], D[4], D[6]);
+        const uint32_t odd = top_bytes(D[1], D[3], D[5], D[7]);
+        return even | (odd << 4);
+    } else {
+        const uint32_t q0 = top_bytes(D[0], D[4], D[8], D[12]);
+        const uint32_t q1 = top_bytes(D[1], D[5], D[9], D[13]);
+        const uint32_t q2 = top_bytes(D[2], D[6], D[10], D[14]);
+        const uint32_t q3 = top_bytes(D[3], D[7], D[11], D[15]);
+        return q0 | (q1 << 2) | (q2 << 4) | (q3 << 6);
+    }
 }
 
 // Store `NWORDS` 32-bit words of packed codes; alignment follows from the chunk size.
@@ -173,7 +171,7 @@ __device__ __forceinline__ void store_words(uint8_t *dst, const uint32_t (&w)[NW
 // the interleaved pair buffer.  fp32 input: rows are gathered straight from `stages` raw
 // buffers (2 when shared memory allows, else 1).
 template <int BITS, bool IN_F32, int H>
-__global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
+__global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     constexpr int Q = H / kE;                        // threads per h-block
     constexpr bool REPL = (BITS <= 4);               // per-lane table copies (conflict-free)
     constexpr int TSH = REPL ? 7 : 2;                // table row stride: 32 lanes x 4 B, or 4 B
@@ -195,28 +193,27 @@ __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
     const uint32_t row_in = (uint32_t)d * IN_BYTES;  // bytes of one input row
 
     // shared memory: [table][entries][partials][mbarriers][raw rows][pair buffers (bf16)]
-    const int table_words = (p.G + 1) * (REPL ? 32 : 1);
     uint32_t *table = reinterpret_cast<uint32_t *>(smem);
-    uint32_t *gent = table + ((table_words + 3) & ~3);
-    float2 *red = reinterpret_cast<float2 *>(gent + GT * kEntStride);
+    uint32_t *gent = table + p.tbl_words;
+    float2 *red = reinterpret_cast<float2 *>(gent + p.ent_words);
     unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + NG * kMaxSeg);
-    unsigned char *raw = reinterpret_cast<unsigned char *>(bars + 2 * NG);
+    unsigned char *raw = reinterpret_cast<unsigned char *>(bars + 2 * NG + 2);
     unsigned char *myraw = raw + (size_t)grp * nstage * 2 * row_in;
     unsigned char *pairs = raw + (size_t)NG * nstage * 2 * row_in;
     unsigned char *mypairs = pairs + (size_t)grp * d * 4;
+    const uint32_t setup_bar = smem_u32(&bars[2 * NG]);
 
-    for (int i = tid; i < table_words; i += blockDim.x)
-        table[i] = p.grid[REPL ? (i >> 5) : i];
-    for (int i = tid; i < d; i += blockDim.x) {
-        const uint32_t v = p.rp[i];
-        const uint32_t j = v & 0x7fffffffu;
-        const uint32_t off = IN_F32 ? 4u * j : 4u * pair_word(j, (uint32_t)d);
-        gent[(i >> 5) * kEntStride + (i & 31)] = off | (v & 0x80000000u);
-    }
-    if (g == 0) {
-        for (int s = 0; s < nstage; ++s)
-            mbar_init(smem_u32(&bars[2 * grp + s]), 1);
+    if (tid == 0) {
+        for (int b = 0; b < 2 * NG + 1; ++b)
+            mbar_init(smem_u32(&bars[b]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // host-built table and entry images: two bulk copies
+        mbar_expect_tx(setup_bar, 4u * (p.tbl_words + p.ent_words));
+        bulk_copy(smem_u32(table), p.tbl_img, 4u * p.tbl_words, setup_bar);
+        bulk_copy(smem_u32(gent), p.ent_img, 4u * p.ent_words, setup_bar);
     }
 
     // this thread's 32 rotated positions: pos0 + e with pos0 = g * 32
@@ -251,8 +248,9 @@ __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
             bulk_copy(dst + row_in, xb + (t0 + 1) * row_in, row_in, bar);
     };
 
-    __syncthreads();
     issue((long long)blockIdx.x * NG + grp, 0);
+    if (!mbar_wait(setup_bar, 0))
+        atomicOr(&g_k1_err, K1_ERR_COPY_WAIT);
 
     int round = 0;
     for (long long base = (long long)blockIdx.x * NG; base < npairs; base += stride, ++round) {
@@ -379,27 +377,46 @@ __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
 
         // ---- nearest centroid + pack ---------------------------------------------------------
         uint32_t w0[NW], w1[NW];
-#pragma unroll
-        for (int i = 0; i < NW; ++i) {
-            w0[i] = 0;
-            w1[i] = 0;
-        }
-#pragma unroll
-        for (int e = 0; e < kE; ++e) {
-            const float a0 = fma_sat(v[e].x, m0, 0.5f);
-            const float a1 = fma_sat(v[e].y, m1, 0.5f);
+        // The code of element e is the top byte of D = q*G + table[q >> F].
+        auto code_word = [&](float vx, float vy, uint32_t &d0, uint32_t &d1) {
+            const float a0 = fma_sat(vx, m0, 0.5f);
+            const float a1 = fma_sat(vy, m1, 0.5f);
             const uint2 qb = f2_add_one_rm_bits(a0, a1);
-            const uint32_t t0w = lds32(tbl_lane + ((qb.x >> F) << TSH));
-            const uint32_t t1w = lds32(tbl_lane + ((qb.y >> F) << TSH));
-            const uint32_t c0 = (qb.x * G + t0w) >> 24;
-            const uint32_t c1 = (qb.y * G + t1w) >> 24;
-            const int bit = e * BITS;
-            const int wi = bit >> 5, sh = bit & 31;
-            w0[wi] |= c0 << sh;
-            w1[wi] |= c1 << sh;
-            if (sh + BITS > 32) {
-                w0[wi + 1] |= c0 >> (32 - sh);
-                w1[wi + 1] |= c1 >> (32 - sh);
+            d0 = qb.x * G + lds32(tbl_lane + ((qb.x >> F) << TSH));
+            d1 = qb.y * G + lds32(tbl_lane + ((qb.y >> F) << TSH));
+        };
+        if constexpr (BITS == 3) {
+#pragma unroll
+            for (int i = 0; i < NW; ++i) {
+                w0[i] = 0;
+                w1[i] = 0;
+            }
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                uint32_t d0, d1;
+                code_word(v[e].x, v[e].y, d0, d1);
+                const uint32_t c0 = d0 >> 24, c1 = d1 >> 24;
+                const int bit = e * BITS;
+                const int wi = bit >> 5, sh = bit & 31;
+                w0[wi] |= c0 << sh;
+                w1[wi] |= c1 << sh;
+                if (sh + BITS > 32) {
+                    w0[wi + 1] |= c0 >> (32 - sh);
+                    w1[wi + 1] |= c1 >> (32 - sh);
+                }
+            }
+        } else {
+            // byte permutes gather the top bytes; 2- and 4-bit codes are then merged into
+            // nibbles / bit pairs with shifted adds (the bytes' upper bits are zero)
+            constexpr int PER = 32 / BITS;                 // codes per output word
+#pragma unroll
+            for (int wi = 0; wi < NW; ++wi) {
+                uint32_t d0[PER], d1[PER];
+#pragma unroll
+                for (int k = 0; k < PER; ++k)
+                    code_word(v[wi * PER + k].x, v[wi * PER + k].y, d0[k], d1[k]);
+                w0[wi] = pack_codes<BITS>(d0);
+                w1[wi] = pack_codes<BITS>(d1);
             }
         }
         if (valid) {
@@ -416,20 +433,54 @@ __global__ void __launch_bounds__(512) k1_rotquant(const K1Params p) {
     }
 }
 
+// Shared-memory attributes are set once per kernel and device, and occupancy is cached per
+// (kernel, device, block size, shared memory), to keep the per-call host cost low.
+cudaError_t k1_prepare(const void *kern, int threads, size_t smem, int *per_sm) {
+    struct Key {
+        const void *k;
+        int dev, threads;
+        size_t smem;
+        bool operator<(const Key &o) const {
+            return std::tie(k, dev, threads, smem) < std::tie(o.k, o.dev, o.threads, o.smem);
+        }
+    };
+    static std::mutex mu;
+    static std::map<Key, int> occ;
+    static std::set<std::pair<const void *, int>> attr_done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!attr_done.count({kern, dev})) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess)
+            return e;
+        attr_done.insert({kern, dev});
+    }
+    const Key key{kern, dev, threads, smem};
+    auto it = occ.find(key);
+    if (it == occ.end()) {
+        int n = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem);
+        if (e != cudaSuccess)
+            return e;
+        it = occ.emplace(key, n).first;
+    }
+    *per_sm = it->second;
+    return cudaSuccess;
+}
+
 template <int BITS, bool F32>
 cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int threads, size_t smem,
                      int num_sms, cudaStream_t st, std::string *why) {
     auto go = [&](auto kern) -> cudaError_t {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) {
-            *why = "cudaFuncSetAttribute(k1)";
-            return e;
-        }
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+        cudaError_t e = k1_prepare((const void *)kern, threads, smem, &per_sm);
         if (e != cudaSuccess || per_sm < 1) {
-            *why = "k1 does not fit on an SM";
+            *why = "k1 attributes / occupancy";
             return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
         }
         long long grid = (long long)num_sms * per_sm;
@@ -452,17 +503,14 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
     }
 }
 
-size_t k1_smem(int d, int G, int bits, int in_f32, int NG, int stages) {
-    const int GT = d / kE;
-    const size_t table_words = (size_t)(G + 1) * (bits <= 4 ? 32 : 1);
-    const size_t row_in = (size_t)d * (in_f32 ? 4 : 2);
-    size_t b = ((table_words + 3) & ~(size_t)3) * 4;       // quantizer table
-    b += (size_t)GT * kEntStride * 4;                      // gather entries
+size_t k1_smem(const K1Params &p, int in_f32, int NG, int stages) {
+    const size_t row_in = (size_t)p.d * (in_f32 ? 4 : 2);
+    size_t b = 4 * (size_t)(p.tbl_words + p.ent_words);    // table + gather entries
     b += sizeof(float2) * NG * kMaxSeg;                    // norm partials
-    b += 16 * (size_t)NG;                                  // mbarriers (2 per group)
+    b += 8 * (size_t)(2 * NG + 2);                         // mbarriers
     b += (size_t)NG * stages * 2 * row_in;                 // raw rows
     if (!in_f32)
-        b += (size_t)NG * d * 4;                           // interleaved pairs
+        b += (size_t)NG * p.d * 4;                         // interleaved pairs
     return b;
 }
 
@@ -474,16 +522,16 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     const int GT = p.d / kE;
     const long long npairs = ((long long)p.T + 1) / 2;
     int stages = in_f32 ? 2 : 1;
-    if (in_f32 && k1_smem(p.d, p.G, bits, in_f32, 1, 2) > 200 * 1024)
+    if (in_f32 && k1_smem(p, in_f32, 1, 2) > 200 * 1024)
         stages = 1;
     int NG = 256 / GT;
     if (NG < 1)
         NG = 1;
     if (NG > npairs)
         NG = (int)npairs;
-    while (NG > 1 && k1_smem(p.d, p.G, bits, in_f32, NG, stages) > 100 * 1024)
+    while (NG > 1 && k1_smem(p, in_f32, NG, stages) > 72 * 1024)
         --NG;
-    const size_t smem = k1_smem(p.d, p.G, bits, in_f32, NG, stages);
+    const size_t smem = k1_smem(p, in_f32, NG, stages);
     if (smem > 227 * 1024) {
         *why = "k1 shared memory exceeds the per-CTA limit";
         return cudaErrorInvalidConfiguration;

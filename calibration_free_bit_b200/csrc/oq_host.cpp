@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <limits>
 #include <new>
@@ -54,17 +55,23 @@ cudaEvent_t take_event() {
     return e;
 }
 
-// Run `launch` (returning cudaError_t), bracketed by events when timing is on.
+// Run `launch` (returning cudaError_t), bracketed by events when timing is on.  While the
+// stream is being captured into a CUDA graph the events are recorded as external event nodes,
+// so each replay of the graph re-records them and they stay readable afterwards.
 template <class F>
 cudaError_t timed(int kernel, cudaStream_t st, F &&launch) {
     if (!g_timing)
         return launch();
     TimedLaunch t{kernel, take_event(), take_event()};
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    const unsigned flags =
+        cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
     if (t.start)
-        cudaEventRecord(t.start, st);
+        cudaEventRecordWithFlags(t.start, st, flags);
     cudaError_t e = launch();
     if (t.stop)
-        cudaEventRecord(t.stop, st);
+        cudaEventRecordWithFlags(t.stop, st, flags);
     if (t.start && t.stop)
         g_timed.push_back(t);
     return e;
@@ -223,9 +230,9 @@ struct oq_rpbh {
     uint64_t seed = 0;
     std::vector<int32_t> perm;
     std::vector<int8_t> sign;
-    std::vector<uint32_t> packed;                 // perm | (sign < 0) << 31
+    std::vector<uint32_t> ent_img[2];             // K1 gather-entry images: [0] bf16, [1] fp32
     std::mutex mu;
-    uint32_t *dev[oq::kMaxDevices] = {};
+    uint32_t *dev_ent[2][oq::kMaxDevices] = {};
 };
 
 struct oq_codebook {
@@ -235,8 +242,9 @@ struct oq_codebook {
     int G = 0, F = 0;
     double delta = 0.0;
     std::vector<uint32_t> grid;                   // G + 1 words
+    std::vector<uint32_t> tbl_img;                // K1 shared-memory image of the table
     std::mutex mu;
-    uint32_t *dev_grid[oq::kMaxDevices] = {};
+    uint32_t *dev_tbl[oq::kMaxDevices] = {};
 };
 
 namespace {
@@ -385,16 +393,20 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
         return rc;
     oq_rpbh *rw = const_cast<oq_rpbh *>(r);
     oq_codebook *cw = const_cast<oq_codebook *>(cb);
-    if ((rc = upload(rw->mu, &rw->dev[dev], rw->packed, "upload rotation table")) != OQ_OK)
+    const int f = dtype == OQ_F32 ? 1 : 0;
+    if ((rc = upload(rw->mu, &rw->dev_ent[f][dev], rw->ent_img[f], "upload rotation table")) !=
+        OQ_OK)
         return rc;
-    if ((rc = upload(cw->mu, &cw->dev_grid[dev], cw->grid, "upload quantizer table")) != OQ_OK)
+    if ((rc = upload(cw->mu, &cw->dev_tbl[dev], cw->tbl_img, "upload quantizer table")) != OQ_OK)
         return rc;
     oq::K1Params p{};
     p.x = x;
     p.codes = codes;
     p.norms = norms;
-    p.rp = rw->dev[dev];
-    p.grid = cw->dev_grid[dev];
+    p.ent_img = rw->dev_ent[f][dev];
+    p.tbl_img = cw->dev_tbl[dev];
+    p.ent_words = (int)rw->ent_img[f].size();
+    p.tbl_words = (int)cw->tbl_img.size();
     p.T = rows;
     p.d = d;
     p.eps = eps;
@@ -431,6 +443,16 @@ cudaMemPool_t device_pool(int dev, DeviceInfo *di, int *rc) {
     return pool;
 }
 
+// OQ_LINEAR_PATH=fused sends 4-bit activation codes straight into the GEMM kernel that
+// decodes them itself (read once per process); the default decodes both operands first.
+bool fused_requested() {
+    static const bool v = [] {
+        const char *e = std::getenv("OQ_LINEAR_PATH");
+        return e != nullptr && std::strcmp(e, "fused") == 0;
+    }();
+    return v;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------------------
@@ -455,7 +477,6 @@ int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out) {
     r->seed = seed;
     r->perm.resize(d);
     r->sign.resize(d);
-    r->packed.resize(d);
     SplitMix64 g{seed};
     for (int i = 0; i < d; ++i)
         r->perm[i] = i;
@@ -465,8 +486,18 @@ int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out) {
     }
     for (int k = 0; k < d; ++k)
         r->sign[k] = (g.next() >> 63) ? -1 : 1;
-    for (int k = 0; k < d; ++k)
-        r->packed[k] = (uint32_t)r->perm[k] | (r->sign[k] < 0 ? 0x80000000u : 0u);
+    // K1 gather-entry images (layout documented in oq_internal.h)
+    for (int f = 0; f < 2; ++f) {
+        r->ent_img[f].assign((size_t)(d / 32) * oq::kK1EntStride, 0u);
+        for (int i = 0; i < d; ++i) {
+            const uint32_t j = (uint32_t)r->perm[i];
+            const uint32_t word = (j & 4u) ? (uint32_t)d / 2 + (j >> 3) * 4 + (j & 3u)
+                                           : (j >> 3) * 4 + (j & 3u);
+            const uint32_t off = (f == 1) ? 4u * j : 4u * word;
+            r->ent_img[f][(size_t)(i >> 5) * oq::kK1EntStride + (i & 31)] =
+                off | (r->sign[i] < 0 ? 0x80000000u : 0u);
+        }
+    }
     *out = r;
     return OQ_OK;
 }
@@ -508,6 +539,12 @@ int oq_lloyd_max(int d, int bits, oq_codebook **out) {
         delete cb;
         return fail(OQ_EINVAL, "oq_lloyd_max: could not build the quantizer grid");
     }
+    // K1 table image: one copy per lane when bits <= 4 (conflict-free lookups), padded to 16 B
+    const int copies = bits <= 4 ? 32 : 1;
+    cb->tbl_img.assign((((size_t)(cb->G + 1) * copies + 3) / 4) * 4, 0u);
+    for (int k = 0; k <= cb->G; ++k)
+        for (int l = 0; l < copies; ++l)
+            cb->tbl_img[(size_t)k * copies + l] = cb->grid[k];
     *out = cb;
     return OQ_OK;
 }
@@ -582,29 +619,48 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     cudaMemPool_t pool = device_pool(dev, di, &rc);
     if (!pool)
         return rc;
-    const size_t ws_bytes = oq::linear_workspace_bytes(T, d, out_features);
+    // Default: both operands decoded to fp16 by the prepass, then the TMA/tcgen05 GEMM.
+    // OQ_LINEAR_PATH=fused with 4-bit activation codes: the codes are decoded inside the GEMM
+    // (only the weights get a prepass).
+    const bool fused = ca->bits == 4 && fused_requested();
+    const size_t ws_bytes = fused ? (size_t)out_features * d * 2
+                                  : oq::linear_workspace_bytes(T, d, out_features);
     void *ws = nullptr;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaMallocFromPoolAsync(&ws, ws_bytes, pool, st);
     if (e != cudaSuccess)
         return fail_cuda(e, "oq_linear: workspace allocation");
-    uint16_t *A16 = static_cast<uint16_t *>(ws);
-    uint16_t *B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
-                                                 oq::linear_workspace_b_offset(T, d));
     std::string why;
-    e = timed(OQ_KERNEL_DECODE, st, [&] {
-        return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
-    });
-    if (e == cudaSuccess)
+    if (fused) {
+        uint16_t *B16 = static_cast<uint16_t *>(ws);
         e = timed(OQ_KERNEL_DECODE, st, [&] {
             return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
                                      di->sms, &why);
         });
-    if (e == cudaSuccess)
-        e = timed(OQ_KERNEL_GEMM, st, [&] {
-            return oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T,
-                                   out_features, d, st, di->sms, &why);
+        if (e == cudaSuccess)
+            e = timed(OQ_KERNEL_GEMM, st, [&] {
+                return oq::launch_gemm_fused_a4(x_codes, ca->lut, B16, s, row_norms,
+                                                static_cast<float *>(y), T, out_features, d, st,
+                                                di->sms, &why);
+            });
+    } else {
+        uint16_t *A16 = static_cast<uint16_t *>(ws);
+        uint16_t *B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
+                                                     oq::linear_workspace_b_offset(T, d));
+        e = timed(OQ_KERNEL_DECODE, st, [&] {
+            return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
         });
+        if (e == cudaSuccess)
+            e = timed(OQ_KERNEL_DECODE, st, [&] {
+                return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
+                                         di->sms, &why);
+            });
+        if (e == cudaSuccess)
+            e = timed(OQ_KERNEL_GEMM, st, [&] {
+                return oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T,
+                                       out_features, d, st, di->sms, &why);
+            });
+    }
     cudaError_t e2 = cudaFreeAsync(ws, st);
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());
@@ -675,15 +731,18 @@ int oq_check(void *stream) {
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess)
         return fail_cuda(e, "oq_check: stream synchronize");
-    unsigned w1 = 0, w2 = 0;
+    unsigned w1 = 0, w2 = 0, w3 = 0;
     if ((e = oq::read_and_clear_k1_error(&w1, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k1 error word");
     if ((e = oq::read_and_clear_k2_error(&w2, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k2 error word");
-    if (w1 || w2)
-        return fail(OQ_EDEVICE, "device error word: quantize=0x%x linear=0x%x (linear bits: "
-                                "1 = TMA stage wait, 2 = slot-release wait, 4 = accumulator "
-                                "wait gave up)", w1, w2);
+    if ((e = oq::read_and_clear_k2f_error(&w3, st)) != cudaSuccess)
+        return fail_cuda(e, "oq_check: read fused k2 error word");
+    if (w1 || w2 || w3)
+        return fail(OQ_EDEVICE, "device error word: quantize=0x%x linear=0x%x fused=0x%x "
+                                "(a bounded wait gave up; quantize bit 1 = row copy, linear "
+                                "bits 1/2/4 = stage/slot/accumulator, fused bits 1/2/4/8 = "
+                                "weight stage/activation stage/slot/accumulator)", w1, w2, w3);
     return OQ_OK;
 }
 
@@ -693,10 +752,11 @@ void oq_free_rpbh(oq_rpbh *r) {
     int cur = -1;
     cudaGetDevice(&cur);
     for (int dev = 0; dev < oq::kMaxDevices; ++dev)
-        if (r->dev[dev]) {
-            cudaSetDevice(dev);
-            cudaFree(r->dev[dev]);
-        }
+        for (int f = 0; f < 2; ++f)
+            if (r->dev_ent[f][dev]) {
+                cudaSetDevice(dev);
+                cudaFree(r->dev_ent[f][dev]);
+            }
     if (cur >= 0)
         cudaSetDevice(cur);
     delete r;
@@ -708,9 +768,9 @@ void oq_free_codebook(oq_codebook *cb) {
     int cur = -1;
     cudaGetDevice(&cur);
     for (int dev = 0; dev < oq::kMaxDevices; ++dev)
-        if (cb->dev_grid[dev]) {
+        if (cb->dev_tbl[dev]) {
             cudaSetDevice(dev);
-            cudaFree(cb->dev_grid[dev]);
+            cudaFree(cb->dev_tbl[dev]);
         }
     if (cur >= 0)
         cudaSetDevice(cur);

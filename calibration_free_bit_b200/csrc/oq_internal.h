@@ -15,13 +15,24 @@ namespace oq {
 
 constexpr int kMaxDevices = 32;
 
+// Shared-memory images of K1, built on the host (oq_host.cpp) and bulk-copied per CTA.
+//   Gather entries: d/32 rows of kK1EntStride words; row g holds, for positions g*32+e,
+//   (byte offset of x[perm[pos]] in the staged row data) | (sign[pos] < 0) << 31.  For fp32
+//   input the offset is 4*perm[pos]; for bf16 input it is 4*pair_word(perm[pos]) with
+//   pair_word(j) = (j & 4) ? d/2 + (j>>3)*4 + (j&3) : (j>>3)*4 + (j&3) (the kernel's interleave
+//   writes the low/high halves of each 8-element chunk into separate regions).
+//   Quantizer table: G+1 words, each repeated 32 times (one copy per lane, k*32 + lane) when
+//   bits <= 4, else stored once; padded to a multiple of 4 words.
+constexpr int kK1EntStride = 36;
+
 // Parameters of the fused rotate + norm + quantize kernel (K1).
 struct K1Params {
     const void *x;          // [T, d] rows, fp32 or bf16
     uint8_t *codes;         // [T, d*bits/8]
     float *norms;           // [T]
-    const uint32_t *rp;     // [d] perm[p] | (sign[p] < 0) << 31
-    const uint32_t *grid;   // [G + 1] quantizer table words
+    const uint32_t *ent_img;   // gather-entry image (see above)
+    const uint32_t *tbl_img;   // quantizer-table image (see above)
+    int ent_words, tbl_words;  // image sizes in 32-bit words (multiples of 4)
     int T, d;
     float eps;              // added to the norm before division (0 for weights)
     float K;                // sqrt(d/h) / (G * delta): z_unnormalised * K / (s+eps) = u/(G delta)
@@ -46,6 +57,13 @@ cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long lo
 cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s,
                         const float *rn, float *y, int T, int N, int d, cudaStream_t st,
                         int num_sms, std::string *why);
+
+// Codebook GEMM with the 4-bit activation codes decoded inside the kernel into tensor memory
+// (k2_fused.cu); B16 is the fp16 weight operand from the decode prepass.  No A workspace.
+cudaError_t launch_gemm_fused_a4(const uint8_t *xc, const uint16_t *lut_a, const uint16_t *B16,
+                                 const float *s, const float *rn, float *y, int T, int N, int d,
+                                 cudaStream_t st, int num_sms, std::string *why);
+cudaError_t read_and_clear_k2f_error(unsigned *out, cudaStream_t st);
 
 // Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
 // its size, and its address on the current device (looked up once per device).

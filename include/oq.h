@@ -115,8 +115,11 @@ int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int 
  * x_codes: device [T, d*ba/8]; s: device fp32 [T]; W_codes: device [out_features, d*bw/8];
  * row_norms: device fp32 [out_features]; y: device [T, out_features] of out_dtype (OQ_F32).
  * Centroids enter the tensor cores as fp16 unit-variance values; accumulation is fp32.
- * Uses stream-ordered temporary device memory (two fp16 operand buffers) from a
- * library-owned pool.  Errors: as above, plus OQ_ECUDA if the pool allocation fails. */
+ * Both code operands are decoded into fp16 buffers first.  With 4-bit activation codes
+ * and the environment variable OQ_LINEAR_PATH=fused (read once per process), the activation
+ * codes are instead decoded inside the GEMM kernel and only the weight codes get an fp16
+ * buffer.  Either way the temporary device memory is stream-ordered, from a library-owned
+ * pool.  Errors: as above, plus OQ_ECUDA if the pool allocation fails. */
 int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
               const float *s, const uint8_t *W_codes, const float *row_norms, int T, int d,
               int out_features, void *y, int out_dtype, void *stream);

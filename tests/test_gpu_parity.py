@@ -216,7 +216,7 @@ def test_linear_toy_on_oracle_codes(oq):
     assert rel_l2(y, ref) <= LINEAR_RTOL
 
 
-@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (4, 3), (8, 4), (2, 8), (8, 8)])
+@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (4, 3), (3, 4), (2, 2), (8, 4), (2, 8), (8, 8)])
 @pytest.mark.parametrize("T,N,d", [(200, 272, 384), (1, 16, 128), (129, 512, 1024)])
 def test_linear_random_codes_ragged(oq, ba, bw, T, N, d):
     """Uniform random codes (every centroid used), ragged M and N tails."""
@@ -279,3 +279,21 @@ def test_linear_video_ffn_up_full_size(oq, variant):
     rows = np.array([0, 5, 32759, 32760, 50000, 65408, 65519])
     cols = np.arange(11, p.out, 977)
     _sampled_linear(oq, p, rows, cols)
+
+
+@pytest.mark.parametrize("path", ["fused", "default"])
+def test_linear_path_selection(oq, path):
+    """Both oq_linear paths for 4-bit activation codes (the decode prepass and, with
+    OQ_LINEAR_PATH=fused, the GEMM that decodes activation codes itself) against the oracle;
+    each runs in a child process because the variable is read once per process."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.pop("OQ_LINEAR_PATH", None)
+    if path == "fused":
+        env["OQ_LINEAR_PATH"] = "fused"
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_linear_path_child.py")
+    r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
