@@ -66,14 +66,22 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_sha(rel):
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_sha(rels):
+    """First 16 hex digits of the SHA-256 of the concatenated source files."""
+    h = hashlib.sha256()
+    for rel in rels:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+GEMM_SOURCES = ("calibration_free_bit_b200/csrc/k2_linear.cu",
+                "calibration_free_bit_b200/csrc/sm100_common.cuh")
 
 
 def profile_traffic(profile_name, kernel_src):
     """DRAM bytes per launch from a committed ncu summary, or None if absent or stale (the
-    summary records the kernel source hash it was captured from)."""
+    summary records the hash of the kernel sources it was captured from)."""
     path = os.path.join(ROOT, "profiles", profile_name)
     if not os.path.exists(path):
         return None, "no profile"
@@ -378,8 +386,7 @@ def run_ours(args, p, rank, world, dev):
     dec_ms = statistics.mean(per_kernel.get("decode", [float("nan")]))
     flops = 2.0 * p.T * p.d * p.out
     gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
-    traffic, traffic_src = profile_traffic(f"k2_gemm_{p.name}.md", "calibration_free_bit_b200/"
-                                           "csrc/k2_linear.cu")
+    traffic, traffic_src = profile_traffic(f"k2_gemm_{p.name}.md", GEMM_SOURCES)
     in_bytes = 2 if p.dtype == torch.bfloat16 else 4
     q_bytes = p.T * (in_bytes * p.d + p.d * p.bits_a // 8 + 4)
     q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9

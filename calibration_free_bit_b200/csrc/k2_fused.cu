@@ -17,16 +17,14 @@
 // 192-column fp32 accumulators and four 32-column A stages: 512 columns.  The epilogue drains
 // the accumulators and releases them before storing the last chunk.
 //
-// Decoding: the 16 centroids of the symmetric Lloyd-Max codebook satisfy c_i = -c_{15-i}, so a
-// code c maps to magnitude index m = c - 8 (c >= 8) or 7 - c (c < 8) and a sign.  The bytes
-// of the 8 fp16 magnitudes sit in four registers; one byte-permute per 4 codes selects the
-// low bytes, one the high bytes, two interleave them into fp16 pairs, and one more permute
-// builds the sign bits.  No shared-memory traffic, ~3 instructions per element.
+// Decoding: decode8() of decode4.cuh (byte permutes on the symmetric codebook, no shared
+// memory).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
 
+#include "decode4.cuh"
 #include "oq_internal.h"
 #include "sm100_common.cuh"
 
@@ -57,7 +55,7 @@ constexpr int kFStageOut = 32 * 32 * 4;             // one 32 x 32 fp32 output c
 constexpr size_t kFusedSmem = 1024 + (size_t)FB_STAGES * FB_STAGE_BYTES +
                               (size_t)kFEpiWarps * 2 * kFStageOut +
                               8 * (2 * FB_STAGES + 2 * FA_STAGES + 3) + 8 +
-                              kFEpiWarps * 32 * sizeof(float) + 64;
+                              kFEpiWarps * 64 * sizeof(float) + 64;
 static_assert(kFusedSmem <= 227 * 1024, "shared memory budget");
 
 enum : unsigned {
@@ -77,23 +75,6 @@ struct FusedParams {
     uint32_t magH0, magH1;      // high bytes of the same
 };
 
-// Eight 4-bit codes (one word, code k in bits 4k..4k+3) -> eight fp16 centroids as four
-// packed pairs (pair j = codes 2j, 2j+1; the lower code in the low half).
-__device__ __forceinline__ void decode8(uint32_t w, uint32_t L0, uint32_t L1, uint32_t H0,
-                                        uint32_t H1, uint32_t (&o)[4]) {
-    const uint32_t nw = ~w;
-    const uint32_t t = (nw >> 3) & 0x11111111u;          // 1 where code < 8 (negative)
-    const uint32_t m = (w ^ (t * 7u)) & 0x77777777u;     // magnitude index per nibble
-    const uint32_t y = nw << 4;                          // bit 7 of byte b <- code 2b's flag
-    const uint32_t lo_a = prmt(L0, L1, m & 0xffffu), hi_a = prmt(H0, H1, m & 0xffffu);
-    const uint32_t lo_b = prmt(L0, L1, m >> 16), hi_b = prmt(H0, H1, m >> 16);
-    // sign of code 2b -> bit 15 (from y, byte b), of code 2b+1 -> bit 31 (from nw, byte b)
-    o[0] = prmt(lo_a, hi_a, 0x5140) ^ (prmt(y, nw, 0x4000) & 0x80008000u);
-    o[1] = prmt(lo_a, hi_a, 0x7362) ^ (prmt(y, nw, 0x5010) & 0x80008000u);
-    o[2] = prmt(lo_b, hi_b, 0x5140) ^ (prmt(y, nw, 0x6020) & 0x80008000u);
-    o[3] = prmt(lo_b, hi_b, 0x7362) ^ (prmt(y, nw, 0x7030) & 0x80008000u);
-}
-
 __device__ __forceinline__ uint4 ldg_nc16(const uint8_t *p) {
     uint4 v;
     asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -106,6 +87,7 @@ __device__ __forceinline__ uint4 ldg_nc16(const uint8_t *p) {
 // Warps 6..13: activation decoders (row quarter = warp % 4, one row per thread, one half of
 // each 64-code block per warp).  When a tile's second 192-column half lies wholly past N,
 // neither its weight box nor its MMAs are issued; its accumulator columns are never stored.
+template <bool BF16>
 __global__ void __launch_bounds__(kFThreads, 1)
     k2_gemm_fused(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmY,
                   const FusedParams p) {
@@ -124,7 +106,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const uint32_t tempty = tfull + 8u;
     const uint32_t drain = tfull + 16u;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain + 8u - base));
-    float *rn_s = reinterpret_cast<float *>(basep + (drain + 16u - base));   // [4][32]
+    float *rn_s = reinterpret_cast<float *>(basep + (drain + 16u - base));   // [4][64]
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -241,19 +223,20 @@ __global__ void __launch_bounds__(kFThreads, 1)
     } else if (warp < 2 + kFEpiWarps) {
         // ---------------- epilogue: TMEM -> registers -> scale -> smem -> TMA store -------
         const int q = warp & 3;
-        float *rn32 = rn_s + (warp - 2) * 32;
+        float *rn_w = rn_s + (warp - 2) * 64;
         const uint32_t out0 = sOut + (uint32_t)((warp - 2) * 2 * kFStageOut);
         unsigned char *out0p = basep + (out0 - base);
-        constexpr int kChunks = FTN / 32;
+        constexpr int kCW = BF16 ? 64 : 32;                 // columns per stored chunk
+        constexpr int kChunks = FTN / kCW;
         uint32_t u = 0;                                     // chunks stored so far
         int i = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
             const int m0 = (tile / n_tiles) * FBM, n0 = (tile % n_tiles) * FTN;
             const int row = m0 + q * 32 + lane;
             const float srow = (row < p.M) ? p.s[row] * p.inv_d : 0.f;
-            float rnv[kChunks];                             // rn of column c*32 + lane
+            float rnv[FTN / 32];                            // rn of column c*32 + lane
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
+            for (int c = 0; c < FTN / 32; ++c) {
                 const int col = n0 + c * 32 + lane;
                 rnv[c] = (col < p.N) ? p.rn[col] : 0.f;
             }
@@ -268,8 +251,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
             const bool rows_in = m0 + q * 32 < p.M;
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_base + (uint32_t)(c * 32), r);   // halves are adjacent in TMEM
+                uint32_t r0[32], r1[32];
+                tmem_ld32(t_base + (uint32_t)(c * kCW), r0);   // halves are adjacent in TMEM
+                if constexpr (BF16)
+                    tmem_ld32(t_base + (uint32_t)(c * kCW + 32), r1);
                 if (c == kChunks - 1) {
                     // every column has been read: hand the accumulators back to the MMA
                     tc_fence_before();
@@ -277,16 +262,25 @@ __global__ void __launch_bounds__(kFThreads, 1)
                     if (lane == 0)
                         mbar_arrive(tempty);
                 }
-                if (!rows_in || n0 + c * 32 >= p.N)
+                if (!rows_in || n0 + c * kCW >= p.N)
                     continue;                               // box wholly outside y
                 const uint32_t b = u & 1;
                 if (lane == 0)
                     bulk_wait_read<1>();                    // the store that used buffer b
                 __syncwarp();
-                rn32[lane] = rnv[c];
+                if constexpr (BF16) {
+                    rn_w[lane] = rnv[2 * c];
+                    rn_w[32 + lane] = rnv[2 * c + 1];
+                } else {
+                    rn_w[lane] = rnv[c];
+                }
                 __syncwarp();
-                store_chunk(&tmY, out0p + b * kFStageOut, out0 + b * kFStageOut, r, srow, rn32,
-                            lane, n0 + c * 32, m0 + q * 32);
+                if constexpr (BF16)
+                    store_chunk_bf16(&tmY, out0p + b * kFStageOut, out0 + b * kFStageOut, r0, r1,
+                                     srow, rn_w, lane, n0 + c * kCW, m0 + q * 32);
+                else
+                    store_chunk(&tmY, out0p + b * kFStageOut, out0 + b * kFStageOut, r0, srow,
+                                rn_w, lane, n0 + c * kCW, m0 + q * 32);
                 ++u;
             }
         }
@@ -358,8 +352,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
 }  // namespace
 
 cudaError_t launch_gemm_fused_a4(const uint8_t *xc, const uint16_t *lut_a, const uint16_t *B16,
-                                 const float *s, const float *rn, float *y, int T, int N, int d,
-                                 cudaStream_t st, int num_sms, std::string *why) {
+                                 const float *s, const float *rn, void *y, bool y_bf16, int T,
+                                 int N, int d, cudaStream_t st, int num_sms, std::string *why) {
     auto fn = tensor_map_encoder();
     if (!fn) {
         *why = "cuTensorMapEncodeTiled unavailable";
@@ -373,7 +367,7 @@ cudaError_t launch_gemm_fused_a4(const uint8_t *xc, const uint16_t *lut_a, const
     if (fn(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(B16), dims, strides,
            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
-        !make_out_map(&my, y, T, N)) {
+        !make_out_map(&my, y, T, N, y_bf16)) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
@@ -381,18 +375,18 @@ cudaError_t launch_gemm_fused_a4(const uint8_t *xc, const uint16_t *lut_a, const
     cudaError_t e = cudaSuccess;
     {
         static std::mutex mu;
-        static bool done[kMaxDevices] = {};
+        static bool done[kMaxDevices][2] = {};
         int dev = 0;
         e = cudaGetDevice(&dev);
         if (e == cudaSuccess && (dev < 0 || dev >= kMaxDevices))
             e = cudaErrorInvalidDevice;
         if (e == cudaSuccess) {
             std::lock_guard<std::mutex> lk(mu);
-            if (!done[dev]) {
-                e = cudaFuncSetAttribute(k2_gemm_fused,
+            if (!done[dev][y_bf16]) {
+                e = cudaFuncSetAttribute(y_bf16 ? k2_gemm_fused<true> : k2_gemm_fused<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
-                done[dev] = (e == cudaSuccess);
+                done[dev][y_bf16] = (e == cudaSuccess);
             }
         }
         if (e != cudaSuccess) {
@@ -408,18 +402,16 @@ cudaError_t launch_gemm_fused_a4(const uint8_t *xc, const uint16_t *lut_a, const
     fp.N = N;
     fp.K = d;
     fp.inv_d = 1.0f / (float)d;
-    auto bytes4 = [&](int i0, bool hi) {
-        uint32_t w = 0;
-        for (int k = 0; k < 4; ++k)
-            w |= (uint32_t)((lut_a[i0 + k] >> (hi ? 8 : 0)) & 0xffu) << (8 * k);
-        return w;
-    };
-    fp.magL0 = bytes4(8, false);
-    fp.magL1 = bytes4(12, false);
-    fp.magH0 = bytes4(8, true);
-    fp.magH1 = bytes4(12, true);
+    if (!decode8_sources(lut_a, &fp.magL0, &fp.magL1, &fp.magH0, &fp.magH1)) {
+        *why = "k2_gemm_fused: activation codebook is not odd-symmetric";
+        return cudaErrorInvalidValue;
+    }
     const int tiles = ((N + FTN - 1) / FTN) * ((T + FBM - 1) / FBM);
-    k2_gemm_fused<<<tiles < num_sms ? tiles : num_sms, kFThreads, smem, st>>>(mb, my, fp);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    if (y_bf16)
+        k2_gemm_fused<true><<<grid, kFThreads, smem, st>>>(mb, my, fp);
+    else
+        k2_gemm_fused<false><<<grid, kFThreads, smem, st>>>(mb, my, fp);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         *why = "k2_gemm_fused launch";

@@ -6,9 +6,9 @@
 // speed-caveat paragraph notes that non-uniform centroids cannot feed integer tensor cores,
 // which is why the codes are decoded to fp16 unit centroids before the MMA.
 //
-// Path: (1) decode prepass: packed codes -> fp16 unit-variance centroids (LUT), for the
-// activation codes and the weight codes, into stream-ordered workspace; (2) a hand-written
-// persistent tcgen05 GEMM: TMA (128B swizzle) brings fp16 K-major tiles into a 4-stage
+// Path: (1) decode prepass (k2_decode.cu): packed codes -> fp16 unit-variance centroids, for
+// the activation codes and the weight codes, into stream-ordered workspace; (2) this file's
+// hand-written persistent tcgen05 GEMM: TMA (128B swizzle) brings fp16 K-major tiles into a 4-stage
 // shared-memory ring, one elected thread issues tcgen05.mma kind::f16 (M=128, N=256, K=16)
 // into one of two TMEM fp32 accumulators (2 x 256 columns), and 4 epilogue warps read the
 // other accumulator back with tcgen05.ld, apply the s_t * rn_o / d scale and hand 32 x 32
@@ -49,95 +49,6 @@ enum : unsigned {
 };
 
 // ------------------------------------------------------------------------------------------
-// Decode prepass: packed codes -> fp16 unit centroids.  A thread handles groups of 8 codes
-// (BITS bytes in, 16 bytes out); consecutive lanes take consecutive groups, so a warp reads
-// 32*BITS contiguous bytes and writes 512 contiguous bytes per group round, and each thread
-// keeps kDecUnroll independent groups in flight.  The lookup goes through a shared table
-// indexed by whole groups of codes (a byte holds 2 codes at b = 4 and 4 codes at b = 2;
-// 6 bits hold 2 codes at b = 3), so one shared load yields 2 or 4 fp16 values.
-// ------------------------------------------------------------------------------------------
-struct DecodeParams {
-    const uint8_t *codes;
-    uint16_t *out;
-    long long groups;           // rows * d / 8
-    uint16_t lut[256];
-};
-
-constexpr int kDecThreads = 256;
-constexpr int kDecUnroll = 4;
-
-template <int BITS>
-__device__ __forceinline__ uint4 decode_group(const uint32_t *tab32, uint64_t v) {
-    uint32_t o[4];
-    if constexpr (BITS == 2) {                        // 2 bytes, 4 codes each -> uint2 entries
-        const uint2 *t = reinterpret_cast<const uint2 *>(tab32);
-        const uint2 a = t[v & 0xffu], b = t[(v >> 8) & 0xffu];
-        o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
-    } else if constexpr (BITS == 3) {                 // 4 pairs of 6 bits
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            o[q] = tab32[(v >> (6 * q)) & 63u];
-    } else if constexpr (BITS == 4) {                 // 4 bytes, 2 codes each
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            o[q] = tab32[(v >> (8 * q)) & 0xffu];
-    } else {                                          // 8 bytes, 1 code each (fp16 entries)
-        const uint16_t *t = reinterpret_cast<const uint16_t *>(tab32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            o[q] = (uint32_t)t[(v >> (16 * q)) & 0xffu] |
-                   ((uint32_t)t[(v >> (16 * q + 8)) & 0xffu] << 16);
-    }
-    return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-template <int BITS>
-__device__ __forceinline__ uint64_t load_group(const uint8_t *codes, long long g) {
-    const uint8_t *src = codes + g * BITS;
-    if constexpr (BITS == 2)
-        return __ldg(reinterpret_cast<const unsigned short *>(src));
-    else if constexpr (BITS == 4)
-        return __ldg(reinterpret_cast<const unsigned int *>(src));
-    else if constexpr (BITS == 8)
-        return __ldg(reinterpret_cast<const unsigned long long *>(src));
-    else
-        return (uint64_t)__ldg(src) | ((uint64_t)__ldg(src + 1) << 8) |
-               ((uint64_t)__ldg(src + 2) << 16);
-}
-
-template <int BITS>
-__global__ void __launch_bounds__(kDecThreads) k2_decode(const __grid_constant__ DecodeParams p) {
-    // b=2: 256 entries of 4 fp16 (uint2); b=3: 64 entries of 2 fp16; b=4: 256 of 2; b=8: 256 of 1
-    constexpr int PER = BITS == 2 ? 4 : (BITS == 8 ? 1 : 2);      // codes per lookup
-    constexpr int IDX_BITS = PER * BITS;
-    constexpr int ENTRIES = 1 << IDX_BITS;
-    __shared__ __align__(16) uint16_t tab[ENTRIES * PER < 512 ? 512 : ENTRIES * PER];
-    for (int e = threadIdx.x; e < ENTRIES; e += blockDim.x)
-#pragma unroll
-        for (int i = 0; i < PER; ++i)
-            tab[e * PER + i] = p.lut[(e >> (i * BITS)) & ((1 << BITS) - 1)];
-    __syncthreads();
-    const uint32_t *tab32 = reinterpret_cast<const uint32_t *>(tab);
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    uint4 *out = reinterpret_cast<uint4 *>(p.out);
-    for (long long g0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; g0 < p.groups;
-         g0 += kDecUnroll * stride) {
-        uint64_t v[kDecUnroll];
-#pragma unroll
-        for (int j = 0; j < kDecUnroll; ++j) {
-            const long long g = g0 + j * stride;
-            v[j] = g < p.groups ? load_group<BITS>(p.codes, g) : 0;
-        }
-#pragma unroll
-        for (int j = 0; j < kDecUnroll; ++j) {
-            const long long g = g0 + j * stride;
-            if (g < p.groups)
-                out[g] = decode_group<BITS>(tab32, v[j]);
-        }
-    }
-}
-
-// ------------------------------------------------------------------------------------------
 // Persistent tcgen05 GEMM on fp16 operands decoded by the prepass.
 // ------------------------------------------------------------------------------------------
 constexpr uint32_t kIdesc = idesc_f16(BM, BN);
@@ -156,7 +67,7 @@ constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kStageOut = 32 * 32 * 4;                        // one 32 x 32 fp32 output chunk
 constexpr size_t kGemmSmem = 1024 + (size_t)STAGES * STAGE_BYTES +
                              (size_t)kEpiWarps * 2 * kStageOut + 8 * (2 * STAGES + 5) + 8 +
-                             kEpiWarps * 32 * sizeof(float) + 64;
+                             kEpiWarps * 64 * sizeof(float) + 64;
 static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
 
 // Persistent, warp-specialised tcgen05 GEMM.  Warp 0 lane 0: TMA producer over a 4-stage
@@ -164,7 +75,9 @@ static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
 // (TMEM lane quarter = warp % 4), each with two 4 KB output staging buffers that TMA tensor
 // stores drain to global memory.  Two 256-column accumulators alternate between tiles, so the
 // epilogue of one tile overlaps the mainloop of the next.  Tiles are walked n-fastest so
-// consecutive CTAs share the same 128-row A block in L2.
+// consecutive CTAs share the same 128-row A block in L2.  BF16: y is bf16 (32 x 64 chunks)
+// instead of fp32 (32 x 32 chunks).
+template <bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     k2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
@@ -181,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto tempty_bar = [&](int a) { return bars + 8u * (2 * STAGES + 2 + a); };
     const uint32_t drain_bar = bars + 8u * (2 * STAGES + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain_bar + 8u - base));
-    float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][32]
+    float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][64]
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -287,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- epilogue: TMEM -> registers -> scale -> smem -> TMA store -------
         // No cross-warp barrier: one warp giving up a wait cannot strand the others.
         const int q = warp & 3;                               // TMEM lane quarter
-        float *rn32 = rn_s + (warp - 2) * 32;
+        float *rn_w = rn_s + (warp - 2) * 64;
         const uint32_t out0 = sOut + (uint32_t)((warp - 2) * 2 * kStageOut);
         unsigned char *out0p = basep + (out0 - base);
         uint32_t u = 0;                                       // chunks stored so far
@@ -313,20 +226,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t t_base =
                 tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
             const bool rows_in = m0 + q * 32 < p.M;
+            constexpr int kCW = BF16 ? 64 : 32;               // columns per stored chunk
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_base + (uint32_t)(c * 32), r);
-                if (!rows_in || n0 + c * 32 >= p.N)
+            for (int c = 0; c < BN / kCW; ++c) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(t_base + (uint32_t)(c * kCW), r0);
+                if constexpr (BF16)
+                    tmem_ld32(t_base + (uint32_t)(c * kCW + 32), r1);
+                if (!rows_in || n0 + c * kCW >= p.N)
                     continue;                                 // box wholly outside y
                 const uint32_t b = u & 1;
                 if (lane == 0)
                     bulk_wait_read<1>();                      // the store that used buffer b
                 __syncwarp();
-                rn32[lane] = rnv[c];
+                if constexpr (BF16) {
+                    rn_w[lane] = rnv[2 * c];
+                    rn_w[32 + lane] = rnv[2 * c + 1];
+                } else {
+                    rn_w[lane] = rnv[c];
+                }
                 __syncwarp();
-                store_chunk(&tmY, out0p + b * kStageOut, out0 + b * kStageOut, r, srow, rn32,
-                            lane, n0 + c * 32, m0 + q * 32);
+                if constexpr (BF16)
+                    store_chunk_bf16(&tmY, out0p + b * kStageOut, out0 + b * kStageOut, r0, r1,
+                                     srow, rn_w, lane, n0 + c * kCW, m0 + q * 32);
+                else
+                    store_chunk(&tmY, out0p + b * kStageOut, out0 + b * kStageOut, r0, srow,
+                                rn_w, lane, n0 + c * kCW, m0 + q * 32);
                 ++u;
             }
             tc_fence_before();
@@ -366,36 +291,6 @@ bool make_map(CUtensorMap *map, const void *ptr, long long rows, int K, int box_
     return r == CUDA_SUCCESS;
 }
 
-template <int BITS>
-cudaError_t decode(const uint8_t *codes, uint16_t *out, long long rows, int d,
-                   const uint16_t *lut, cudaStream_t st, int num_sms) {
-    DecodeParams dp;
-    dp.codes = codes;
-    dp.out = out;
-    dp.groups = rows * (d / 8);
-    for (int i = 0; i < 256; ++i)
-        dp.lut[i] = lut[i];
-    long long blocks = (dp.groups + kDecThreads - 1) / kDecThreads;
-    const long long cap = (long long)num_sms * (2048 / kDecThreads);   // one resident wave
-    if (blocks > cap)
-        blocks = cap;
-    if (blocks < 1)
-        blocks = 1;
-    k2_decode<BITS><<<(unsigned)blocks, kDecThreads, 0, st>>>(dp);
-    return cudaGetLastError();
-}
-
-cudaError_t decode_any(int bits, const uint8_t *codes, uint16_t *out, long long rows, int d,
-                       const uint16_t *lut, cudaStream_t st, int num_sms) {
-    switch (bits) {
-        case 2: return decode<2>(codes, out, rows, d, lut, st, num_sms);
-        case 3: return decode<3>(codes, out, rows, d, lut, st, num_sms);
-        case 4: return decode<4>(codes, out, rows, d, lut, st, num_sms);
-        case 8: return decode<8>(codes, out, rows, d, lut, st, num_sms);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
@@ -414,17 +309,19 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-bool make_out_map(CUtensorMap *map, float *y, int T, int N) {
+bool make_out_map(CUtensorMap *map, void *y, int T, int N, bool bf16) {
     auto fn = tensor_map_encoder();
     if (!fn)
         return false;
+    const int esize = bf16 ? 2 : 4;
     cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)T};
-    cuuint64_t strides[1] = {(cuuint64_t)N * 4};
-    cuuint32_t box[2] = {32, 32};
+    cuuint64_t strides[1] = {(cuuint64_t)N * esize};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 32};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -434,39 +331,31 @@ size_t linear_workspace_bytes(int T, int d, int N) {
 
 size_t linear_workspace_b_offset(int T, int d) { return align_up((size_t)T * d * 2, 1024); }
 
-cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long long rows, int d,
-                          const uint16_t *lut, cudaStream_t st, int num_sms, std::string *why) {
-    cudaError_t e = decode_any(bits, codes, out, rows, d, lut, st, num_sms);
-    if (e != cudaSuccess)
-        *why = "decode launch";
-    return e;
-}
-
 cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s,
-                        const float *rn, float *y, int T, int N, int d, cudaStream_t st,
-                        int num_sms, std::string *why) {
+                        const float *rn, void *y, bool y_bf16, int T, int N, int d,
+                        cudaStream_t st, int num_sms, std::string *why) {
     CUtensorMap ma, mb, my;
     if (!make_map(&ma, A16, T, d, BM) || !make_map(&mb, B16, N, d, BN) ||
-        !make_out_map(&my, y, T, N)) {
+        !make_out_map(&my, y, T, N, y_bf16)) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
     const size_t smem = kGemmSmem;
     cudaError_t e = cudaSuccess;
     {
-        // once per device
+        // once per device and output type
         static std::mutex mu;
-        static bool done[kMaxDevices] = {};
+        static bool done[kMaxDevices][2] = {};
         int dev = 0;
         e = cudaGetDevice(&dev);
         if (e == cudaSuccess && (dev < 0 || dev >= kMaxDevices))
             e = cudaErrorInvalidDevice;
         if (e == cudaSuccess) {
             std::lock_guard<std::mutex> lk(mu);
-            if (!done[dev]) {
-                e = cudaFuncSetAttribute(k2_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-                done[dev] = (e == cudaSuccess);
+            if (!done[dev][y_bf16]) {
+                e = cudaFuncSetAttribute(y_bf16 ? k2_gemm<true> : k2_gemm<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                done[dev][y_bf16] = (e == cudaSuccess);
             }
         }
         if (e != cudaSuccess) {
@@ -482,7 +371,11 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s
     gp.K = d;
     gp.inv_d = 1.0f / (float)d;
     const int tiles = ((N + BN - 1) / BN) * ((T + BM - 1) / BM);
-    k2_gemm<<<tiles < num_sms ? tiles : num_sms, kThreads, smem, st>>>(ma, mb, my, gp);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    if (y_bf16)
+        k2_gemm<true><<<grid, kThreads, smem, st>>>(ma, mb, my, gp);
+    else
+        k2_gemm<false><<<grid, kThreads, smem, st>>>(ma, mb, my, gp);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         *why = "k2_gemm launch";

@@ -598,8 +598,8 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     if (ca->d != d || cw->d != d)
         return fail(OQ_EINVAL, "%s: d = %d but codebooks have d = %d / %d", who, d, ca->d,
                     cw->d);
-    if (out_dtype != OQ_F32)
-        return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32", who);
+    if (out_dtype != OQ_F32 && out_dtype != OQ_BF16)
+        return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32 or OQ_BF16", who);
     if (T < 0 || out_features < 1 || out_features % 16 != 0)
         return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
                                "multiple of 16", who, T, out_features);
@@ -639,8 +639,8 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
         });
         if (e == cudaSuccess)
             e = timed(OQ_KERNEL_GEMM, st, [&] {
-                return oq::launch_gemm_fused_a4(x_codes, ca->lut, B16, s, row_norms,
-                                                static_cast<float *>(y), T, out_features, d, st,
+                return oq::launch_gemm_fused_a4(x_codes, ca->lut, B16, s, row_norms, y,
+                                                out_dtype == OQ_BF16, T, out_features, d, st,
                                                 di->sms, &why);
             });
     } else {
@@ -657,7 +657,7 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
             });
         if (e == cudaSuccess)
             e = timed(OQ_KERNEL_GEMM, st, [&] {
-                return oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T,
+                return oq::launch_gemm(A16, B16, s, row_norms, y, out_dtype == OQ_BF16, T,
                                        out_features, d, st, di->sms, &why);
             });
     }
@@ -680,8 +680,8 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
     if (ca->d != d || cw->d != d)
         return fail(OQ_EINVAL, "%s: d = %d but codebooks have d = %d / %d", who, d, ca->d,
                     cw->d);
-    if (out_dtype != OQ_F32)
-        return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32", who);
+    if (out_dtype != OQ_F32 && out_dtype != OQ_BF16)
+        return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32 or OQ_BF16", who);
     if (T < 0 || out_features < 1 || out_features % 16 != 0)
         return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
                                "multiple of 16", who, T, out_features);
@@ -719,7 +719,7 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
         e = oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st, di->sms,
                               &why);
     if (e == cudaSuccess)
-        e = oq::launch_gemm(A16, B16, s, row_norms, static_cast<float *>(y), T, out_features,
+        e = oq::launch_gemm(A16, B16, s, row_norms, y, out_dtype == OQ_BF16, T, out_features,
                             d, st, di->sms, &why);
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());

@@ -5,16 +5,18 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <cstdint>
 
 namespace oq {
 
 // Host side (k2_linear.cu): the driver's tensor-map encoder, looked up once through the
-// runtime (nullptr if unavailable), and the output map of y: fp32 [T, N] row-major in
-// 32 x 32 boxes with 128-byte swizzle, the layout store_chunk() writes.
+// runtime (nullptr if unavailable), and the output map of y [T, N] row-major with 128-byte
+// swizzle: fp32 in 32 x 32 boxes (the layout store_chunk writes) or bf16 in 32-row x
+// 64-column boxes (store_chunk_bf16).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
-bool make_out_map(CUtensorMap *map, float *y, int T, int N);
+bool make_out_map(CUtensorMap *map, void *y, int T, int N, bool bf16);
 
 namespace sm100 {
 
@@ -213,6 +215,39 @@ __device__ __forceinline__ void store_chunk(const CUtensorMap *map, unsigned cha
         o.y = __uint_as_float(acc[4 * k + 1]) * srow * rn4.y;
         o.z = __uint_as_float(acc[4 * k + 2]) * srow * rn4.z;
         o.w = __uint_as_float(acc[4 * k + 3]) * srow * rn4.w;
+        rowp[k ^ (lane & 7)] = o;
+    }
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(map, stage, x, y);
+        bulk_commit();
+    }
+}
+
+// bf16 variant: 32 rows x 64 columns (two 32-column accumulator loads acc0, acc1), each
+// value scaled by srow * rn64[j] in fp32 and rounded to nearest-even bf16; same staging
+// layout (a row is 64 bf16 = 128 bytes) and issue rules as store_chunk.
+__device__ __forceinline__ void store_chunk_bf16(const CUtensorMap *map, unsigned char *stage_ptr,
+                                                 uint32_t stage, const uint32_t (&acc0)[32],
+                                                 const uint32_t (&acc1)[32], float srow,
+                                                 const float *rn64, int lane, int x, int y) {
+    uint4 *rowp = reinterpret_cast<uint4 *>(stage_ptr + lane * 128);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {                       // 16-byte piece k = columns 8k .. 8k+7
+        const float4 ra = reinterpret_cast<const float4 *>(rn64)[2 * k];
+        const float4 rb = reinterpret_cast<const float4 *>(rn64)[2 * k + 1];
+        const uint32_t *a = (k < 4) ? &acc0[8 * k] : &acc1[8 * (k - 4)];
+        auto pk = [&](uint32_t u0, float r0, uint32_t u1, float r1) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(u0) * srow * r0,
+                                                          __uint_as_float(u1) * srow * r1);
+            return *reinterpret_cast<const uint32_t *>(&h);
+        };
+        uint4 o;
+        o.x = pk(a[0], ra.x, a[1], ra.y);
+        o.y = pk(a[2], ra.z, a[3], ra.w);
+        o.z = pk(a[4], rb.x, a[5], rb.y);
+        o.w = pk(a[6], rb.z, a[7], rb.w);
         rowp[k ^ (lane & 7)] = o;
     }
     fence_async_smem();

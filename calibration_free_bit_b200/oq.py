@@ -199,14 +199,23 @@ def oq_quantize_act(r: RPBH, ca: Codebook, x: torch.Tensor, x_codes=None, s=None
     return x_codes, s
 
 
-def oq_linear(ca: Codebook, cw: Codebook, x_codes: torch.Tensor, s: torch.Tensor,
-              W_codes: torch.Tensor, row_norms: torch.Tensor, y=None, stream=None):
-    """Codebook linear layer: y fp32 [T, out] = s_t rn_o sum_k ca[xc] cw[wc]."""
-    T, N, d = x_codes.shape[0], W_codes.shape[0], ca.d
+def _out(y, T, N, out_dtype, device):
     if y is None:
-        y = torch.empty((T, N), dtype=torch.float32, device=x_codes.device)
+        return torch.empty((T, N), dtype=out_dtype, device=device)
+    if y.dtype not in (torch.float32, torch.bfloat16) or tuple(y.shape) != (T, N):
+        raise ValueError(f"y must be fp32 or bf16 of shape {(T, N)}")
+    return y
+
+
+def oq_linear(ca: Codebook, cw: Codebook, x_codes: torch.Tensor, s: torch.Tensor,
+              W_codes: torch.Tensor, row_norms: torch.Tensor, y=None, stream=None,
+              out_dtype=torch.float32):
+    """Codebook linear layer: y [T, out] = s_t rn_o sum_k ca[xc] cw[wc], fp32 or bf16 (the
+    dtype of y when given, else out_dtype)."""
+    T, N, d = x_codes.shape[0], W_codes.shape[0], ca.d
+    y = _out(y, T, N, out_dtype, x_codes.device)
     _check(lib().oq_linear(ca.handle, cw.handle, _ptr(x_codes), _ptr(s), _ptr(W_codes),
-                           _ptr(row_norms), T, d, N, _ptr(y), OQ_F32, _stream(stream)))
+                           _ptr(row_norms), T, d, N, _ptr(y), _dtype_code(y), _stream(stream)))
     return y
 
 
@@ -216,8 +225,10 @@ def oq_linear_noalloc(ca: Codebook, cw: Codebook, x_codes: torch.Tensor, s: torc
     """oq_linear with the library's fixed workspace: the caller passes y; nothing is
     allocated on the device (see include/oq.h for the size limit and sharing rules)."""
     T, N, d = x_codes.shape[0], W_codes.shape[0], ca.d
+    y = _out(y, T, N, None, x_codes.device)
     _check(lib().oq_linear_noalloc(ca.handle, cw.handle, _ptr(x_codes), _ptr(s), _ptr(W_codes),
-                                   _ptr(row_norms), T, d, N, _ptr(y), OQ_F32, _stream(stream)))
+                                   _ptr(row_norms), T, d, N, _ptr(y), _dtype_code(y),
+                                   _stream(stream)))
     return y
 
 

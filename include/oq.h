@@ -113,7 +113,9 @@ int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int 
  * which equals the quantized W x because W R^T R x = W x ([RCAP] rotation-cancellation
  * paragraph; the fused low-bit GEMM is the speed caveat paragraph's missing piece).
  * x_codes: device [T, d*ba/8]; s: device fp32 [T]; W_codes: device [out_features, d*bw/8];
- * row_norms: device fp32 [out_features]; y: device [T, out_features] of out_dtype (OQ_F32).
+ * row_norms: device fp32 [out_features]; y: device [T, out_features] of out_dtype: OQ_F32,
+ * or OQ_BF16 (the fp32 epilogue value s*rn/d*acc rounded to nearest even; adds up to 2^-9
+ * relative error per element on top of the fp32 result).
  * Centroids enter the tensor cores as fp16 unit-variance values; accumulation is fp32.
  * Both code operands are decoded into fp16 buffers first.  With 4-bit activation codes
  * and the environment variable OQ_LINEAR_PATH=fused (read once per process), the activation

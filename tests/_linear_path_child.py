@@ -1,7 +1,7 @@
 """Child process for the oq_linear path test: OQ_LINEAR_PATH is read once per process, so the
 opt-in fused 4-bit path is exercised in a process of its own.  Checks oq_linear on uniform
-random codes (every centroid used, ragged M and N tails) against the fp64 oracle and exits
-non-zero on any failure."""
+random codes (every centroid used, ragged M and N tails) against the fp64 oracle, and the bf16
+output against the fp32 output rounded to nearest even; exits non-zero on any failure."""
 import os
 import sys
 
@@ -31,7 +31,15 @@ def main():
                              torch.from_numpy(s.astype(np.float32)).cuda(),
                              torch.from_numpy(wc).cuda(),
                              torch.from_numpy(rn.astype(np.float32)).cuda())
+            y16 = oq.oq_linear(ca, cw, torch.from_numpy(xc).cuda(),
+                               torch.from_numpy(s.astype(np.float32)).cuda(),
+                               torch.from_numpy(wc).cuda(),
+                               torch.from_numpy(rn.astype(np.float32)).cuda(),
+                               out_dtype=torch.bfloat16)
             oq.oq_check()
+            if not torch.equal(y.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16)):
+                print(f"FAIL bf16 output ba={ba} bw={bw} T={T} N={N} d={d}")
+                return 1
             got = y.cpu().double().numpy()
             ref = O.linear(xc, s, wc, rn, d, ba, bw)
             err = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))

@@ -26,6 +26,7 @@ CODE_MATCH = 0.9999
 BOUNDARY_TOL = 1e-5        # in sigma units (unit-codebook units)
 NORM_RTOL = 5e-6
 LINEAR_RTOL = 1e-3
+BF16_REL = 2.0 ** -9       # round-to-nearest bf16: relative error bound per element
 
 
 @pytest.fixture(scope="module")
@@ -297,3 +298,39 @@ def test_linear_path_selection(oq, path):
     r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
+
+
+@pytest.mark.parametrize("ba,bw", [(4, 4), (2, 8)])
+@pytest.mark.parametrize("T,N,d", [(200, 272, 384), (129, 784, 1024)])
+def test_linear_bf16_output(oq, ba, bw, T, N, d):
+    """out_dtype bf16: every element is the fp32 result rounded to nearest even (the same
+    epilogue arithmetic), so bf16(y_f32) == y_bf16 bit for bit, and the oracle bound widens by
+    at most the rounding bound 2^-9."""
+    rng = np.random.default_rng(T + 3 * N + ba)
+    xc = O.pack(rng.integers(0, 1 << ba, (T, d)).astype(np.uint8), ba)
+    wc = O.pack(rng.integers(0, 1 << bw, (N, d)).astype(np.uint8), bw)
+    s = rng.uniform(0.1, 50.0, T)
+    rn = rng.uniform(0.5, 2.0, N)
+    ca, cw = oq.oq_lloyd_max(d, ba), oq.oq_lloyd_max(d, bw)
+    args = [torch.from_numpy(xc).cuda(), torch.from_numpy(s.astype(np.float32)).cuda(),
+            torch.from_numpy(wc).cuda(), torch.from_numpy(rn.astype(np.float32)).cuda()]
+    y32 = oq.oq_linear(ca, cw, *args)
+    y16 = oq.oq_linear(ca, cw, *args, out_dtype=torch.bfloat16)
+    oq.oq_check()
+    assert y16.dtype == torch.bfloat16
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+    ref = O.linear(xc, s, wc, rn, d, ba, bw)
+    assert rel_l2(y16.cpu().double().numpy(), ref) <= LINEAR_RTOL + BF16_REL
+
+
+def test_linear_bf16_output_full_size(oq):
+    """The attention projection at full size with bf16 y: bit-identical to rounding the fp32
+    output of the same call."""
+    p = synth.get("flux_attn_w4a4")[0]
+    r, ca, cw = handles(oq, p.d, p.h, p.bits_a, p.bits_w)
+    xc, s = oq.oq_quantize_act(r, ca, synth.activations(p).cuda())
+    wc, rn = oq.oq_quantize_weight(r, cw, synth.weight(p).cuda())
+    y32 = oq.oq_linear(ca, cw, xc, s, wc, rn)
+    y16 = oq.oq_linear(ca, cw, xc, s, wc, rn, out_dtype=torch.bfloat16)
+    oq.oq_check()
+    assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))

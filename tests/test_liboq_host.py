@@ -119,11 +119,14 @@ def test_validation_rejects_bad_arguments_without_a_gpu():
     # T = 0 is a no-op that succeeds without touching a device
     assert L.oq_quantize_act(r.handle, ca.handle, None, oq.OQ_BF16, 0, 3072, None, None,
                              None) == oq.OQ_OK
-    # linear: out_features not a multiple of 16, bf16 output, d mismatch
+    # linear: out_features not a multiple of 16, unknown output type, d mismatch
     assert L.oq_linear(ca.handle, ca.handle, fake, fake, fake, fake, 8, 3072, 100, fake,
                        oq.OQ_F32, None) == oq.OQ_EINVAL
     assert L.oq_linear(ca.handle, ca.handle, fake, fake, fake, fake, 8, 3072, 128, fake,
-                       oq.OQ_BF16, None) == oq.OQ_EINVAL
+                       2, None) == oq.OQ_EINVAL
+    assert b"out_dtype" in L.oq_last_error()
+    assert L.oq_linear(ca.handle, ca.handle, None, None, None, None, 0, 3072, 128, None,
+                       oq.OQ_BF16, None) == oq.OQ_OK
     assert L.oq_linear(ca.handle, c_other.handle, fake, fake, fake, fake, 8, 3072, 128, fake,
                        oq.OQ_F32, None) == oq.OQ_EINVAL
     assert L.oq_linear(ca.handle, ca.handle, None, None, None, None, 0, 3072, 128, None,
