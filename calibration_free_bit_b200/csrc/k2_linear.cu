@@ -20,6 +20,7 @@
 
 #include <mutex>
 
+#include "decode4.cuh"
 #include "oq_internal.h"
 #include "sm100_common.cuh"
 
@@ -49,50 +50,75 @@ enum : unsigned {
 };
 
 // ------------------------------------------------------------------------------------------
-// Persistent tcgen05 GEMM on fp16 operands decoded by the prepass.
+// Persistent tcgen05 GEMM.  The B operand (fp16 weight centroids from the prepass) always
+// comes in by TMA.  The A operand either comes in by TMA as well (fp16 activation centroids
+// from the prepass), or, for 4-bit activation codes of a symmetric codebook (ACODES), four
+// decoder warps read the packed codes and write the fp16 A tile into the same shared-memory
+// ring, in the layout TMA would have produced.
 // ------------------------------------------------------------------------------------------
 constexpr uint32_t kIdesc = idesc_f16(BM, BN);
 
 struct GemmParams {
     const float *s;
     const float *rn;
+    uint32_t L0, L1, H0, H1;    // ACODES: decode8 sources of the activation codebook
     int M, N, K;
     float inv_d;
 };
 
-constexpr int kThreads = 192;        // 6 warps
 constexpr int kEpiWarps = 4;         // warps 2..5
+constexpr int kDecWarps = 8;         // ACODES: warps 6..13, two per TMEM lane quarter
 constexpr int kAccCols = BN;         // one fp32 accumulator: 256 TMEM columns
 constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kStageOut = 32 * 32 * 4;                        // one 32 x 32 fp32 output chunk
-constexpr size_t kGemmSmem = 1024 + (size_t)STAGES * STAGE_BYTES +
-                             (size_t)kEpiWarps * 2 * kStageOut + 8 * (2 * STAGES + 5) + 8 +
-                             kEpiWarps * 64 * sizeof(float) + 64;
-static_assert(kGemmSmem <= 227 * 1024, "shared memory budget");
+constexpr int kCodeStageBytes = BM * BK / 2;                  // ACODES: 128 rows x 32 bytes
+constexpr int kNumBars = 3 * STAGES + 5;
+
+// ACODES keeps one output staging buffer per epilogue warp (room for the code stages).
+template <bool ACODES>
+__host__ __device__ constexpr int out_bufs() { return ACODES ? 1 : 2; }
+
+template <bool ACODES>
+__host__ __device__ constexpr size_t gemm_smem() {
+    return 1024 + (size_t)STAGES * (STAGE_BYTES + (ACODES ? kCodeStageBytes : 0)) +
+           (size_t)kEpiWarps * out_bufs<ACODES>() * kStageOut + 8 * kNumBars + 8 +
+           kEpiWarps * 64 * sizeof(float) + 64;
+}
+static_assert(gemm_smem<false>() <= 227 * 1024 && gemm_smem<true>() <= 227 * 1024,
+              "shared memory budget");
+
+template <bool ACODES>
+__host__ __device__ constexpr int gemm_threads() { return 32 * (2 + kEpiWarps + (ACODES ? kDecWarps : 0)); }
 
 // Persistent, warp-specialised tcgen05 GEMM.  Warp 0 lane 0: TMA producer over a 4-stage
 // shared-memory ring.  Warp 1: TMEM owner; its lane 0 issues the MMAs.  Warps 2..5: epilogue
-// (TMEM lane quarter = warp % 4), each with two 4 KB output staging buffers that TMA tensor
-// stores drain to global memory.  Two 256-column accumulators alternate between tiles, so the
-// epilogue of one tile overlaps the mainloop of the next.  Tiles are walked n-fastest so
-// consecutive CTAs share the same 128-row A block in L2.  BF16: y is bf16 (32 x 64 chunks)
-// instead of fp32 (32 x 32 chunks).
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+// (TMEM lane quarter = warp % 4), each with 4 KB output staging buffers that TMA tensor
+// stores drain to global memory.  ACODES: tmA maps the packed codes (uint8 [M, K/2], 32 x 128
+// byte boxes), TMA brings each stage's code tile in with its B tile, and warps 6..9 decode the
+// codes of rows (warp % 4) * 32 + lane into the stage's A tile (warps 6..9 the first 32 codes
+// of each row and k-block, warps 10..13 the last 32).  Two 256-column accumulators alternate between
+// tiles, so the epilogue of one tile overlaps the mainloop of the next.  Tiles are walked
+// n-fastest so consecutive CTAs share the same 128-row A block in L2.  BF16: y is bf16
+// (32 x 64 chunks) instead of fp32 (32 x 32 chunks).
+template <bool BF16, bool ACODES>
+__global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
     k2_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
             const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;                 // 1 KB aligned tiles
     unsigned char *basep = smem_raw + (base - raw);
+    constexpr int kOutBufs = out_bufs<ACODES>();
     const uint32_t sA = base, sB = base + STAGES * A_STAGE_BYTES;
-    const uint32_t sOut = sB + STAGES * B_STAGE_BYTES;            // [4 warps][2][4 KB]
-    const uint32_t bars = sOut + kEpiWarps * 2 * kStageOut;
-    auto full_bar = [&](int s) { return bars + 8u * s; };
-    auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
-    auto tfull_bar = [&](int a) { return bars + 8u * (2 * STAGES + a); };
-    auto tempty_bar = [&](int a) { return bars + 8u * (2 * STAGES + 2 + a); };
-    const uint32_t drain_bar = bars + 8u * (2 * STAGES + 4);
+    const uint32_t sC = sB + STAGES * B_STAGE_BYTES;              // ACODES: code stages
+    const uint32_t sOut = sC + (ACODES ? STAGES * kCodeStageBytes : 0);   // [4][bufs][4 KB]
+    const uint32_t bars = sOut + kEpiWarps * kOutBufs * kStageOut;
+    auto full_bar = [&](int s) { return bars + 8u * s; };                   // TMA bytes
+    auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };       // MMA done
+    auto afull_bar = [&](int s) { return bars + 8u * (2 * STAGES + s); };   // ACODES: A
+    auto tfull_bar = [&](int a) { return bars + 8u * (3 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bars + 8u * (3 * STAGES + 2 + a); };
+    const uint32_t drain_bar = bars + 8u * (3 * STAGES + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain_bar + 8u - base));
     float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][64]
     __shared__ int abort_flag;
@@ -106,6 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
+            mbar_init(afull_bar(s), kDecWarps);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
@@ -145,8 +172,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (aborted())
                         break;
-                    mbar_expect_tx(full_bar(s), STAGE_BYTES);
-                    tma_load_2d(sA + s * A_STAGE_BYTES, &tmA, kb * BK, m0, full_bar(s));
+                    if constexpr (ACODES) {
+                        mbar_expect_tx(full_bar(s), B_STAGE_BYTES + kCodeStageBytes);
+                        tma_load_2d(sC + s * kCodeStageBytes, &tmA, kb * (BK / 2), m0,
+                                    full_bar(s));
+                    } else {
+                        mbar_expect_tx(full_bar(s), STAGE_BYTES);
+                        tma_load_2d(sA + s * A_STAGE_BYTES, &tmA, kb * BK, m0, full_bar(s));
+                    }
                     tma_load_2d(sB + s * B_STAGE_BYTES, &tmB, kb * BK, n0, full_bar(s));
                 }
             }
@@ -174,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool ok = true;
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = it % STAGES;
-                    if (!mbar_wait(full_bar(s), (it / STAGES) & 1)) {
+                    if (!mbar_wait(full_bar(s), (it / STAGES) & 1) ||
+                        (ACODES && !mbar_wait(afull_bar(s), (it / STAGES) & 1))) {
                         give_up(ERR_WAIT_FULL);
                         ok = false;
                         break;
@@ -196,12 +230,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(drain_bar, 0))
                 atomicOr(&g_k2_err, ERR_WAIT_ACCUM);
         }
-    } else {
+    } else if (warp < 2 + kEpiWarps) {
         // ---------------- epilogue: TMEM -> registers -> scale -> smem -> TMA store -------
         // No cross-warp barrier: one warp giving up a wait cannot strand the others.
         const int q = warp & 3;                               // TMEM lane quarter
         float *rn_w = rn_s + (warp - 2) * 64;
-        const uint32_t out0 = sOut + (uint32_t)((warp - 2) * 2 * kStageOut);
+        const uint32_t out0 = sOut + (uint32_t)((warp - 2) * kOutBufs * kStageOut);
         unsigned char *out0p = basep + (out0 - base);
         uint32_t u = 0;                                       // chunks stored so far
         int i = 0;
@@ -235,9 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(t_base + (uint32_t)(c * kCW + 32), r1);
                 if (!rows_in || n0 + c * kCW >= p.N)
                     continue;                                 // box wholly outside y
-                const uint32_t b = u & 1;
+                const uint32_t b = kOutBufs == 2 ? (u & 1) : 0;
                 if (lane == 0)
-                    bulk_wait_read<1>();                      // the store that used buffer b
+                    bulk_wait_read<kOutBufs - 1>();           // the store that used buffer b
                 __syncwarp();
                 if constexpr (BF16) {
                     rn_w[lane] = rnv[2 * c];
@@ -261,6 +295,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0)
             bulk_wait_all();
+    } else if constexpr (ACODES) {
+        // ---------------- activation decoders: 4-bit codes -> fp16 A stages ----------------
+        // Thread = row r of the 128-row tile and one half of its 64 codes per k-block: it reads
+        // 16 bytes of codes from the stage's code tile and writes 64 bytes of the fp16 row in
+        // the 128-byte swizzled layout (16-byte piece k at piece k ^ (r % 8) of the row; 8-row
+        // atoms of 1024 bytes), which is what a TMA load of the decoded operand would have
+        // written.  The stage's full barrier also means the MMA has released its A tile.
+        const int r = (warp & 3) * 32 + lane;
+        const int half = (warp - 2 - kEpiWarps) >> 2;        // which 32 codes of the 64
+        const uint32_t row_off = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+        unsigned char *sAp = basep + (sA - base);
+        const unsigned char *sCp = basep + (sC - base);
+        uint32_t it = 0;
+        bool stop = false;
+        for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % STAGES;
+                const bool ok = mbar_wait(full_bar(s), (it / STAGES) & 1);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0)
+                        give_up(ERR_WAIT_FULL);
+                    stop = true;
+                    break;
+                }
+                if (__shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0)) {
+                    stop = true;
+                    break;
+                }
+                const uint4 c = *reinterpret_cast<const uint4 *>(
+                    sCp + s * kCodeStageBytes + r * (BK / 2) + half * 16);
+                const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+                unsigned char *dst = sAp + s * A_STAGE_BYTES + row_off;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int k = half * 4 + j;               // 16-byte piece of the row
+                    uint32_t o[4];
+                    decode8(words[j], p.L0, p.L1, p.H0, p.H1, o);
+                    *reinterpret_cast<uint4 *>(dst + ((k ^ (r & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                fence_async_smem();                           // visible to the tensor core
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(afull_bar(s));
+            }
+        }
     }
     __syncwarp();
     tc_fence_before();
@@ -331,55 +411,86 @@ size_t linear_workspace_bytes(int T, int d, int N) {
 
 size_t linear_workspace_b_offset(int T, int d) { return align_up((size_t)T * d * 2, 1024); }
 
-cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s,
-                        const float *rn, void *y, bool y_bf16, int T, int N, int d,
-                        cudaStream_t st, int num_sms, std::string *why) {
-    CUtensorMap ma, mb, my;
-    if (!make_map(&ma, A16, T, d, BM) || !make_map(&mb, B16, N, d, BN) ||
-        !make_out_map(&my, y, T, N, y_bf16)) {
-        *why = "cuTensorMapEncodeTiled failed";
-        return cudaErrorInvalidValue;
-    }
-    const size_t smem = kGemmSmem;
-    cudaError_t e = cudaSuccess;
-    {
-        // once per device and output type
-        static std::mutex mu;
-        static bool done[kMaxDevices][2] = {};
-        int dev = 0;
-        e = cudaGetDevice(&dev);
-        if (e == cudaSuccess && (dev < 0 || dev >= kMaxDevices))
-            e = cudaErrorInvalidDevice;
-        if (e == cudaSuccess) {
-            std::lock_guard<std::mutex> lk(mu);
-            if (!done[dev][y_bf16]) {
-                e = cudaFuncSetAttribute(y_bf16 ? k2_gemm<true> : k2_gemm<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-                done[dev][y_bf16] = (e == cudaSuccess);
-            }
+namespace {
+
+// 4-bit codes, uint8 [rows, K/2] row-major -> 128-row x 32-byte boxes (one k-block), no
+// swizzle.
+bool make_code_map(CUtensorMap *map, const uint8_t *codes, long long rows, int K) {
+    auto fn = tensor_map_encoder();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K / 2, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K / 2};
+    cuuint32_t box[2] = {(cuuint32_t)(BK / 2), (cuuint32_t)BM};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool BF16, bool ACODES>
+cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const CUtensorMap &my,
+                          const GemmParams &gp, int grid, cudaStream_t st, std::string *why) {
+    auto kern = k2_gemm<BF16, ACODES>;
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess && (dev < 0 || dev >= kMaxDevices))
+        e = cudaErrorInvalidDevice;
+    if (e == cudaSuccess) {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!done[dev]) {        // once per device and instantiation
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gemm_smem<ACODES>());
+            done[dev] = (e == cudaSuccess);
         }
-        if (e != cudaSuccess) {
-            *why = "cudaFuncSetAttribute(k2_gemm)";
-            return e;
-        }
     }
-    GemmParams gp;
-    gp.s = s;
-    gp.rn = rn;
-    gp.M = T;
-    gp.N = N;
-    gp.K = d;
-    gp.inv_d = 1.0f / (float)d;
-    const int tiles = ((N + BN - 1) / BN) * ((T + BM - 1) / BM);
-    const int grid = tiles < num_sms ? tiles : num_sms;
-    if (y_bf16)
-        k2_gemm<true><<<grid, kThreads, smem, st>>>(ma, mb, my, gp);
-    else
-        k2_gemm<false><<<grid, kThreads, smem, st>>>(ma, mb, my, gp);
+    if (e != cudaSuccess) {
+        *why = "cudaFuncSetAttribute(k2_gemm)";
+        return e;
+    }
+    kern<<<grid, gemm_threads<ACODES>(), gemm_smem<ACODES>(), st>>>(ma, mb, my, gp);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         *why = "k2_gemm launch";
     return e;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
+                        const uint16_t *B16, const float *s, const float *rn, void *y,
+                        bool y_bf16, int T, int N, int d, cudaStream_t st, int num_sms,
+                        std::string *why) {
+    const bool acodes = A16 == nullptr;
+    GemmParams gp;
+    gp.s = s;
+    gp.rn = rn;
+    gp.L0 = gp.L1 = gp.H0 = gp.H1 = 0;
+    gp.M = T;
+    gp.N = N;
+    gp.K = d;
+    gp.inv_d = 1.0f / (float)d;
+    if (acodes && (!x_codes4 || !lut_a ||
+                   !decode8_sources(lut_a, &gp.L0, &gp.L1, &gp.H0, &gp.H1))) {
+        *why = "k2_gemm: activation codes need a 4-bit odd-symmetric codebook";
+        return cudaErrorInvalidValue;
+    }
+    CUtensorMap ma, mb, my;
+    const bool a_ok = acodes ? make_code_map(&ma, x_codes4, T, d) : make_map(&ma, A16, T, d, BM);
+    if (!a_ok || !make_map(&mb, B16, N, d, BN) || !make_out_map(&my, y, T, N, y_bf16)) {
+        *why = "cuTensorMapEncodeTiled failed";
+        return cudaErrorInvalidValue;
+    }
+    const int tiles = ((N + BN - 1) / BN) * ((T + BM - 1) / BM);
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    if (acodes)
+        return y_bf16 ? launch_gemm_t<true, true>(ma, mb, my, gp, grid, st, why)
+                      : launch_gemm_t<false, true>(ma, mb, my, gp, grid, st, why);
+    return y_bf16 ? launch_gemm_t<true, false>(ma, mb, my, gp, grid, st, why)
+                  : launch_gemm_t<false, false>(ma, mb, my, gp, grid, st, why);
 }
 
 size_t noalloc_workspace_bytes() { return kNoAllocWorkspaceBytes; }

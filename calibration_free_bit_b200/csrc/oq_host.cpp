@@ -443,8 +443,9 @@ cudaMemPool_t device_pool(int dev, DeviceInfo *di, int *rc) {
     return pool;
 }
 
-// OQ_LINEAR_PATH=fused sends 4-bit activation codes straight into the GEMM kernel that
-// decodes them itself (read once per process); the default decodes both operands first.
+// OQ_LINEAR_PATH=fused decodes 4-bit activation codes inside the GEMM kernel instead of in
+// the prepass (read once per process): no [T, d] fp16 workspace, but each 128-row tile of
+// codes is decoded once per 256-column tile of the output.
 bool fused_requested() {
     static const bool v = [] {
         const char *e = std::getenv("OQ_LINEAR_PATH");
@@ -619,9 +620,9 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     cudaMemPool_t pool = device_pool(dev, di, &rc);
     if (!pool)
         return rc;
-    // Default: both operands decoded to fp16 by the prepass, then the TMA/tcgen05 GEMM.
-    // OQ_LINEAR_PATH=fused with 4-bit activation codes: the codes are decoded inside the GEMM
-    // (only the weights get a prepass).
+    // Both operands decoded to fp16 by the prepass, then the TMA/tcgen05 GEMM; with
+    // OQ_LINEAR_PATH=fused, 4-bit activation codes are decoded inside the GEMM kernel and only
+    // the weight codes get the prepass.
     const bool fused = ca->bits == 4 && fused_requested();
     const size_t ws_bytes = fused ? (size_t)out_features * d * 2
                                   : oq::linear_workspace_bytes(T, d, out_features);
@@ -631,36 +632,25 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     if (e != cudaSuccess)
         return fail_cuda(e, "oq_linear: workspace allocation");
     std::string why;
-    if (fused) {
-        uint16_t *B16 = static_cast<uint16_t *>(ws);
+    uint16_t *A16 = nullptr, *B16 = static_cast<uint16_t *>(ws);
+    if (!fused) {
+        A16 = static_cast<uint16_t *>(ws);
+        B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
+                                           oq::linear_workspace_b_offset(T, d));
+        e = timed(OQ_KERNEL_DECODE, st, [&] {
+            return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
+        });
+    }
+    if (e == cudaSuccess)
         e = timed(OQ_KERNEL_DECODE, st, [&] {
             return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
                                      di->sms, &why);
         });
-        if (e == cudaSuccess)
-            e = timed(OQ_KERNEL_GEMM, st, [&] {
-                return oq::launch_gemm_fused_a4(x_codes, ca->lut, B16, s, row_norms, y,
-                                                out_dtype == OQ_BF16, T, out_features, d, st,
-                                                di->sms, &why);
-            });
-    } else {
-        uint16_t *A16 = static_cast<uint16_t *>(ws);
-        uint16_t *B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
-                                                     oq::linear_workspace_b_offset(T, d));
-        e = timed(OQ_KERNEL_DECODE, st, [&] {
-            return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
+    if (e == cudaSuccess)
+        e = timed(OQ_KERNEL_GEMM, st, [&] {
+            return oq::launch_gemm(A16, x_codes, ca->lut, B16, s, row_norms, y,
+                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why);
         });
-        if (e == cudaSuccess)
-            e = timed(OQ_KERNEL_DECODE, st, [&] {
-                return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
-                                         di->sms, &why);
-            });
-        if (e == cudaSuccess)
-            e = timed(OQ_KERNEL_GEMM, st, [&] {
-                return oq::launch_gemm(A16, B16, s, row_norms, y, out_dtype == OQ_BF16, T,
-                                       out_features, d, st, di->sms, &why);
-            });
-    }
     cudaError_t e2 = cudaFreeAsync(ws, st);
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());
@@ -719,8 +709,8 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
         e = oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st, di->sms,
                               &why);
     if (e == cudaSuccess)
-        e = oq::launch_gemm(A16, B16, s, row_norms, y, out_dtype == OQ_BF16, T, out_features,
-                            d, st, di->sms, &why);
+        e = oq::launch_gemm(A16, nullptr, nullptr, B16, s, row_norms, y, out_dtype == OQ_BF16, T,
+                            out_features, d, st, di->sms, &why);
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());
     return OQ_OK;
@@ -731,18 +721,15 @@ int oq_check(void *stream) {
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess)
         return fail_cuda(e, "oq_check: stream synchronize");
-    unsigned w1 = 0, w2 = 0, w3 = 0;
+    unsigned w1 = 0, w2 = 0;
     if ((e = oq::read_and_clear_k1_error(&w1, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k1 error word");
     if ((e = oq::read_and_clear_k2_error(&w2, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k2 error word");
-    if ((e = oq::read_and_clear_k2f_error(&w3, st)) != cudaSuccess)
-        return fail_cuda(e, "oq_check: read fused k2 error word");
-    if (w1 || w2 || w3)
-        return fail(OQ_EDEVICE, "device error word: quantize=0x%x linear=0x%x fused=0x%x "
-                                "(a bounded wait gave up; quantize bit 1 = row copy, linear "
-                                "bits 1/2/4 = stage/slot/accumulator, fused bits 1/2/4/8 = "
-                                "weight stage/activation stage/slot/accumulator)", w1, w2, w3);
+    if (w1 || w2)
+        return fail(OQ_EDEVICE, "device error word: quantize=0x%x linear=0x%x (a bounded wait "
+                                "gave up; quantize bit 1 = row copy, linear bits 1/2/4 = "
+                                "operand stage/ring slot/accumulator)", w1, w2);
     return OQ_OK;
 }
 

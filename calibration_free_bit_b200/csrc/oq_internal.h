@@ -53,18 +53,14 @@ size_t linear_workspace_b_offset(int T, int d);
 cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long long rows, int d,
                           const uint16_t *lut, cudaStream_t st, int num_sms, std::string *why);
 
-// y[T, N] = (s_t rn_o / d) * A16[T, d] . B16[N, d]^T   (fp16 x fp16 -> fp32 in TMEM)
+// y[T, N] = (s_t rn_o / d) * A[T, d] . B16[N, d]^T   (fp16 x fp16 -> fp32 in TMEM)
+// A is A16 (fp16 centroids from the prepass) or, when A16 is null, x_codes4: 4-bit codes of
+// the codebook whose fp16 LUT is lut_a (must be odd-symmetric), decoded inside the kernel.
 // y is fp32, or bf16 (round to nearest even of the fp32 epilogue value) when y_bf16.
-cudaError_t launch_gemm(const uint16_t *A16, const uint16_t *B16, const float *s,
-                        const float *rn, void *y, bool y_bf16, int T, int N, int d,
-                        cudaStream_t st, int num_sms, std::string *why);
-
-// Codebook GEMM with the 4-bit activation codes decoded inside the kernel into tensor memory
-// (k2_fused.cu); B16 is the fp16 weight operand from the decode prepass.  No A workspace.
-cudaError_t launch_gemm_fused_a4(const uint8_t *xc, const uint16_t *lut_a, const uint16_t *B16,
-                                 const float *s, const float *rn, void *y, bool y_bf16, int T,
-                                 int N, int d, cudaStream_t st, int num_sms, std::string *why);
-cudaError_t read_and_clear_k2f_error(unsigned *out, cudaStream_t st);
+cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
+                        const uint16_t *B16, const float *s, const float *rn, void *y,
+                        bool y_bf16, int T, int N, int d, cudaStream_t st, int num_sms,
+                        std::string *why);
 
 // Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
 // its size, and its address on the current device (looked up once per device).

@@ -117,10 +117,11 @@ int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int 
  * or OQ_BF16 (the fp32 epilogue value s*rn/d*acc rounded to nearest even; adds up to 2^-9
  * relative error per element on top of the fp32 result).
  * Centroids enter the tensor cores as fp16 unit-variance values; accumulation is fp32.
- * Both code operands are decoded into fp16 buffers first.  With 4-bit activation codes
- * and the environment variable OQ_LINEAR_PATH=fused (read once per process), the activation
- * codes are instead decoded inside the GEMM kernel and only the weight codes get an fp16
- * buffer.  Either way the temporary device memory is stream-ordered, from a library-owned
+ * Both code operands are decoded into fp16 buffers first.  With 4-bit activation codes and
+ * the environment variable OQ_LINEAR_PATH=fused (read once per process), the activation codes
+ * are instead decoded inside the GEMM kernel, into its shared-memory operand tiles, and only
+ * the weight codes get an fp16 buffer (less device memory, more decode work per call).
+ * Either way the temporary device memory is stream-ordered, from a library-owned
  * pool.  Errors: as above, plus OQ_ECUDA if the pool allocation fails. */
 int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
               const float *s, const uint8_t *W_codes, const float *row_norms, int T, int d,

@@ -1,5 +1,5 @@
-"""Child process for the oq_linear path test: OQ_LINEAR_PATH is read once per process, so the
-opt-in fused 4-bit path is exercised in a process of its own.  Checks oq_linear on uniform
+"""Child process for the oq_linear path test: OQ_LINEAR_PATH is read once per process, so each
+path for 4-bit activation codes (in-GEMM decode, prepass) is exercised in a process of its own.  Checks oq_linear on uniform
 random codes (every centroid used, ragged M and N tails) against the fp64 oracle, and the bf16
 output against the fp32 output rounded to nearest even; exits non-zero on any failure."""
 import os

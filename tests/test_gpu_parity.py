@@ -284,9 +284,9 @@ def test_linear_video_ffn_up_full_size(oq, variant):
 
 @pytest.mark.parametrize("path", ["fused", "default"])
 def test_linear_path_selection(oq, path):
-    """Both oq_linear paths for 4-bit activation codes (the decode prepass and, with
-    OQ_LINEAR_PATH=fused, the GEMM that decodes activation codes itself) against the oracle;
-    each runs in a child process because the variable is read once per process."""
+    """Both oq_linear paths for 4-bit activation codes (the fp16 prepass by default; decoded
+    inside the GEMM with OQ_LINEAR_PATH=fused) against the oracle; each runs in a child
+    process because the variable is read once per process."""
     import os
     import subprocess
     import sys
