@@ -257,6 +257,161 @@ double orc_gauss_mse(int levels, const double *centroids, const double *bounds)
 }
 
 /* ---------------------------------------------------------------------------------------
+ * Exact marginal f_d.  A coordinate X of a uniform unit vector in R^d has
+ * P(|X| <= r) = I_{r^2}(1/2, (d-1)/2) (X^2 ~ Beta(1/2, (d-1)/2)), density
+ * (1 - x^2)^((d-3)/2) / B(1/2, (d-1)/2), and first moment over a cell in closed form:
+ * int_a^b x f_d(x) dx = ((1 - a^2)^((d-1)/2) - (1 - b^2)^((d-1)/2)) / ((d-1) B(1/2, (d-1)/2)).
+ * [RCAP] change-of-basis paragraph; the f3 variant of the codebook.
+ * ------------------------------------------------------------------------------------- */
+
+/* Continued fraction of I_x(a, b): I_x(a, b) = x^a (1-x)^b / (a B(a, b) F) with
+ * F = 1 + d1 / (1 + d2 / (1 + ...)), d_{2m+1} = -(a+m)(a+b+m)x / ((a+2m)(a+2m+1)),
+ * d_{2m} = m(b-m)x / ((a+2m-1)(a+2m)).  Returns F; converges quickly for
+ * x < (a+1)/(a+b+2). */
+static double betacf(double a, double b, double x)
+{
+    /* modified Lentz evaluation of F */
+    const double tiny = 1e-300;
+    double f = 1.0, C = 1.0, D = 0.0;
+    int n;
+    for (n = 1; n <= 100000; ++n) {
+        int m = n / 2;
+        double dn;
+        if (n % 2 == 1)
+            dn = -(a + m) * (a + b + m) * x / ((a + 2.0 * m) * (a + 2.0 * m + 1.0));
+        else
+            dn = m * (b - m) * x / ((a + 2.0 * m - 1.0) * (a + 2.0 * m));
+        D = 1.0 + dn * D;
+        if (fabs(D) < tiny)
+            D = tiny;
+        D = 1.0 / D;
+        C = 1.0 + dn / C;
+        if (fabs(C) < tiny)
+            C = tiny;
+        f *= C * D;
+        if (fabs(C * D - 1.0) < 1e-16)
+            break;
+    }
+    return f;
+}
+
+double orc_betainc(double a, double b, double x)
+{
+    double lfront;
+    if (x <= 0.0)
+        return 0.0;
+    if (x >= 1.0)
+        return 1.0;
+    lfront = lgamma(a + b) - lgamma(a) - lgamma(b) + a * log(x) + b * log1p(-x);
+    if (x < (a + 1.0) / (a + b + 2.0))
+        return exp(lfront) / (a * betacf(a, b, x));
+    return 1.0 - exp(lfront) / (b * betacf(b, a, 1.0 - x));
+}
+
+static double log_beta_half(int d)   /* log B(1/2, (d-1)/2) */
+{
+    double b = 0.5 * (d - 1);
+    return lgamma(0.5) + lgamma(b) - lgamma(0.5 + b);
+}
+
+double orc_sphere_density(int d, double x)
+{
+    if (x <= -1.0 || x >= 1.0)
+        return (d == 3 && fabs(x) == 1.0) ? 0.5 : 0.0;
+    return exp(0.5 * (d - 3) * log1p(-x * x) - log_beta_half(d));
+}
+
+double orc_sphere_cdf(int d, double x)
+{
+    double half;
+    if (x <= -1.0)
+        return 0.0;
+    if (x >= 1.0)
+        return 1.0;
+    half = 0.5 * orc_betainc(0.5, 0.5 * (d - 1), x * x);   /* P(0 <= X <= |x|) */
+    return x >= 0.0 ? 0.5 + half : 0.5 - half;
+}
+
+/* P(|X| >= r) for r >= 0, without the cancellation of 1 - cdf. */
+static double sphere_upper(int d, double r)
+{
+    if (r >= 1.0)
+        return 0.0;
+    return 0.5 * orc_betainc(0.5 * (d - 1), 0.5, 1.0 - r * r);   /* I_{1-r^2}(b, 1/2) / 2 */
+}
+
+
+
+int orc_lloyd_max_sphere(int d, int bits, double tol, int max_iter,
+                         double *centroids, double *bounds, int *iters, double *residual)
+{
+    int L, i, it;
+    double *t, *up, *g;
+    double sd, k1, norm, move = INFINITY;
+    if (d < 3 || bits < 1 || bits > 12 || !centroids || !bounds)
+        return -1;
+    L = 1 << bits;
+    sd = 1.0 / sqrt((double)d);
+    k1 = 0.5 * (d - 1);
+    norm = (d - 1) * exp(log_beta_half(d));
+    t = (double *)malloc(sizeof(double) * (size_t)(3 * (L + 1)));
+    if (!t)
+        return -2;
+    up = t + (L + 1);     /* P(|X| >= |t_i|) at every boundary */
+    g = up + (L + 1);     /* (1 - t_i^2)^((d-1)/2) at every boundary */
+    /* Start: the Gaussian companding start scaled to the standard deviation 1/sqrt(d) and
+     * squashed into (-1, 1).  f_d is log-concave for d >= 3, so the optimum is unique. */
+    for (i = 0; i < L; ++i)
+        centroids[i] = tanh(sqrt(3.0) * normal_quantile((i + 0.5) / L) * sd);
+    t[0] = -1.0;
+    t[L] = 1.0;
+    for (it = 0; it < max_iter; ++it) {
+        /* condition 1: boundaries at the midpoints of neighbouring centroids */
+        for (i = 1; i < L; ++i)
+            t[i] = 0.5 * (centroids[i - 1] + centroids[i]);
+        /* tail and first-moment term at every boundary, shared by the two cells there */
+        for (i = 0; i <= L; ++i) {
+            up[i] = sphere_upper(d, fabs(t[i]));
+            g[i] = fabs(t[i]) >= 1.0 ? 0.0 : exp(k1 * log1p(-t[i] * t[i]));
+        }
+        /* condition 2: centroid = E[X | cell] = first moment / probability */
+        move = 0.0;
+        for (i = 0; i < L; ++i) {
+            double a = t[i], b = t[i + 1], P;
+            if (a >= 0.0)
+                P = up[i] - up[i + 1];
+            else if (b <= 0.0)
+                P = up[i + 1] - up[i];
+            else
+                P = 1.0 - up[i] - up[i + 1];
+            double c = (g[i] - g[i + 1]) / norm / P;
+            double dm = fabs(c - centroids[i]);
+            if (dm > move)
+                move = dm;
+            centroids[i] = c;
+        }
+        for (i = 0; i < L / 2; ++i) {
+            double m = 0.5 * (centroids[L - 1 - i] - centroids[i]);
+            centroids[i] = -m;
+            centroids[L - 1 - i] = m;
+        }
+        move /= sd;
+        if (move <= tol) {
+            ++it;
+            break;
+        }
+    }
+    for (i = 1; i < L; ++i)
+        bounds[i - 1] = 0.5 * (centroids[i - 1] + centroids[i]);
+    if (iters)
+        *iters = it;
+    if (residual)
+        *residual = move;
+    free(t);
+    return move <= tol ? 0 : 1;
+}
+
+/* ---------------------------------------------------------------------------------------
  * Nearest centroid and packing.  [RCAP] pseudocode "nearest_centroid(...)".  The boundary
  * count with "<=" sends an exact tie to the upper cell (a reading).
  * ------------------------------------------------------------------------------------- */

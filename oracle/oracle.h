@@ -66,6 +66,25 @@ int orc_lloyd_max_gauss(int bits, double tol, int max_iter,
 /* Mean squared error of a quantizer (centroids, bounds) under N(0,1), in closed form. */
 double orc_gauss_mse(int levels, const double *centroids, const double *bounds);
 
+/* Regularized incomplete beta function I_x(a, b) for a, b > 0, 0 <= x <= 1, by its
+ * continued fraction (evaluated where it converges fast, else through
+ * I_x(a, b) = 1 - I_{1-x}(b, a)). */
+double orc_betainc(double a, double b, double x);
+
+/* The exact marginal of one coordinate of a uniformly random unit vector in R^d ([RCAP]
+ * change-of-basis paragraph: "one fixed marginal that depends only on the dimension d"):
+ * f_d(x) = (1 - x^2)^((d-3)/2) / B(1/2, (d-1)/2) on [-1, 1], d >= 3.
+ * orc_sphere_cdf(d, x) = P(X <= x); orc_sphere_density(d, x) = f_d(x). */
+double orc_sphere_cdf(int d, double x);
+double orc_sphere_density(int d, double x);
+
+/* Lloyd-Max quantizer with 2^bits levels for f_d (same two conditions and stopping rule as
+ * orc_lloyd_max_gauss; tol is in units of the standard deviation 1/sqrt(d)).  Centroids and
+ * bounds are in the coordinate's own units (inside [-1, 1]); multiplied by sqrt(d) they are
+ * the unit codebook the quantizer compares against.  d >= 3. */
+int orc_lloyd_max_sphere(int d, int bits, double tol, int max_iter,
+                         double *centroids, double *bounds, int *iters, double *residual);
+
 /* Nearest-centroid code of v against sigma-scaled unit boundaries:
  * code = #{ j : sigma * t_j <= v }. */
 int orc_code_of(double v, int levels, const double *unit_bounds, double sigma);

@@ -41,6 +41,15 @@ def lib():
                                           C.POINTER(C.c_int), C.POINTER(C.c_double)]
         L.orc_gauss_mse.restype = C.c_double
         L.orc_gauss_mse.argtypes = [C.c_int, _f64p, _f64p]
+        L.orc_betainc.restype = C.c_double
+        L.orc_betainc.argtypes = [C.c_double, C.c_double, C.c_double]
+        L.orc_sphere_cdf.restype = C.c_double
+        L.orc_sphere_cdf.argtypes = [C.c_int, C.c_double]
+        L.orc_sphere_density.restype = C.c_double
+        L.orc_sphere_density.argtypes = [C.c_int, C.c_double]
+        L.orc_lloyd_max_sphere.restype = C.c_int
+        L.orc_lloyd_max_sphere.argtypes = [C.c_int, C.c_int, C.c_double, C.c_int, _f64p,
+                                           _f64p, C.POINTER(C.c_int), C.POINTER(C.c_double)]
         L.orc_code_of.restype = C.c_int
         L.orc_code_of.argtypes = [C.c_double, C.c_int, _f64p, C.c_double]
         L.orc_pack.restype = None
@@ -118,17 +127,56 @@ def lloyd_max(bits: int, tol: float = 4e-14, max_iter: int = 2_000_000):
     return c, t, it.value, res.value
 
 
+def betainc(a: float, b: float, x: float) -> float:
+    """Regularized incomplete beta I_x(a, b) (continued fraction)."""
+    return lib().orc_betainc(a, b, x)
+
+
+def sphere_cdf(d: int, x: float) -> float:
+    """CDF of one coordinate of a uniform unit vector in R^d."""
+    return lib().orc_sphere_cdf(d, x)
+
+
+def sphere_density(d: int, x: float) -> float:
+    """f_d(x) = (1 - x^2)^((d-3)/2) / B(1/2, (d-1)/2) on [-1, 1]."""
+    return lib().orc_sphere_density(d, x)
+
+
+def lloyd_max_sphere(d: int, bits: int, tol: float = 1e-12, max_iter: int = 2_000_000):
+    """Lloyd-Max quantizer for the exact marginal f_d, in the coordinate's own units:
+    (centroids[L], bounds[L-1], iters, residual); residual in units of 1/sqrt(d)."""
+    L = 1 << bits
+    c = np.empty(L, dtype=np.float64)
+    t = np.empty(L - 1, dtype=np.float64)
+    it = C.c_int(0)
+    res = C.c_double(0.0)
+    lib().orc_lloyd_max_sphere(d, bits, tol, max_iter, c, t, C.byref(it), C.byref(res))
+    return c, t, it.value, res.value
+
+
 _CB_CACHE = {}
 
 
-def codebook(bits: int):
-    """Cached unit codebook (centroids, bounds) for `bits`."""
-    if bits not in _CB_CACHE:
-        c, t, _, res = lloyd_max(bits)
-        if not res <= 1e-12:
-            raise RuntimeError(f"Lloyd-Max at {bits} bits did not converge: {res}")
-        _CB_CACHE[bits] = (c, t)
-    return _CB_CACHE[bits]
+def codebook(bits: int, marginal: str = "gauss", d: int = 0):
+    """Cached unit codebook (centroids, bounds) for `bits`: the N(0,1) Lloyd-Max quantizer
+    (marginal "gauss"), or sqrt(d) times the Lloyd-Max quantizer of the exact marginal f_d
+    (marginal "sphere"), so that both compare against sqrt(d) * x_rot / s."""
+    key = (bits, marginal, d if marginal == "sphere" else 0)
+    if key not in _CB_CACHE:
+        if marginal == "gauss":
+            c, t, _, res = lloyd_max(bits)
+            if not res <= 1e-12:
+                raise RuntimeError(f"Lloyd-Max at {bits} bits did not converge: {res}")
+        elif marginal == "sphere":
+            tol = 1e-12 if bits <= 4 else 1e-10   # plain Lloyd is slow at 256 levels
+            c, t, _, res = lloyd_max_sphere(d, bits, tol=tol)
+            if not res <= tol:
+                raise RuntimeError(f"f_d Lloyd-Max at d={d}, {bits} bits: {res}")
+            c, t = c * np.sqrt(d), t * np.sqrt(d)
+        else:
+            raise ValueError(marginal)
+        _CB_CACHE[key] = (c, t)
+    return _CB_CACHE[key]
 
 
 def gauss_mse(centroids, bounds) -> float:
@@ -166,12 +214,14 @@ def unpack(packed, n: int, bits: int) -> np.ndarray:
 
 # --- quantizers and the linear layer ------------------------------------------------------
 
-def quantize_rows(x, h: int, perm, sign, bits: int, eps: float, detail: bool = False):
+def quantize_rows(x, h: int, perm, sign, bits: int, eps: float, detail: bool = False,
+                  marginal: str = "gauss"):
     """[RCAP] pseudocode per-row quantizer.  Returns (packed codes, norms) and, with
-    detail=True, also (z, u) where u = (z/(s+eps)) * sqrt(d) in unit-codebook units."""
+    detail=True, also (z, u) where u = (z/(s+eps)) * sqrt(d) in unit-codebook units.
+    marginal: the codebook's target, "gauss" (N(0, 1/d)) or "sphere" (exact f_d)."""
     x = _f64(np.atleast_2d(x))
     rows, d = x.shape
-    _, t = codebook(bits)
+    _, t = codebook(bits, marginal, d)
     packed = np.empty((rows, d * bits // 8), dtype=np.uint8)
     norms = np.empty(rows, dtype=np.float64)
     z = np.empty_like(x) if detail else None
@@ -186,20 +236,21 @@ def quantize_rows(x, h: int, perm, sign, bits: int, eps: float, detail: bool = F
     return packed, norms
 
 
-def quantize_act(x, h, perm, sign, bits, detail=False):
+def quantize_act(x, h, perm, sign, bits, detail=False, marginal="gauss"):
     """Online activation step: eps = EPS_ACT."""
-    return quantize_rows(x, h, perm, sign, bits, EPS_ACT, detail)
+    return quantize_rows(x, h, perm, sign, bits, EPS_ACT, detail, marginal)
 
 
-def quantize_weight(W, h, perm, sign, bits, detail=False):
+def quantize_weight(W, h, perm, sign, bits, detail=False, marginal="gauss"):
     """Offline weight step: no eps; rows of W are the 'tokens'."""
-    return quantize_rows(W, h, perm, sign, bits, 0.0, detail)
+    return quantize_rows(W, h, perm, sign, bits, 0.0, detail, marginal)
 
 
-def linear(x_packed, s, w_packed, rn, d: int, bits_a: int, bits_w: int) -> np.ndarray:
+def linear(x_packed, s, w_packed, rn, d: int, bits_a: int, bits_w: int,
+           marginal: str = "gauss") -> np.ndarray:
     """y[t,o] = s_t rn_o sum_k sigma ca[xc] sigma cw[wc], naive fp64 triple loop."""
-    ca, _ = codebook(bits_a)
-    cw, _ = codebook(bits_w)
+    ca, _ = codebook(bits_a, marginal, d)
+    cw, _ = codebook(bits_w, marginal, d)
     xp = np.ascontiguousarray(np.atleast_2d(x_packed), dtype=np.uint8)
     wp = np.ascontiguousarray(np.atleast_2d(w_packed), dtype=np.uint8)
     T, out = xp.shape[0], wp.shape[0]
