@@ -67,6 +67,16 @@ int orc_build_rpbh(int d, uint64_t seed, int32_t *perm, int8_t *sign)
     return 0;
 }
 
+int orc_build_block_rht(int d, uint64_t seed, int32_t *perm, int8_t *sign)
+{
+    int i, rc = orc_build_rpbh(d, seed, perm, sign);
+    if (rc != 0)
+        return rc;
+    for (i = 0; i < d; ++i)
+        perm[i] = i;
+    return 0;
+}
+
 /* ---------------------------------------------------------------------------------------
  * Rotation.  [RCAP] RPBH paragraph and pseudocode "x_rot = x @ rotation[d].T".
  * R = B D P with P the gather y[i] = x[perm[i]], D = diag(sign), B = blockdiag(H_h/sqrt h).

@@ -47,6 +47,11 @@ uint64_t orc_uniform_below(uint64_t *state, uint64_t n);
 /* RPBH tables: perm[d] (a bijection on 0..d-1) and sign[d] (+1/-1). Returns 0 on success. */
 int orc_build_rpbh(int d, uint64_t seed, int32_t *perm, int8_t *sign);
 
+/* Block-RHT tables, the ablation of [RCAP]'s results list ("removing the leading uniform
+ * permutation"): the RPBH tables of the same seed with perm replaced by the identity, so the
+ * sign flips and blocks are those of RPBH and only P differs (a reading). */
+int orc_build_block_rht(int d, uint64_t seed, int32_t *perm, int8_t *sign);
+
 /* Sylvester Hadamard matrix entry (-1)^popcount(i & j) as an integer. */
 int orc_hadamard_entry(int i, int j);
 

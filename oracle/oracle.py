@@ -32,6 +32,8 @@ def lib():
         L.orc_uniform_below.argtypes = [C.POINTER(C.c_uint64), C.c_uint64]
         L.orc_build_rpbh.restype = C.c_int
         L.orc_build_rpbh.argtypes = [C.c_int, C.c_uint64, _i32p, _i8p]
+        L.orc_build_block_rht.restype = C.c_int
+        L.orc_build_block_rht.argtypes = [C.c_int, C.c_uint64, _i32p, _i8p]
         L.orc_hadamard_entry.restype = C.c_int
         L.orc_hadamard_entry.argtypes = [C.c_int, C.c_int]
         L.orc_rotate_row.restype = C.c_int
@@ -92,6 +94,16 @@ def build_rpbh(d: int, seed: int):
     rc = lib().orc_build_rpbh(d, seed, perm, sign)
     if rc != 0:
         raise ValueError(f"orc_build_rpbh({d}) failed: {rc}")
+    return perm, sign
+
+
+def build_block_rht(d: int, seed: int):
+    """Block-RHT ablation: the RPBH tables of `seed` with the identity permutation."""
+    perm = np.empty(d, dtype=np.int32)
+    sign = np.empty(d, dtype=np.int8)
+    rc = lib().orc_build_block_rht(d, seed, perm, sign)
+    if rc != 0:
+        raise ValueError(f"orc_build_block_rht({d}) failed: {rc}")
     return perm, sign
 
 

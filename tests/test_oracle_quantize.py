@@ -150,8 +150,8 @@ def test_rotated_marginal_is_near_gaussian_statistical():
     adv = np.zeros((8, p.d))
     adv[:, : p.h] = rng.standard_normal((8, p.h))
     _, _, _, u_p = O.quantize_act(adv, p.h, perm, sign, 4, detail=True)
-    _, _, _, u_id = O.quantize_act(adv, p.h, np.arange(p.d, dtype=np.int32), sign, 4,
-                                   detail=True)
+    perm_id, sign_id = O.build_block_rht(p.d, 0)
+    _, _, _, u_id = O.quantize_act(adv, p.h, perm_id, sign_id, 4, detail=True)
     ks_p = stats.kstest(u_p.ravel(), "norm").statistic
     ks_id = stats.kstest(u_id.ravel(), "norm").statistic
     assert ks_p < 0.05 and ks_id > 0.4

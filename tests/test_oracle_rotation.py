@@ -102,3 +102,26 @@ def test_weight_rotation_cancels():
     W_rot = O.rotate(W, h, perm, sign)                # rows R w_o, i.e. W R^T
     x_rot = O.rotate(x, h, perm, sign)[0]
     np.testing.assert_allclose(W_rot @ x_rot, W @ x, rtol=0, atol=1e-12)
+
+
+def test_block_rht_tables_are_rpbh_without_the_permutation():
+    """Block-RHT (the ablation): identity permutation, the RPBH signs of the same seed."""
+    for d, seed in [(256, 0), (3072, 7)]:
+        perm, sign = O.build_rpbh(d, seed)
+        pid, sid = O.build_block_rht(d, seed)
+        assert np.array_equal(pid, np.arange(d))
+        assert np.array_equal(sid, sign)
+
+
+def test_block_rht_is_orthogonal_and_block_local():
+    """With P = I the rotation is blockdiag(H_h/sqrt h) D: orthogonal, and a vector supported
+    on one block of positions stays on that block."""
+    d, h = 256, 64
+    perm, sign = O.build_block_rht(d, 3)
+    R = np.stack([O.rotate(e, h, perm, sign)[0] for e in np.eye(d)], axis=1)
+    np.testing.assert_allclose(R @ R.T, np.eye(d), atol=1e-13)
+    x = np.zeros(d)
+    x[h:2 * h] = np.arange(1, h + 1)
+    z = O.rotate(x, h, perm, sign)[0]
+    assert np.all(z[:h] == 0) and np.all(z[2 * h:] == 0)
+    np.testing.assert_allclose(np.linalg.norm(z), np.linalg.norm(x), rtol=1e-14)
