@@ -25,7 +25,7 @@
 //     a = sat(z*K/(s+eps) + 1/2) (one FFMA.SAT), q = floor(a*2^23) via an fp32x2 add with
 //     round-down, word = table[q >> F], code = (word + q*G) >> 24.  The table words fold the
 //     cell's base code and its boundary, so the decision is exact in the fixed-point q grid
-//     (2^-23 of the grid span, < 1.2e-6 sigma).  Bit widths 2/3/4/8 pack LSB-first.
+//     (2^-23 of the grid span, < 1.2e-6 sigma).  Bit widths 2/3/4/6/8 pack LSB-first.
 //   * Every mbarrier wait is bounded (2 s of %globaltimer); a wait that gives up sets a bit
 //     in the device error word (read by oq_check) and the round's outputs are not written.
 #include <cuda_bf16.h>
@@ -170,8 +170,16 @@ __device__ __forceinline__ void store_words(uint8_t *dst, const uint32_t (&w)[NW
 // the NEXT round's two rows stream into a raw buffer while the current round computes from
 // the interleaved pair buffer.  fp32 input: rows are gathered straight from `stages` raw
 // buffers (2 when shared memory allows, else 1).
-template <int BITS, bool IN_F32, int H>
+// GELU in its erf form, x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2, in fp32 (CUDA's erff).
+__device__ __forceinline__ float gelu_erf(float x) {
+    return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+// GELU (bf16 input only): the kernel quantizes R * GELU(x) instead of R * x; GELU is applied
+// to each gathered element before its sign flip (it is elementwise, so it commutes with P).
+template <int BITS, bool IN_F32, int H, bool GELU = false>
 __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
+    static_assert(!(GELU && IN_F32), "fused GELU is bf16-only");
     constexpr int Q = H / kE;                        // threads per h-block
     constexpr bool REPL = (BITS <= 4);               // per-lane table copies (conflict-free)
     constexpr int TSH = REPL ? 7 : 2;                // table row stride: 32 lanes x 4 B, or 4 B
@@ -305,7 +313,13 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
                     const uint32_t en = en4[i];
                     const uint32_t sg = en & 0x80000000u;
                     const uint32_t off = en & 0x7fffffffu;
-                    if constexpr (!IN_F32) {
+                    if constexpr (GELU) {
+                        const uint32_t w = lds32(base0 + off);
+                        const float a = gelu_erf(__uint_as_float(w << 16));
+                        const float b = gelu_erf(__uint_as_float(w & 0xffff0000u));
+                        v[e].x = __uint_as_float(__float_as_uint(a) ^ sg);
+                        v[e].y = __uint_as_float(__float_as_uint(b) ^ sg);
+                    } else if constexpr (!IN_F32) {
                         const uint32_t w = lds32(base0 + off);
                         v[e].x = __uint_as_float((w << 16) + sg);
                         v[e].y = __uint_as_float((w ^ en) & 0xffff0000u);
@@ -385,7 +399,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             d0 = qb.x * G + lds32(tbl_lane + ((qb.x >> F) << TSH));
             d1 = qb.y * G + lds32(tbl_lane + ((qb.y >> F) << TSH));
         };
-        if constexpr (BITS == 3) {
+        if constexpr (BITS == 3 || BITS == 6) {
 #pragma unroll
             for (int i = 0; i < NW; ++i) {
                 w0[i] = 0;
@@ -473,7 +487,7 @@ cudaError_t k1_prepare(const void *kern, int threads, size_t smem, int *per_sm) 
     return cudaSuccess;
 }
 
-template <int BITS, bool F32>
+template <int BITS, bool F32, bool GELU = false>
 cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int threads, size_t smem,
                      int num_sms, cudaStream_t st, std::string *why) {
     auto go = [&](auto kern) -> cudaError_t {
@@ -493,12 +507,12 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
         return e;
     };
     switch (h) {
-        case 32: return go(k1_rotquant<BITS, F32, 32>);
-        case 64: return go(k1_rotquant<BITS, F32, 64>);
-        case 128: return go(k1_rotquant<BITS, F32, 128>);
-        case 256: return go(k1_rotquant<BITS, F32, 256>);
-        case 512: return go(k1_rotquant<BITS, F32, 512>);
-        case 1024: return go(k1_rotquant<BITS, F32, 1024>);
+        case 32: return go(k1_rotquant<BITS, F32, 32, GELU>);
+        case 64: return go(k1_rotquant<BITS, F32, 64, GELU>);
+        case 128: return go(k1_rotquant<BITS, F32, 128, GELU>);
+        case 256: return go(k1_rotquant<BITS, F32, 256, GELU>);
+        case 512: return go(k1_rotquant<BITS, F32, 512, GELU>);
+        case 1024: return go(k1_rotquant<BITS, F32, 1024, GELU>);
         default: *why = "unsupported h"; return cudaErrorInvalidValue;
     }
 }
@@ -540,6 +554,20 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     p.stages = stages;
     const int threads = NG * GT;
     const long long ctas_needed = (npairs + NG - 1) / NG;
+    if (p.gelu) {
+        if (in_f32) {
+            *why = "fused GELU takes bf16 input";
+            return cudaErrorInvalidValue;
+        }
+        switch (bits) {
+            case 2: return launch_h<2, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+            case 3: return launch_h<3, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+            case 4: return launch_h<4, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+            case 6: return launch_h<6, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+            case 8: return launch_h<8, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+            default: *why = "unsupported bit width"; return cudaErrorInvalidValue;
+        }
+    }
     switch (bits * 2 + (in_f32 ? 1 : 0)) {
         case 4: return launch_h<2, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
         case 5: return launch_h<2, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
@@ -547,6 +575,8 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
         case 7: return launch_h<3, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
         case 8: return launch_h<4, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
         case 9: return launch_h<4, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 12: return launch_h<6, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 13: return launch_h<6, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
         case 16: return launch_h<8, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
         case 17: return launch_h<8, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
         default: *why = "unsupported bit width"; return cudaErrorInvalidValue;

@@ -32,7 +32,13 @@ constexpr int kDecUnroll = 8;
 template <int BITS>
 __device__ __forceinline__ uint4 decode_group(const uint32_t *tab32, uint64_t v) {
     uint32_t o[4];
-    if constexpr (BITS == 2) {                        // 2 bytes, 4 codes each -> uint2 entries
+    if constexpr (BITS == 6) {                        // 6 bytes, 8 codes of 6 bits (fp16 entries)
+        const uint16_t *t = reinterpret_cast<const uint16_t *>(tab32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            o[q] = (uint32_t)t[(v >> (12 * q)) & 63u] |
+                   ((uint32_t)t[(v >> (12 * q + 6)) & 63u] << 16);
+    } else if constexpr (BITS == 2) {                        // 2 bytes, 4 codes each -> uint2 entries
         const uint2 *t = reinterpret_cast<const uint2 *>(tab32);
         const uint2 a = t[v & 0xffu], b = t[(v >> 8) & 0xffu];
         o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
@@ -63,6 +69,10 @@ __device__ __forceinline__ uint64_t load_group(const uint8_t *codes, long long g
         return __ldg(reinterpret_cast<const unsigned int *>(src));
     else if constexpr (BITS == 8)
         return __ldg(reinterpret_cast<const unsigned long long *>(src));
+    else if constexpr (BITS == 6)                     // 6 bytes at an even address
+        return (uint64_t)__ldg(reinterpret_cast<const unsigned short *>(src)) |
+               ((uint64_t)__ldg(reinterpret_cast<const unsigned short *>(src + 2)) << 16) |
+               ((uint64_t)__ldg(reinterpret_cast<const unsigned short *>(src + 4)) << 32);
     else
         return (uint64_t)__ldg(src) | ((uint64_t)__ldg(src + 1) << 8) |
                ((uint64_t)__ldg(src + 2) << 16);
@@ -71,8 +81,9 @@ __device__ __forceinline__ uint64_t load_group(const uint8_t *codes, long long g
 // SYM (BITS == 4 only): decode with byte permutes instead of the shared table.
 template <int BITS, bool SYM>
 __global__ void __launch_bounds__(kDecThreads) k2_decode(const __grid_constant__ DecodeParams p) {
-    // b=2: 256 entries of 4 fp16 (uint2); b=3: 64 entries of 2 fp16; b=4: 256 of 2; b=8: 256 of 1
-    constexpr int PER = BITS == 2 ? 4 : (BITS == 8 ? 1 : 2);      // codes per lookup
+    // b=2: 256 entries of 4 fp16 (uint2); b=3: 64 entries of 2 fp16; b=4: 256 of 2;
+    // b=6: 64 of 1; b=8: 256 of 1
+    constexpr int PER = BITS == 2 ? 4 : ((BITS == 8 || BITS == 6) ? 1 : 2);   // codes per lookup
     constexpr int IDX_BITS = PER * BITS;
     constexpr int ENTRIES = 1 << IDX_BITS;
     static_assert(!SYM || BITS == 4, "byte-permute decode is 4-bit only");
@@ -143,6 +154,7 @@ cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long lo
                     ? decode<4, true>(dp, st, num_sms)
                     : decode<4, false>(dp, st, num_sms);
             break;
+        case 6: e = decode<6, false>(dp, st, num_sms); break;
         case 8: e = decode<8, false>(dp, st, num_sms); break;
         default: e = cudaErrorInvalidValue;
     }

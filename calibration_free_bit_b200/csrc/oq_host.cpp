@@ -101,9 +101,10 @@ struct SplitMix64 {
 };
 
 // ---------------------------------------------------------------------------------------
-// Lloyd-Max for N(0,1): Lloyd warm-up, then Newton on the centroid conditions
-// c_i = E[X | t_i <= X < t_{i+1}], t_i = (c_{i-1} + c_i)/2, with the tridiagonal Jacobian
-// d mu_i / d t_i = phi(t_i)(mu_i - t_i)/P_i,  d mu_i / d t_{i+1} = phi(t_{i+1})(t_{i+1} - mu_i)/P_i.
+// Lloyd-Max: Lloyd warm-up, then Newton on the centroid conditions
+// c_i = E[U | t_i <= U < t_{i+1}], t_i = (c_{i-1} + c_i)/2, with the tridiagonal Jacobian
+// d mu_i / d t_i = f(t_i)(mu_i - t_i)/P_i,  d mu_i / d t_{i+1} = f(t_{i+1})(t_{i+1} - mu_i)/P_i,
+// for a symmetric log-concave density f of the unit-scale coordinate U = sqrt(d) * x_rot / s.
 // ---------------------------------------------------------------------------------------
 double npdf(double x) { return std::isinf(x) ? 0.0 : std::exp(-0.5 * x * x) * 0.3989422804014327; }
 double ntail(double x) {   // P(X > x)
@@ -119,24 +120,105 @@ double nprob(double a, double b) {   // P(a <= X < b), a < b
     return 1.0 - ntail(-a) - ntail(b);
 }
 
-bool solve_lloyd_max(int L, std::vector<double> &c) {
-    const double inf = std::numeric_limits<double>::infinity();
+// N(0,1): the marginal read as N(0, 1/d), in unit scale ([RCAP] change-of-basis paragraph).
+struct GaussMarginal {
+    double lo = -std::numeric_limits<double>::infinity();
+    double hi = std::numeric_limits<double>::infinity();
+    double pdf(double u) const { return npdf(u); }
+    double prob(double a, double b) const { return nprob(a, b); }
+    double moment(double a, double b) const { return npdf(a) - npdf(b); }
+};
+
+// Gauss-Legendre rule on [-1, 1]: nodes are the roots of P_n found by Newton's method from
+// the usual cosine estimates, weights 2 / ((1 - x^2) P_n'(x)^2).
+struct GaussLegendre {
+    static constexpr int n = 12;
+    double x[n], w[n];
+    GaussLegendre() {
+        const double pi = 3.14159265358979323846;
+        for (int i = 0; i < n; ++i) {
+            double z = std::cos(pi * (i + 0.75) / (n + 0.5)), dp = 1.0;
+            for (int it = 0; it < 100; ++it) {
+                double p0 = 1.0, p1 = z;                 // P_0, P_1
+                for (int k = 2; k <= n; ++k) {           // (k) P_k = (2k-1) z P_{k-1} - (k-1) P_{k-2}
+                    const double p2 = ((2.0 * k - 1.0) * z * p1 - (k - 1.0) * p0) / k;
+                    p0 = p1;
+                    p1 = p2;
+                }
+                dp = n * (z * p1 - p0) / (z * z - 1.0);  // P_n'(z)
+                const double dz = p1 / dp;
+                z -= dz;
+                if (std::fabs(dz) < 1e-16)
+                    break;
+            }
+            x[i] = z;
+            w[i] = 2.0 / ((1.0 - z * z) * dp * dp);
+        }
+    }
+};
+
+// The exact marginal f_d of one coordinate of a uniform unit vector in R^d, in unit scale
+// u = sqrt(d) x: f(u) = (1 - u^2/d)^((d-3)/2) / (sqrt(d) B(1/2, (d-1)/2)) on [-sqrt(d), sqrt(d)].
+// Cell probabilities by composite 12-point Gauss-Legendre quadrature (panels of width <= 1/2,
+// outside |u| > 45 the density is below 1e-400 and is dropped); first moments in closed form,
+// int_a^b u f(u) du = sqrt(d) ((1 - a^2/d)^((d-1)/2) - (1 - b^2/d)^((d-1)/2)) / ((d-1) B).
+struct SphereMarginal {
+    double d, lo, hi, log_norm_pdf, mom_scale, cut;
+    const GaussLegendre *gl;
+    SphereMarginal(int dim, const GaussLegendre *rule) : d(dim), gl(rule) {
+        hi = std::sqrt(d);
+        lo = -hi;
+        const double log_b = std::lgamma(0.5) + std::lgamma(0.5 * (d - 1)) - std::lgamma(0.5 * d);
+        log_norm_pdf = -0.5 * std::log(d) - log_b;
+        mom_scale = std::sqrt(d) / ((d - 1) * std::exp(log_b));
+        cut = std::min(hi, 45.0);
+    }
+    double pdf(double u) const {
+        if (u <= lo || u >= hi)
+            return 0.0;
+        return std::exp(0.5 * (d - 3) * std::log1p(-u * u / d) + log_norm_pdf);
+    }
+    double prob(double a, double b) const {
+        a = std::max(a, -cut);
+        b = std::min(b, cut);
+        if (!(b > a))
+            return 0.0;
+        const int panels = (int)std::ceil((b - a) / 0.5);
+        const double h = (b - a) / panels;
+        double sum = 0.0;
+        for (int k = 0; k < panels; ++k) {
+            const double m = a + (k + 0.5) * h;
+            for (int i = 0; i < GaussLegendre::n; ++i)
+                sum += gl->w[i] * pdf(m + 0.5 * h * gl->x[i]);
+        }
+        return 0.5 * h * sum;
+    }
+    double moment(double a, double b) const {
+        auto g = [&](double u) {
+            return (u <= lo || u >= hi) ? 0.0 : std::exp(0.5 * (d - 1) * std::log1p(-u * u / d));
+        };
+        return mom_scale * (g(a) - g(b));
+    }
+};
+
+template <class Marginal>
+bool solve_lloyd_max(const Marginal &f, int L, std::vector<double> &c) {
     c.assign(L, 0.0);
-    const double span = 1.5 + 0.4 * std::log2((double)L);
+    const double span = std::min(1.5 + 0.4 * std::log2((double)L), 0.9 * f.hi);
     for (int i = 0; i < L; ++i)
         c[i] = span * (2.0 * (i + 0.5) / L - 1.0);
     std::vector<double> t(L + 1), mu(L), da(L), db(L);
     auto cells = [&]() {
-        t[0] = -inf;
-        t[L] = inf;
+        t[0] = f.lo;
+        t[L] = f.hi;
         for (int i = 1; i < L; ++i)
             t[i] = 0.5 * (c[i - 1] + c[i]);
         for (int i = 0; i < L; ++i) {
             const double a = t[i], b = t[i + 1];
-            const double P = nprob(a, b);
-            mu[i] = (npdf(a) - npdf(b)) / P;
-            da[i] = std::isinf(a) ? 0.0 : npdf(a) * (mu[i] - a) / P;
-            db[i] = std::isinf(b) ? 0.0 : npdf(b) * (b - mu[i]) / P;
+            const double P = f.prob(a, b);
+            mu[i] = f.moment(a, b) / P;
+            da[i] = i == 0 ? 0.0 : f.pdf(a) * (mu[i] - a) / P;          // support edges
+            db[i] = i == L - 1 ? 0.0 : f.pdf(b) * (b - mu[i]) / P;      // are not free
         }
     };
     // Lloyd iterations bring every cell near the optimum
@@ -181,7 +263,7 @@ bool solve_lloyd_max(int L, std::vector<double> &c) {
         for (int i = 0; i < L; ++i)
             c[i] -= lam * step[i];
     }
-    // exact symmetry of the N(0,1) problem
+    // exact symmetry of the (symmetric) problem
     for (int i = 0; i < L / 2; ++i) {
         const double m = 0.5 * (c[L - 1 - i] - c[i]);
         c[i] = -m;
@@ -236,7 +318,7 @@ struct oq_rpbh {
 };
 
 struct oq_codebook {
-    int d = 0, bits = 0;
+    int d = 0, bits = 0, marginal = OQ_MARGINAL_GAUSSIAN;
     std::vector<double> c, t;                     // unit centroids / boundaries
     uint16_t lut[256] = {};                       // unit centroids, fp16 bits
     int G = 0, F = 0;
@@ -368,7 +450,7 @@ int check_dims(int d, const char *who) {
 
 int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dtype, int rows,
                   int d, uint8_t *codes, float *norms, void *stream, float eps,
-                  const char *who) {
+                  const char *who, bool gelu = false) {
     if (!r || !cb)
         return fail(OQ_EINVAL, "%s: null handle", who);
     if (check_dims(d, who) != OQ_OK)
@@ -378,6 +460,8 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
                     r->d, cb->d);
     if (dtype != OQ_F32 && dtype != OQ_BF16)
         return fail(OQ_EINVAL, "%s: dtype must be OQ_F32 or OQ_BF16", who);
+    if (gelu && dtype != OQ_BF16)
+        return fail(OQ_EINVAL, "%s: the fused GELU takes bf16 input", who);
     if (rows < 0)
         return fail(OQ_EINVAL, "%s: negative row count %d", who, rows);
     if (rows == 0)
@@ -413,6 +497,7 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
     p.K = (float)(std::sqrt((double)d / r->h) / (cb->G * cb->delta));
     p.G = cb->G;
     p.F = cb->F;
+    p.gelu = gelu ? 1 : 0;
     std::string why;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = timed(OQ_KERNEL_QUANTIZE, st, [&] {
@@ -461,18 +546,21 @@ bool fused_requested() {
 // ---------------------------------------------------------------------------------------
 extern "C" {
 
-int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out) {
+namespace {
+
+// RPBH tables (permute = true) or Block-RHT tables (the same draws, identity permutation).
+int build_rotation(int d, int h, uint64_t seed, bool permute, oq_rpbh **out, const char *who) {
     if (!out)
-        return fail(OQ_EINVAL, "oq_build_rpbh: out is NULL");
+        return fail(OQ_EINVAL, "%s: out is NULL", who);
     *out = nullptr;
-    if (check_dims(d, "oq_build_rpbh") != OQ_OK)
+    if (check_dims(d, who) != OQ_OK)
         return OQ_EINVAL;
     if (h < 32 || h > 1024 || (h & (h - 1)) != 0 || d % h != 0)
-        return fail(OQ_EINVAL, "oq_build_rpbh: h = %d must be a power of two in [32, 1024] "
-                               "dividing d = %d", h, d);
+        return fail(OQ_EINVAL, "%s: h = %d must be a power of two in [32, 1024] dividing "
+                               "d = %d", who, h, d);
     oq_rpbh *r = new (std::nothrow) oq_rpbh;
     if (!r)
-        return fail(OQ_ENOMEM, "oq_build_rpbh: out of host memory");
+        return fail(OQ_ENOMEM, "%s: out of host memory", who);
     r->d = d;
     r->h = h;
     r->seed = seed;
@@ -487,6 +575,9 @@ int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out) {
     }
     for (int k = 0; k < d; ++k)
         r->sign[k] = (g.next() >> 63) ? -1 : 1;
+    if (!permute)
+        for (int i = 0; i < d; ++i)
+            r->perm[i] = i;
     // K1 gather-entry images (layout documented in oq_internal.h)
     for (int f = 0; f < 2; ++f) {
         r->ent_img[f].assign((size_t)(d / 32) * oq::kK1EntStride, 0u);
@@ -503,6 +594,16 @@ int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out) {
     return OQ_OK;
 }
 
+}  // namespace
+
+int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out) {
+    return build_rotation(d, h, seed, true, out, "oq_build_rpbh");
+}
+
+int oq_build_block_rht(int d, int h, uint64_t seed, oq_rpbh **out) {
+    return build_rotation(d, h, seed, false, out, "oq_build_block_rht");
+}
+
 int oq_rpbh_tables(const oq_rpbh *r, int32_t *perm_out, int8_t *sign_out) {
     if (!r)
         return fail(OQ_EINVAL, "oq_rpbh_tables: null handle");
@@ -513,23 +614,35 @@ int oq_rpbh_tables(const oq_rpbh *r, int32_t *perm_out, int8_t *sign_out) {
     return OQ_OK;
 }
 
-int oq_lloyd_max(int d, int bits, oq_codebook **out) {
+int oq_lloyd_max_marginal(int d, int bits, int marginal, oq_codebook **out) {
+    const char *who = "oq_lloyd_max";
     if (!out)
-        return fail(OQ_EINVAL, "oq_lloyd_max: out is NULL");
+        return fail(OQ_EINVAL, "%s: out is NULL", who);
     *out = nullptr;
-    if (d < 1)
-        return fail(OQ_EINVAL, "oq_lloyd_max: d = %d", d);
-    if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
-        return fail(OQ_EINVAL, "oq_lloyd_max: bits = %d not in {2, 3, 4, 8}", bits);
+    if (marginal != OQ_MARGINAL_GAUSSIAN && marginal != OQ_MARGINAL_EXACT)
+        return fail(OQ_EINVAL, "%s: marginal = %d (OQ_MARGINAL_GAUSSIAN or OQ_MARGINAL_EXACT)",
+                    who, marginal);
+    if (d < 1 || (marginal == OQ_MARGINAL_EXACT && d < 3))
+        return fail(OQ_EINVAL, "%s: d = %d (the exact marginal needs d >= 3)", who, d);
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 6 && bits != 8)
+        return fail(OQ_EINVAL, "%s: bits = %d not in {2, 3, 4, 6, 8}", who, bits);
     oq_codebook *cb = new (std::nothrow) oq_codebook;
     if (!cb)
-        return fail(OQ_ENOMEM, "oq_lloyd_max: out of host memory");
+        return fail(OQ_ENOMEM, "%s: out of host memory", who);
     cb->d = d;
     cb->bits = bits;
+    cb->marginal = marginal;
     const int L = 1 << bits;
-    if (!solve_lloyd_max(L, cb->c)) {
+    bool ok;
+    if (marginal == OQ_MARGINAL_GAUSSIAN) {
+        ok = solve_lloyd_max(GaussMarginal{}, L, cb->c);
+    } else {
+        static const GaussLegendre rule;
+        ok = solve_lloyd_max(SphereMarginal(d, &rule), L, cb->c);
+    }
+    if (!ok) {
         delete cb;
-        return fail(OQ_EINVAL, "oq_lloyd_max: solver did not converge for %d levels", L);
+        return fail(OQ_EINVAL, "%s: solver did not converge for %d levels", who, L);
     }
     cb->t.resize(L - 1);
     for (int j = 0; j < L - 1; ++j)
@@ -538,7 +651,7 @@ int oq_lloyd_max(int d, int bits, oq_codebook **out) {
         cb->lut[i] = to_half_bits(cb->c[i]);
     if (!build_grid(cb)) {
         delete cb;
-        return fail(OQ_EINVAL, "oq_lloyd_max: could not build the quantizer grid");
+        return fail(OQ_EINVAL, "%s: could not build the quantizer grid", who);
     }
     // K1 table image: one copy per lane when bits <= 4 (conflict-free lookups), padded to 16 B
     const int copies = bits <= 4 ? 32 : 1;
@@ -548,6 +661,10 @@ int oq_lloyd_max(int d, int bits, oq_codebook **out) {
             cb->tbl_img[(size_t)k * copies + l] = cb->grid[k];
     *out = cb;
     return OQ_OK;
+}
+
+int oq_lloyd_max(int d, int bits, oq_codebook **out) {
+    return oq_lloyd_max_marginal(d, bits, OQ_MARGINAL_GAUSSIAN, out);
 }
 
 int oq_codebook_values(const oq_codebook *cb, double *centroids, double *bounds) {
@@ -586,6 +703,12 @@ int oq_quantize_weight(const oq_rpbh *r, const oq_codebook *cw, const void *W, i
 int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype, int T,
                     int d, uint8_t *x_codes, float *s, void *stream) {
     return quantize_rows(r, ca, x, dtype, T, d, x_codes, s, stream, 1e-8f, "oq_quantize_act");
+}
+
+int oq_quantize_act_gelu(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype,
+                         int T, int d, uint8_t *x_codes, float *s, void *stream) {
+    return quantize_rows(r, ca, x, dtype, T, d, x_codes, s, stream, 1e-8f,
+                         "oq_quantize_act_gelu", true);
 }
 
 int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,

@@ -39,6 +39,7 @@ struct K1Params {
     int G, F;               // grid cells (power of two), F = 23 - log2(G)
     int groups;             // token pairs processed at once per CTA (set by launch_k1)
     int stages;             // raw row buffers per group, fp32 input only (set by launch_k1)
+    int gelu;               // 1: quantize R GELU(x) (erf form; bf16 input only)
 };
 
 // Launch K1 for (bits, h, dtype); `num_sms` sizes the grid.

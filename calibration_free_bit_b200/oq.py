@@ -45,12 +45,15 @@ def lib():
     L = C.CDLL(LIB_PATH)
     vp, i32, u64 = C.c_void_p, C.c_int, C.c_uint64
     L.oq_build_rpbh.argtypes = [i32, i32, u64, C.POINTER(vp)]
+    L.oq_build_block_rht.argtypes = [i32, i32, u64, C.POINTER(vp)]
     L.oq_rpbh_tables.argtypes = [vp, vp, vp]
     L.oq_lloyd_max.argtypes = [i32, i32, C.POINTER(vp)]
+    L.oq_lloyd_max_marginal.argtypes = [i32, i32, i32, C.POINTER(vp)]
     L.oq_codebook_values.argtypes = [vp, vp, vp]
     L.oq_codebook_grid.argtypes = [vp, C.POINTER(i32), C.POINTER(C.c_double), vp]
     L.oq_quantize_weight.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.oq_quantize_act.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
+    L.oq_quantize_act_gelu.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.oq_linear.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp]
     L.oq_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp]
     L.oq_check.argtypes = [vp]
@@ -62,8 +65,10 @@ def lib():
     L.oq_timing_collect.argtypes = [vp, i32, C.POINTER(i32)]
     L.oq_last_error.restype = C.c_char_p
     L.oq_version.restype = C.c_char_p
-    for name in ("oq_build_rpbh", "oq_rpbh_tables", "oq_lloyd_max", "oq_codebook_values",
-                 "oq_codebook_grid", "oq_quantize_weight", "oq_quantize_act", "oq_linear",
+    for name in ("oq_build_rpbh", "oq_build_block_rht", "oq_rpbh_tables", "oq_lloyd_max", "oq_lloyd_max_marginal",
+                 "oq_codebook_values",
+                 "oq_codebook_grid", "oq_quantize_weight", "oq_quantize_act",
+                 "oq_quantize_act_gelu", "oq_linear",
                  "oq_linear_noalloc", "oq_check", "oq_timing_enable", "oq_timing_collect"):
         getattr(L, name).restype = i32
     _lib = L
@@ -109,12 +114,14 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 class RPBH:
-    """Handle of an RPBH rotation (oq_build_rpbh)."""
+    """Handle of an RPBH rotation (oq_build_rpbh), or of its Block-RHT ablation without the
+    leading permutation (oq_build_block_rht, permute=False)."""
 
-    def __init__(self, d: int, h: int, seed: int = 0):
+    def __init__(self, d: int, h: int, seed: int = 0, permute: bool = True):
         self._h = C.c_void_p()
-        _check(lib().oq_build_rpbh(d, h, seed, C.byref(self._h)))
-        self.d, self.h, self.seed = d, h, seed
+        build = lib().oq_build_rpbh if permute else lib().oq_build_block_rht
+        _check(build(d, h, seed, C.byref(self._h)))
+        self.d, self.h, self.seed, self.permute = d, h, seed, permute
 
     @property
     def handle(self):
@@ -132,13 +139,17 @@ class RPBH:
             self._h = C.c_void_p()
 
 
-class Codebook:
-    """Handle of a Lloyd-Max codebook for N(0, 1/d) (oq_lloyd_max)."""
+MARGINALS = {"gauss": 0, "exact": 1}      # OQ_MARGINAL_GAUSSIAN, OQ_MARGINAL_EXACT
 
-    def __init__(self, d: int, bits: int):
+
+class Codebook:
+    """Handle of a Lloyd-Max codebook (oq_lloyd_max_marginal): for N(0, 1/d) ("gauss") or for
+    the exact coordinate marginal f_d ("exact")."""
+
+    def __init__(self, d: int, bits: int, marginal: str = "gauss"):
         self._h = C.c_void_p()
-        _check(lib().oq_lloyd_max(d, bits, C.byref(self._h)))
-        self.d, self.bits = d, bits
+        _check(lib().oq_lloyd_max_marginal(d, bits, MARGINALS[marginal], C.byref(self._h)))
+        self.d, self.bits, self.marginal = d, bits, marginal
 
     @property
     def handle(self):
@@ -169,8 +180,12 @@ def oq_build_rpbh(d: int, h: int, seed: int = 0) -> RPBH:
     return RPBH(d, h, seed)
 
 
-def oq_lloyd_max(d: int, bits: int) -> Codebook:
-    return Codebook(d, bits)
+def oq_build_block_rht(d: int, h: int, seed: int = 0) -> RPBH:
+    return RPBH(d, h, seed, permute=False)
+
+
+def oq_lloyd_max(d: int, bits: int, marginal: str = "gauss") -> Codebook:
+    return Codebook(d, bits, marginal)
 
 
 def _rows_out(x: torch.Tensor, bits: int, codes, norms):
@@ -191,11 +206,14 @@ def oq_quantize_weight(r: RPBH, cw: Codebook, W: torch.Tensor, W_codes=None, row
     return W_codes, row_norms
 
 
-def oq_quantize_act(r: RPBH, ca: Codebook, x: torch.Tensor, x_codes=None, s=None, stream=None):
-    """Online activation step: returns (x_codes uint8 [T, d*ba/8], s fp32 [T])."""
+def oq_quantize_act(r: RPBH, ca: Codebook, x: torch.Tensor, x_codes=None, s=None, stream=None,
+                    gelu: bool = False):
+    """Online activation step: returns (x_codes uint8 [T, d*ba/8], s fp32 [T]); with
+    gelu=True the codes and norms are those of GELU(x) (oq_quantize_act_gelu, bf16 x)."""
     x_codes, s = _rows_out(x, ca.bits, x_codes, s)
-    _check(lib().oq_quantize_act(r.handle, ca.handle, _ptr(x), _dtype_code(x), x.shape[0],
-                                 x.shape[1], _ptr(x_codes), _ptr(s), _stream(stream)))
+    fn = lib().oq_quantize_act_gelu if gelu else lib().oq_quantize_act
+    _check(fn(r.handle, ca.handle, _ptr(x), _dtype_code(x), x.shape[0], x.shape[1],
+              _ptr(x_codes), _ptr(s), _stream(stream)))
     return x_codes, s
 
 

@@ -22,7 +22,7 @@
  *     small tables to that device synchronously; make that first use outside any CUDA graph
  *     capture.
  *   - Sizes: d is a multiple of 128 and of h, 128 <= d <= 16384; h is a power of two,
- *     32 <= h <= 1024; bits in {2, 3, 4, 8}; 0 <= T < 2^31 rows (T = 0 is a no-op returning
+ *     32 <= h <= 1024; bits in {2, 3, 4, 6, 8}; 0 <= T < 2^31 rows (T = 0 is a no-op returning
  *     OQ_OK); the linear layer also needs 1 <= out_features < 2^31.
  *   - Packed codes: row-major, one row per token (or weight row), row stride d*bits/8 bytes,
  *     element k of a row in bits [k*bits, k*bits + bits) of the row's byte stream, bit i of
@@ -63,6 +63,12 @@ typedef struct oq_codebook oq_codebook;
  * Errors: OQ_EINVAL for d, h outside the limits above or out == NULL. */
 int oq_build_rpbh(int d, int h, uint64_t seed, oq_rpbh **out);
 
+/* Block-RHT: the ablation in [RCAP]'s results list that removes the leading uniform
+ * permutation.  The handle is that of oq_build_rpbh(d, h, seed) with the permutation replaced
+ * by the identity (same sign flips, same blocks), so it runs through the same calls
+ * (oq_quantize_act / oq_quantize_weight) and only P differs.  Same arguments and errors. */
+int oq_build_block_rht(int d, int h, uint64_t seed, oq_rpbh **out);
+
 /* Copy the handle's tables to host memory: perm_out[d] (int32), sign_out[d] (+1/-1).
  * Either pointer may be NULL.  Host-only. */
 int oq_rpbh_tables(const oq_rpbh *r, int32_t *perm_out, int8_t *sign_out);
@@ -71,8 +77,20 @@ int oq_rpbh_tables(const oq_rpbh *r, int32_t *perm_out, int8_t *sign_out);
  * [RCAP] change-of-basis paragraph ("the standard Lloyd-Max quantizer construction" against
  * the fixed marginal, close to N(0, 1/d) for d > 64) and pseudocode lloyd_max(f_d, b).
  * The unit (N(0,1)) quantizer is solved in fp64 and scaled by sigma = 1/sqrt(d).
- * Host-only; no GPU needed.  Errors: OQ_EINVAL for bits not in {2,3,4,8}, d < 1. */
+ * Host-only; no GPU needed.  Errors: OQ_EINVAL for bits not in {2,3,4,6,8}, d < 1. */
 int oq_lloyd_max(int d, int bits, oq_codebook **out);
+
+#define OQ_MARGINAL_GAUSSIAN 0   /* N(0, 1/d), the reading oq_lloyd_max uses                */
+#define OQ_MARGINAL_EXACT 1      /* f_d, the exact law of one coordinate of a unit vector   */
+
+/* oq_lloyd_max against a chosen marginal.  OQ_MARGINAL_EXACT: f_d(x) = (1 - x^2)^((d-3)/2) /
+ * B(1/2, (d-1)/2) on [-1, 1], the law of one coordinate of a uniformly random unit vector in
+ * R^d ([RCAP] change-of-basis paragraph: the fixed marginal that depends only on d, which
+ * N(0, 1/d) approximates above d = 64).  The codebook is stored as sqrt(d) times the f_d
+ * quantizer, so it plugs into the same kernels as the Gaussian one (oq_codebook_values
+ * returns the f_d quantizer itself).  Host-only.  Errors: OQ_EINVAL for an unknown
+ * marginal, bits not in {2,3,4,6,8}, d < 1 (d < 3 for the exact marginal). */
+int oq_lloyd_max_marginal(int d, int bits, int marginal, oq_codebook **out);
 
 /* Copy the codebook to host memory in fp64, sigma-scaled: centroids[2^bits] ascending,
  * bounds[2^bits - 1] ascending (bounds[j] is the midpoint of centroids j and j+1).
@@ -107,6 +125,15 @@ int oq_quantize_weight(const oq_rpbh *r, const oq_codebook *cw, const void *W, i
  * Errors: as oq_quantize_weight. */
 int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype, int T,
                     int d, uint8_t *x_codes, float *s, void *stream);
+
+/* oq_quantize_act applied to GELU(x) = x Phi(x) = x (1 + erf(x/sqrt 2)) / 2, computed inside
+ * the kernel: the quantized input of an MLP's down projection straight from the up
+ * projection's pre-activation, with no GELU pass over memory.  GELU is evaluated in fp32
+ * on each bf16 element (CUDA's erff); s = ||R GELU(x)||.  x must be OQ_BF16.  Same layouts and
+ * errors as oq_quantize_act, plus OQ_EINVAL for fp32 input.  The pages' models (FLUX, Wan)
+ * feed their MLP down projections through GELU; this is the fused form of that step. */
+int oq_quantize_act_gelu(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype,
+                         int T, int d, uint8_t *x_codes, float *s, void *stream);
 
 /* Codebook linear layer: y[t][o] = s[t] * row_norms[o] * sum_k ca[x_codes[t][k]] *
  * cw[W_codes[o][k]] with sigma-scaled centroids, i.e. x_hat . w_hat in the rotated basis,

@@ -8,6 +8,7 @@ import ctypes as C
 import math
 
 import numpy as np
+from scipy import special
 
 from . import build as _build
 
@@ -248,8 +249,17 @@ def quantize_rows(x, h: int, perm, sign, bits: int, eps: float, detail: bool = F
     return packed, norms
 
 
-def quantize_act(x, h, perm, sign, bits, detail=False, marginal="gauss"):
-    """Online activation step: eps = EPS_ACT."""
+def gelu(x) -> np.ndarray:
+    """GELU in its erf form, x Phi(x) = x (1 + erf(x / sqrt 2)) / 2, in fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + special.erf(x / math.sqrt(2.0)))
+
+
+def quantize_act(x, h, perm, sign, bits, detail=False, marginal="gauss", gelu_input=False):
+    """Online activation step: eps = EPS_ACT.  gelu_input: quantize GELU(x) (the MLP down
+    projection's input formed from the up projection's pre-activation)."""
+    if gelu_input:
+        x = gelu(_f64(np.atleast_2d(x)))
     return quantize_rows(x, h, perm, sign, bits, EPS_ACT, detail, marginal)
 
 

@@ -12,6 +12,8 @@ Inputs are the seeded synthetic workloads of calibration_free_bit_b200.synth; la
 workloads are checked on sampled rows / columns (the oracle computes those one by one) and
 on properties that hold at any size (norm preservation, code range).
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -47,7 +49,7 @@ def handles(oq, d, h, ba, bw, seed=0):
     return _HANDLES[key]
 
 
-def check_codes(gpu_packed, orc_packed, orc_u, d, bits, what):
+def check_codes(gpu_packed, orc_packed, orc_u, d, bits, what, marginal="gauss"):
     """Code-parity rule on a block of rows; returns the number of mismatches."""
     gpu_packed = np.ascontiguousarray(gpu_packed)
     gcodes = O.unpack(gpu_packed, d, bits)
@@ -57,7 +59,7 @@ def check_codes(gpu_packed, orc_packed, orc_u, d, bits, what):
     bad = np.argwhere(gcodes != ocodes)
     n = gcodes.size
     assert len(bad) <= (1 - CODE_MATCH) * n + 1e-9, f"{what}: {len(bad)} of {n} codes differ"
-    _, t = O.codebook(bits)
+    _, t = O.codebook(bits, marginal, d)
     for r, k in bad:
         u = orc_u[r, k]
         j = int(np.argmin(np.abs(t - u)))
@@ -74,12 +76,12 @@ def k1_gpu(oq, r, cb, x_cpu, weight=False):
     return codes.cpu().numpy(), s.cpu().numpy().astype(np.float64)
 
 
-def k1_oracle(x_cpu, h, bits, weight=False, seed=0):
+def k1_oracle(x_cpu, h, bits, weight=False, seed=0, marginal="gauss", permute=True):
     d = x_cpu.shape[1]
-    perm, sign = O.build_rpbh(d, seed)
+    perm, sign = (O.build_rpbh if permute else O.build_block_rht)(d, seed)
     x64 = x_cpu.double().numpy()
     fn = O.quantize_weight if weight else O.quantize_act
-    return fn(x64, h, perm, sign, bits, detail=True)
+    return fn(x64, h, perm, sign, bits, detail=True, marginal=marginal)
 
 
 # ----------------------------------------------------------------------------------------
@@ -101,7 +103,7 @@ def test_k1_toy_fp32_activations_and_weights(oq):
 
 
 @pytest.mark.parametrize("h", [32, 64, 128, 256, 512, 1024])
-@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
 def test_k1_every_block_size_and_bit_width(oq, h, bits):
     d = 2048 if h <= 512 else 3072
     T = 37                                  # odd: the last token pair has one token
@@ -113,6 +115,55 @@ def test_k1_every_block_size_and_bit_width(oq, h, bits):
     o, os_, _, ou = k1_oracle(x, h, bits)
     check_codes(g, o, ou, d, bits, f"h={h} b={bits}")
     np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+
+
+@pytest.mark.parametrize("d,h,bits", [(128, 64, 2), (128, 128, 4), (256, 64, 8), (384, 128, 3)])
+def test_exact_marginal_codebook_k1_and_linear(oq, d, h, bits):
+    """The f_d codebook (oq_lloyd_max_marginal, OQ_MARGINAL_EXACT) through K1 and the linear
+    layer, at the small d where it differs most from N(0, 1/d)."""
+    T, N = 150, 272
+    p = synth.sweep_projection(d, h, 4, T)
+    x = synth.activations(p)
+    W = torch.randn(N, d, generator=torch.Generator().manual_seed(d + bits)) / math.sqrt(d)
+    r = oq.oq_build_rpbh(d, h, 0)
+    cb = oq.oq_lloyd_max(d, bits, "exact")
+    g, gs = k1_gpu(oq, r, cb, x)
+    o, os_, _, ou = k1_oracle(x, h, bits, marginal="sphere")
+    check_codes(g, o, ou, d, bits, f"exact d={d} b={bits}", marginal="sphere")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+    gw, gws = k1_gpu(oq, r, cb, W, weight=True)
+    ow, ows, _, wu = k1_oracle(W, h, bits, weight=True, marginal="sphere")
+    check_codes(gw, ow, wu, d, bits, f"exact W d={d} b={bits}", marginal="sphere")
+    y = linear_gpu(oq, cb, cb, o, os_, ow, ows)
+    ref = O.linear(o, os_, ow, ows, d, bits, bits, marginal="sphere")
+    assert rel_l2(y, ref) <= LINEAR_RTOL
+
+
+def test_block_rht_k1_and_linear(oq):
+    """The Block-RHT ablation (identity permutation) through K1 and the linear layer on sampled
+    rows of the attention workload, and on an input concentrated on one block of positions,
+    which Block-RHT leaves concentrated."""
+    p = synth.get("flux_attn_w4a4")[0]
+    rows = np.arange(0, p.T, 53)
+    x = synth.activations(p, rows=rows)
+    rng = np.random.default_rng(1)
+    adv = np.zeros((9, p.d), np.float32)
+    adv[:, p.h:2 * p.h] = rng.standard_normal((9, p.h))
+    x = torch.cat([x, torch.from_numpy(adv).to(x.dtype)])
+    r = oq.oq_build_block_rht(p.d, p.h, 0)
+    ca, cw = oq.oq_lloyd_max(p.d, 4), oq.oq_lloyd_max(p.d, 4)
+    g, gs = k1_gpu(oq, r, ca, x)
+    o, os_, _, ou = k1_oracle(x, p.h, 4, permute=False)
+    check_codes(g, o, ou, p.d, 4, "block-rht x")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+    half = 1 << 3                                     # code of 0: the block stays local
+    codes = O.unpack(g[-9:], p.d, 4)
+    assert np.all(codes[:, :p.h] == half) and np.all(codes[:, 2 * p.h:] == half)
+    W = synth.weight(p)[:272]
+    gw, gws = k1_gpu(oq, r, cw, W, weight=True)
+    y = linear_gpu(oq, ca, cw, g, gs, gw, gws)
+    ref = O.linear(g, gs, gw, gws, p.d, 4, 4)
+    assert rel_l2(y, ref) <= LINEAR_RTOL
 
 
 def test_k1_flux_attention_full_size(oq):
@@ -217,7 +268,8 @@ def test_linear_toy_on_oracle_codes(oq):
     assert rel_l2(y, ref) <= LINEAR_RTOL
 
 
-@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (4, 3), (3, 4), (2, 2), (8, 4), (2, 8), (8, 8)])
+@pytest.mark.parametrize("ba,bw", [(4, 4), (4, 2), (4, 3), (3, 4), (2, 2), (8, 4), (2, 8), (8, 8),
+                                   (3, 2), (6, 6), (4, 6)])
 @pytest.mark.parametrize("T,N,d", [(200, 272, 384), (1, 16, 128), (129, 512, 1024)])
 def test_linear_random_codes_ragged(oq, ba, bw, T, N, d):
     """Uniform random codes (every centroid used), ragged M and N tails."""
@@ -334,3 +386,31 @@ def test_linear_bf16_output_full_size(oq):
     y16 = oq.oq_linear(ca, cw, xc, s, wc, rn, out_dtype=torch.bfloat16)
     oq.oq_check()
     assert torch.equal(y32.to(torch.bfloat16).view(torch.int16), y16.view(torch.int16))
+
+
+@pytest.mark.parametrize("bits,h,d,T", [(4, 128, 12288, 40), (2, 128, 3072, 37),
+                                        (8, 64, 1024, 33), (6, 256, 2048, 31),
+                                        (3, 32, 512, 29)])
+def test_k1_fused_gelu(oq, bits, h, d, T):
+    """oq_quantize_act_gelu: codes and norms of R GELU(x) against the oracle's fp64 GELU, on
+    pre-activations with outlier channels and a per-token lognormal scale (so GELU sees both
+    large positive and large negative arguments)."""
+    p = synth.sweep_projection(d, 128, 4, T)
+    g = torch.Generator().manual_seed(d + bits)
+    u = (synth.activations(p).float() * torch.exp(torch.randn(T, 1, generator=g))).to(
+        torch.bfloat16)
+    r = oq.oq_build_rpbh(d, h, 0)
+    cb = oq.oq_lloyd_max(d, bits)
+    xc, s = oq.oq_quantize_act(r, cb, u.cuda(), gelu=True)
+    oq.oq_check()
+    perm, sign = O.build_rpbh(d, 0)
+    o, os_, _, ou = O.quantize_act(u.double().numpy(), h, perm, sign, bits, detail=True,
+                                   gelu_input=True)
+    check_codes(xc.cpu().numpy(), o, ou, d, bits, f"gelu d={d} b={bits}")
+    np.testing.assert_allclose(s.cpu().numpy(), os_, rtol=NORM_RTOL)
+
+
+def test_k1_fused_gelu_rejects_fp32(oq):
+    r, cb = oq.oq_build_rpbh(256, 64, 0), oq.oq_lloyd_max(256, 4)
+    with pytest.raises(oq.OQError):
+        oq.oq_quantize_act(r, cb, torch.zeros(4, 256, device="cuda"), gelu=True)

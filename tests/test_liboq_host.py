@@ -42,7 +42,15 @@ def test_rpbh_tables_bit_exact_vs_oracle(d, h, seed):
     assert np.array_equal(sign, osign)
 
 
-@pytest.mark.parametrize("bits,tol", [(2, 1e-11), (3, 1e-11), (4, 1e-11), (8, 1e-8)])
+@pytest.mark.parametrize("d,h,seed", [(256, 64, 0), (3072, 128, 9)])
+def test_block_rht_tables_bit_exact_vs_oracle(d, h, seed):
+    perm, sign = oq.oq_build_block_rht(d, h, seed).tables()
+    operm, osign = O.build_block_rht(d, seed)
+    assert np.array_equal(perm, operm) and np.array_equal(sign, osign)
+
+
+@pytest.mark.parametrize("bits,tol", [(2, 1e-11), (3, 1e-11), (4, 1e-11), (6, 1e-10),
+                                      (8, 1e-8)])
 def test_codebook_matches_oracle(bits, tol):
     """Two independent solvers (liboq: Lloyd warm-up + Newton to a residual < 1e-15; oracle:
     plain Lloyd stopped at a step <= 4e-14).  The oracle's distance to the fixed point is
@@ -54,6 +62,33 @@ def test_codebook_matches_oracle(bits, tol):
     sig = 1.0 / np.sqrt(d)
     np.testing.assert_allclose(c, sig * oc, rtol=0, atol=tol * sig)
     np.testing.assert_allclose(t, sig * ot, rtol=0, atol=tol * sig)
+
+
+@pytest.mark.parametrize("d,bits,tol", [(128, 2, 1e-10), (128, 4, 1e-10), (256, 3, 1e-10),
+                                        (3072, 4, 1e-10), (16384, 4, 1e-8), (128, 8, 1e-8)])
+def test_exact_marginal_codebook_matches_oracle(d, bits, tol):
+    """f_d codebook (the f3 variant): liboq solves it by Newton with Gauss-Legendre cell
+    probabilities, the oracle by plain Lloyd with a continued-fraction incomplete beta.
+    Tolerances in unit-codebook units: the oracle's incomplete beta is good to ~1e-11 in
+    absolute probability at d = 16384 (b = 8191.5), and its 8-bit Lloyd stops at a step of
+    1e-12 with a contraction close to 1."""
+    cb = oq.oq_lloyd_max(d, bits, "exact")
+    c, t = cb.values()                                   # the f_d quantizer itself
+    if bits == 8:
+        oc, ot, _, res = O.lloyd_max_sphere(d, bits, tol=1e-12)
+        assert res <= 1e-12
+    else:
+        oc, ot = (v / np.sqrt(d) for v in O.codebook(bits, "sphere", d))
+    sd = 1.0 / np.sqrt(d)
+    np.testing.assert_allclose(c, oc, rtol=0, atol=tol * sd)
+    np.testing.assert_allclose(t, ot, rtol=0, atol=tol * sd)
+    assert np.all(np.abs(c) < 1.0) and np.all(np.diff(c) > 0)
+
+
+def test_exact_marginal_rejects_small_d():
+    h = C.c_void_p()
+    assert oq.lib().oq_lloyd_max_marginal(2, 4, 1, C.byref(h)) == oq.OQ_EINVAL
+    assert oq.lib().oq_lloyd_max_marginal(128, 4, 7, C.byref(h)) == oq.OQ_EINVAL
 
 
 def emulate_kernel_codes(u, G, delta, table):
@@ -68,12 +103,15 @@ def emulate_kernel_codes(u, G, delta, table):
     return (D >> 24).astype(np.int64)
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 8])
-def test_quantizer_grid_matches_boundary_count(bits):
-    cb = oq.oq_lloyd_max(3072, bits)
+@pytest.mark.parametrize("bits,marginal", [(2, "gauss"), (3, "gauss"), (4, "gauss"),
+                                           (6, "gauss"), (8, "gauss"), (4, "exact"),
+                                           (8, "exact")])
+def test_quantizer_grid_matches_boundary_count(bits, marginal):
+    d = 3072 if marginal == "gauss" else 128
+    cb = oq.oq_lloyd_max(d, bits, marginal)
     G, delta, table = cb.grid()
     assert G & (G - 1) == 0 and len(table) == G + 1
-    _, t = O.codebook(bits)
+    t = cb.values()[1] * np.sqrt(d)                     # unit boundaries the grid encodes
     rng = np.random.default_rng(bits)
     u = np.concatenate([rng.standard_normal(400000) * 1.3,
                         rng.uniform(-60, 60, 20000),

@@ -48,13 +48,13 @@ def _cell(t, i):
     return lo, hi
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
 def test_fixed_point_conditions_by_quadrature(bits):
     c, t = O.codebook(bits)
     L = 1 << bits
     # boundaries are exact midpoints
     np.testing.assert_array_equal(t, 0.5 * (c[:-1] + c[1:]))
-    cells = range(L) if bits <= 4 else list(range(0, 8)) + list(range(124, 132)) + \
+    cells = range(L) if bits <= 4 else list(range(0, 8)) + list(range(L // 2 - 4, L // 2 + 4)) + \
         list(range(L - 8, L))
     for i in cells:
         lo, hi = _cell(t, i)
@@ -75,7 +75,7 @@ def test_mse_matches_quadrature(bits):
     assert O.gauss_mse(c, t) == pytest.approx(total, rel=1e-9)
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
 def test_codebook_is_symmetric_and_sorted(bits):
     c, t = O.codebook(bits)
     np.testing.assert_array_equal(c, -c[::-1])
@@ -88,3 +88,11 @@ def test_eight_bit_high_resolution_distortion():
     c, t = O.codebook(8)
     ratio = O.gauss_mse(c, t) * 4 ** 8 / (math.sqrt(3) * math.pi / 2)
     assert 0.985 < ratio < 1.0
+
+
+def test_high_resolution_ratio_approaches_panter_dite_monotonically():
+    """L^2 * MSE / (sqrt(3) pi / 2) rises towards 1 with the bit width (4, 6, 8 bits): the
+    6-bit codebook (the W6A6 setting) sits between its neighbours."""
+    r = [O.gauss_mse(*O.codebook(b)) * 4 ** b / (math.sqrt(3) * math.pi / 2) for b in (4, 6, 8)]
+    assert r[0] < r[1] < r[2] < 1.0
+    assert 0.95 < r[1] < 0.99

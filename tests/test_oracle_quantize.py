@@ -60,7 +60,7 @@ def test_pack_golden_bytes():
         assert np.array_equal(O.unpack(want, len(codes), b)[0], codes)
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
 def test_pack_matches_numpy_bitstream(bits):
     rng = np.random.default_rng(bits)
     n = 128 * 3
@@ -155,3 +155,24 @@ def test_rotated_marginal_is_near_gaussian_statistical():
     ks_p = stats.kstest(u_p.ravel(), "norm").statistic
     ks_id = stats.kstest(u_id.ravel(), "norm").statistic
     assert ks_p < 0.05 and ks_id > 0.4
+
+
+def test_gelu_pins():
+    """GELU(x) = x Phi(x): Phi(1) and Phi(-1) from the normal table, the odd part
+    GELU(x) - GELU(-x) = x (Phi(x) + Phi(-x) = 1), GELU(0) = 0, GELU(x) -> x and -> 0 in the
+    tails."""
+    assert O.gelu(1.0) == pytest.approx(0.8413447460685429, abs=1e-15)
+    assert O.gelu(-1.0) == pytest.approx(-0.15865525393145707, abs=1e-15)
+    x = np.linspace(-9, 9, 1001)
+    np.testing.assert_allclose(O.gelu(x) - O.gelu(-x), x, atol=1e-14)
+    assert O.gelu(0.0) == 0.0
+    assert O.gelu(40.0) == 40.0 and abs(O.gelu(-40.0)) < 1e-300
+
+
+def test_quantize_gelu_input_is_quantize_of_gelu():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3, 256)) * 2
+    perm, sign = O.build_rpbh(256, 0)
+    a = O.quantize_act(x, 64, perm, sign, 4, gelu_input=True)
+    b = O.quantize_act(O.gelu(x), 64, perm, sign, 4)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
