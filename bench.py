@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="flux_attn_w4a4")
+    ap.add_argument("--proj", type=int, default=0, help="projection index within the workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -162,9 +163,12 @@ class OracleStep:
     def __init__(self, p):
         import oracle as O
         self.O, self.p = O, p
-        self.perm, self.sign = O.build_rpbh(p.d, 0)
+        self.perm, self.sign = (O.build_rpbh if p.rotation == "rpbh" else O.build_block_rht)(
+            p.d, 0)
+        self.marginal = "sphere" if p.marginal == "exact" else "gauss"
         W = synth.weight(p).double().numpy()
-        self.wc, self.rn = O.quantize_weight(W, p.h, self.perm, self.sign, p.bits_w)
+        self.wc, self.rn = O.quantize_weight(W, p.h, self.perm, self.sign, p.bits_w,
+                                             marginal=self.marginal)
         self.x = synth.activations(p, rows=np.arange(min(p.T, 2048))).double().numpy()
         self.cursor = 0
 
@@ -172,8 +176,10 @@ class OracleStep:
         rows = (self.cursor + np.arange(S)) % len(self.x)
         self.cursor = int(rows[-1] + 1)
         t0 = time.perf_counter()
-        xc, s = self.O.quantize_act(self.x[rows], self.p.h, self.perm, self.sign, self.p.bits_a)
-        self.O.linear(xc, s, self.wc, self.rn, self.p.d, self.p.bits_a, self.p.bits_w)
+        xc, s = self.O.quantize_act(self.x[rows], self.p.h, self.perm, self.sign, self.p.bits_a,
+                                    marginal=self.marginal, gelu_input=self.p.fused_gelu)
+        self.O.linear(xc, s, self.wc, self.rn, self.p.d, self.p.bits_a, self.p.bits_w,
+                      marginal=self.marginal)
         return time.perf_counter() - t0
 
 
@@ -237,6 +243,8 @@ def workload_config(p, world):
             "T_per_gpu": p.T, "d": p.d, "out": p.out, "h": p.h, "bits_w": p.bits_w,
             "bits_a": p.bits_a, "input": "bf16" if p.dtype == torch.bfloat16 else "fp32",
             "l2": f"{NSETS} rotating buffer sets (x, codes, s, y, W codes) > 126 MB L2",
+            "rotation": p.rotation, "codebook_marginal": p.marginal,
+            "fused_gelu": p.fused_gelu,
             "parallelism": f"dp{world}: independent token batches, no collective"}
 
 
@@ -249,8 +257,9 @@ def run_ours(args, p, rank, world, dev):
     B.build()
     from calibration_free_bit_b200 import oq
 
-    r = oq.oq_build_rpbh(p.d, p.h, 0)
-    ca, cw = oq.oq_lloyd_max(p.d, p.bits_a), oq.oq_lloyd_max(p.d, p.bits_w)
+    r = (oq.oq_build_rpbh if p.rotation == "rpbh" else oq.oq_build_block_rht)(p.d, p.h, 0)
+    ca = oq.oq_lloyd_max(p.d, p.bits_a, p.marginal)
+    cw = oq.oq_lloyd_max(p.d, p.bits_w, p.marginal)
     x_cpu = synth.activations(p)
     W = synth.weight(p).to(dev)
     wc0, rn = oq.oq_quantize_weight(r, cw, W)                # offline, untimed
@@ -269,7 +278,7 @@ def run_ours(args, p, rank, world, dev):
 
     def step(i):
         b = sets[i % NSETS]
-        oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"])
+        oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"], gelu=p.fused_gelu)
         oq.oq_linear(ca, cw, b["xc"], b["s"], b["wc"], rn, b["y"])
 
     def barrier():
@@ -375,7 +384,7 @@ def run_ours(args, p, rank, world, dev):
                 s_comp.wait_event(ev["in"][k])
                 if used[k]:
                     s_comp.wait_event(ev["out"][k])        # y[k] read out by step i - NB
-                oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"])
+                oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"], gelu=p.fused_gelu)
                 oq.oq_linear(ca, cw, b["xc"], b["s"], b["wc"], rn, b["y"])
                 ev["comp"][k].record(s_comp)
             with torch.cuda.stream(s_out):
@@ -464,7 +473,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    p = synth.get(args.workload)[0]
+    p = synth.get(args.workload)[args.proj]
 
     if args.impl == "reference":
         if rank == 0:

@@ -45,6 +45,10 @@ class Projection:
     w_outlier_scale: float = 1.0
     cfg: int = 0
     proj: int = 0
+    # variants of the path (how the projection is quantized, not how its data are drawn)
+    rotation: str = "rpbh"      # "rpbh" | "block_rht" (identity permutation)
+    marginal: str = "gauss"     # codebook target: "gauss" (N(0, 1/d)) | "exact" (f_d)
+    fused_gelu: bool = False    # rows are pre-activations; the quantizer applies GELU itself
 
 
 def _outliers(d: int, frac: float) -> int:
@@ -74,6 +78,33 @@ WORKLOADS = {
         Projection("video_ffn_down_w3a4", 65520, 13824, 5120, 128, 3, 4, _bf16(),
                    _outliers(13824, 0.005), 100.0, "lognormal_cfg", cfg=4, proj=1),
     ],
+    # The MLP down projection quantized from the up projection's pre-activation u = z * scale
+    # (GELU applied by the quantizer: oq_quantize_act_gelu).
+    "flux_mlp_down_gelu_w2a4": [
+        Projection("flux_mlp_down_gelu_w2a4", 4608, 12288, 3072, 128, 2, 4, _bf16(),
+                   _outliers(12288, 0.01), 50.0, "lognormal", cfg=6, proj=0,
+                   fused_gelu=True)],
+    # W6A6, the setting the FLUX-3-Klein card gives its Qwen3-VL-4B text encoder: the
+    # language model's MLP (hidden 2560, intermediate 9728) on a 4096-token batch.
+    "text_encoder_w6a6": [
+        Projection("text_encoder_up_w6a6", 4096, 2560, 9728, 128, 6, 6, _bf16(),
+                   _outliers(2560, 0.01), 50.0, "lognormal", cfg=7, proj=0),
+        Projection("text_encoder_down_w6a6", 4096, 9728, 2560, 128, 6, 6, _bf16(),
+                   _outliers(9728, 0.01), 50.0, "lognormal", cfg=7, proj=1),
+    ],
+    # W2A3, the floor setting of the pages' Z-Image-Turbo remark, on the attention shape.
+    "flux_attn_w2a3": [Projection("flux_attn_w2a3", 4608, 3072, 3072, 128, 2, 3, _bf16(),
+                                  _outliers(3072, 0.01), 50.0, "lognormal", cfg=2, proj=0)],
+    # The attention projection under the Block-RHT ablation and under the exact-marginal
+    # codebook (same data as flux_attn_w4a4).
+    "flux_attn_w4a4_block_rht": [
+        Projection("flux_attn_w4a4_block_rht", 4608, 3072, 3072, 128, 4, 4, _bf16(),
+                   _outliers(3072, 0.01), 50.0, "lognormal", cfg=2, proj=0,
+                   rotation="block_rht")],
+    "flux_attn_w4a4_exact": [
+        Projection("flux_attn_w4a4_exact", 4608, 3072, 3072, 128, 4, 4, _bf16(),
+                   _outliers(3072, 0.01), 50.0, "lognormal", cfg=2, proj=0,
+                   marginal="exact")],
     "video_ffn_w4a8": [
         Projection("video_ffn_up_w4a8", 65520, 5120, 13824, 128, 4, 8, _bf16(),
                    _outliers(5120, 0.005), 100.0, "lognormal_cfg", cfg=4, proj=0),
@@ -146,6 +177,7 @@ def activations(p: Projection, rows: Optional[Sequence[int]] = None) -> torch.Te
         x[:, ch] *= p.outlier_scale
     if p.gelu:
         x = torch.nn.functional.gelu(x, approximate="none")
+    # (fused_gelu rows are left as pre-activations z * scale; the quantizer applies GELU)
     if p.token_scale == "lognormal":
         x *= torch.exp(_rows_scalar_normal(seed_of(p, 4), rows))[:, None]
     elif p.token_scale == "lognormal_cfg":
