@@ -26,7 +26,7 @@
 //     round-down, word = table[q >> F], code = (word + q*G) >> 24.  The table words fold the
 //     cell's base code and its boundary, so the decision is exact in the fixed-point q grid
 //     (2^-23 of the grid span, < 1.2e-6 sigma).  Bit widths 2/3/4/6/8 pack LSB-first.
-//   * Every mbarrier wait is bounded (2 s of %globaltimer); a wait that gives up sets a bit
+//   * Every mbarrier wait is bounded (about 2 s of SM clock); a wait that gives up sets a bit
 //     in the device error word (read by oq_check) and the round's outputs are not written.
 #include <cuda_bf16.h>
 
@@ -85,12 +85,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ unsigned long long globaltimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
@@ -100,19 +94,29 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
                  : "memory");
 }
 
-// Wait for the phase of the given parity; false after 2 s (the caller records an error).
+// A waiting thread may sleep in try_wait up to this long (it wakes when the phase completes).
+constexpr unsigned kSuspendHintNs = 200000;
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done) : "r"(bar), "r"(parity), "n"(kSuspendHintNs) : "memory");
+    return done != 0;
+}
+
+// Wait for the phase of the given parity; false after 4e9 SM cycles (about 2 s at the boost
+// clock; the caller records an error).  The first test reads no clock.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    const unsigned long long t0 = globaltimer();
+    if (mbar_try(bar, parity))
+        return true;
+    const long long t0 = clock64();
     for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-        if (done)
+        if (mbar_try(bar, parity))
             return true;
-        if (globaltimer() - t0 > 2000000000ull)
+        if (clock64() - t0 > 4000000000ll)
             return false;
     }
 }

@@ -14,7 +14,7 @@
 // other accumulator back with tcgen05.ld, apply the s_t * rn_o / d scale and hand 32 x 32
 // chunks to TMA tensor stores.  sigma^2 = 1/d is folded into the epilogue so the fp16 values
 // are unit-variance (best fp16 precision).  Every mbarrier wait is bounded by
-// wall time (%globaltimer); a wait that gives up sets a bit in the device error word.
+// SM clock cycles (about 2 s); a wait that gives up sets a bit in the device error word.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

@@ -313,8 +313,10 @@ struct oq_rpbh {
     std::vector<int32_t> perm;
     std::vector<int8_t> sign;
     std::vector<uint32_t> ent_img[2];             // K1 gather-entry images: [0] bf16, [1] fp32
+    std::vector<uint16_t> ent16;                  // tensor-core K1: perm[i] | sign bit << 15
     std::mutex mu;
     uint32_t *dev_ent[2][oq::kMaxDevices] = {};
+    uint32_t *dev_ent16[oq::kMaxDevices] = {};
 };
 
 struct oq_codebook {
@@ -448,6 +450,16 @@ int check_dims(int d, const char *who) {
     return OQ_OK;
 }
 
+// OQ_K1_PATH=tc sends bf16 rows (h <= 256, d up to ~3.9K) to the tensor-core rotate+quantize
+// kernel instead of the CUDA-core one (read once per process).
+bool tc_k1_requested() {
+    static const bool v = [] {
+        const char *e = std::getenv("OQ_K1_PATH");
+        return e != nullptr && std::strcmp(e, "tc") == 0;
+    }();
+    return v;
+}
+
 int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dtype, int rows,
                   int d, uint8_t *codes, float *norms, void *stream, float eps,
                   const char *who, bool gelu = false) {
@@ -477,11 +489,41 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
         return rc;
     oq_rpbh *rw = const_cast<oq_rpbh *>(r);
     oq_codebook *cw = const_cast<oq_codebook *>(cb);
+    if ((rc = upload(cw->mu, &cw->dev_tbl[dev], cw->tbl_img, "upload quantizer table")) != OQ_OK)
+        return rc;
+    const float Kq = (float)(std::sqrt((double)d / r->h) / (cb->G * cb->delta));
+    std::string why;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == OQ_BF16 && !gelu && tc_k1_requested() &&
+        oq::k1_tc_supported(d, r->h, cb->bits, (int)cw->tbl_img.size())) {
+        // block transform on the tensor cores
+        if ((rc = upload(rw->mu, &rw->dev_ent16[dev], rw->ent16, "upload rotation entries")) !=
+            OQ_OK)
+            return rc;
+        oq::K1TcParams p{};
+        p.x = static_cast<const uint8_t *>(x);
+        p.codes = codes;
+        p.norms = norms;
+        p.ent = reinterpret_cast<const uint16_t *>(rw->dev_ent16[dev]);
+        p.tbl_img = cw->dev_tbl[dev];
+        p.tbl_words = (int)cw->tbl_img.size();
+        p.T = rows;
+        p.d = d;
+        p.h = r->h;
+        p.eps = eps;
+        p.K = Kq;
+        p.G = cb->G;
+        p.F = cb->F;
+        cudaError_t e = timed(OQ_KERNEL_QUANTIZE, st, [&] {
+            return oq::launch_k1_tc(p, cb->bits, st, di->sms, &why);
+        });
+        if (e != cudaSuccess)
+            return fail_cuda(e, why.c_str());
+        return OQ_OK;
+    }
     const int f = dtype == OQ_F32 ? 1 : 0;
     if ((rc = upload(rw->mu, &rw->dev_ent[f][dev], rw->ent_img[f], "upload rotation table")) !=
         OQ_OK)
-        return rc;
-    if ((rc = upload(cw->mu, &cw->dev_tbl[dev], cw->tbl_img, "upload quantizer table")) != OQ_OK)
         return rc;
     oq::K1Params p{};
     p.x = x;
@@ -494,12 +536,10 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
     p.T = rows;
     p.d = d;
     p.eps = eps;
-    p.K = (float)(std::sqrt((double)d / r->h) / (cb->G * cb->delta));
+    p.K = Kq;
     p.G = cb->G;
     p.F = cb->F;
     p.gelu = gelu ? 1 : 0;
-    std::string why;
-    cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = timed(OQ_KERNEL_QUANTIZE, st, [&] {
         return oq::launch_k1(p, cb->bits, r->h, dtype == OQ_F32, st, di->sms, &why);
     });
@@ -578,6 +618,9 @@ int build_rotation(int d, int h, uint64_t seed, bool permute, oq_rpbh **out, con
     if (!permute)
         for (int i = 0; i < d; ++i)
             r->perm[i] = i;
+    r->ent16.resize(d);
+    for (int i = 0; i < d; ++i)
+        r->ent16[i] = (uint16_t)(r->perm[i] | (r->sign[i] < 0 ? 0x8000 : 0));
     // K1 gather-entry images (layout documented in oq_internal.h)
     for (int f = 0; f < 2; ++f) {
         r->ent_img[f].assign((size_t)(d / 32) * oq::kK1EntStride, 0u);
@@ -844,15 +887,19 @@ int oq_check(void *stream) {
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess)
         return fail_cuda(e, "oq_check: stream synchronize");
-    unsigned w1 = 0, w2 = 0;
+    unsigned w1 = 0, w2 = 0, w3 = 0;
     if ((e = oq::read_and_clear_k1_error(&w1, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k1 error word");
+    if ((e = oq::read_and_clear_k1tc_error(&w3, st)) != cudaSuccess)
+        return fail_cuda(e, "oq_check: read k1 (tensor-core) error word");
     if ((e = oq::read_and_clear_k2_error(&w2, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k2 error word");
-    if (w1 || w2)
-        return fail(OQ_EDEVICE, "device error word: quantize=0x%x linear=0x%x (a bounded wait "
-                                "gave up; quantize bit 1 = row copy, linear bits 1/2/4 = "
-                                "operand stage/ring slot/accumulator)", w1, w2);
+    if (w1 || w2 || w3)
+        return fail(OQ_EDEVICE, "device error word: quantize=0x%x quantize_tc=0x%x linear=0x%x "
+                                "(a bounded wait gave up; quantize bit 1 = row copy; quantize_tc "
+                                "bits 1/2/4/8/16 = staging/operand ring/accumulator/norm/code "
+                                "tile; linear bits 1/2/4 = operand stage/ring slot/accumulator)",
+                    w1, w3, w2);
     return OQ_OK;
 }
 
@@ -861,12 +908,17 @@ void oq_free_rpbh(oq_rpbh *r) {
         return;
     int cur = -1;
     cudaGetDevice(&cur);
-    for (int dev = 0; dev < oq::kMaxDevices; ++dev)
+    for (int dev = 0; dev < oq::kMaxDevices; ++dev) {
         for (int f = 0; f < 2; ++f)
             if (r->dev_ent[f][dev]) {
                 cudaSetDevice(dev);
                 cudaFree(r->dev_ent[f][dev]);
             }
+        if (r->dev_ent16[dev]) {
+            cudaSetDevice(dev);
+            cudaFree(r->dev_ent16[dev]);
+        }
+    }
     if (cur >= 0)
         cudaSetDevice(cur);
     delete r;

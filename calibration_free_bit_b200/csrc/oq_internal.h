@@ -42,6 +42,24 @@ struct K1Params {
     int gelu;               // 1: quantize R GELU(x) (erf form; bf16 input only)
 };
 
+// Tensor-core K1 (k1_tc.cu): bf16 rows; the block transform as tcgen05.mma.
+struct K1TcParams {
+    const uint8_t *x;          // [T, d] bf16 rows
+    uint8_t *codes;            // [T, d*bits/8]
+    float *norms;              // [T]
+    const uint16_t *ent;       // [d] perm[i] | (sign[i] < 0) << 15
+    const uint32_t *tbl_img;   // quantizer-table image (as K1)
+    int tbl_words;
+    int T, d, h;
+    float eps, K;              // as K1
+    int G, F;
+};
+bool k1_tc_supported(int d, int h, int bits, int tbl_words);
+size_t k1_tc_smem(int d, int tbl_words);
+cudaError_t launch_k1_tc(const K1TcParams &p, int bits, cudaStream_t st, int num_sms,
+                         std::string *why);
+cudaError_t read_and_clear_k1tc_error(unsigned *out, cudaStream_t st);
+
 // Launch K1 for (bits, h, dtype); `num_sms` sizes the grid.
 cudaError_t launch_k1(const K1Params &p, int bits, int h, int in_f32, cudaStream_t st,
                       int num_sms, std::string *why);

@@ -20,16 +20,12 @@ bool make_out_map(CUtensorMap *map, void *y, int T, int N, bool bf16);
 
 namespace sm100 {
 
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per bounded wait
+// A bounded wait gives up after this many SM clock cycles (about 2 s at the B200's 1.9 GHz
+// boost clock, longer at lower clocks).
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long globaltimer() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -45,19 +41,30 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
+// A waiting thread may sleep in try_wait up to this long (it wakes when the phase completes),
+// so warps parked on a barrier do not take issue slots from the warps doing the work.
+constexpr unsigned kSuspendHintNs = 200000;
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done) : "r"(bar), "r"(parity), "n"(kSuspendHintNs) : "memory");
+    return done != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after kWaitLimitCycles.  The
+// first test costs no clock read (most waits in a running pipeline are already satisfied).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    const unsigned long long t0 = globaltimer();
+    if (mbar_try(bar, parity))
+        return true;
+    const long long t0 = clock64();
     for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-        if (done)
+        if (mbar_try(bar, parity))
             return true;
-        if (globaltimer() - t0 > kWaitLimitNs)
+        if (clock64() - t0 > kWaitLimitCycles)
             return false;
     }
 }

@@ -121,7 +121,10 @@ int oq_quantize_weight(const oq_rpbh *r, const oq_codebook *cw, const void *W, i
  * x: device, [T, d] row-major of `dtype`.  x_codes: device, [T, d*ba/8] packed codes.
  * s: device, fp32 [T], the per-token norm ("the only input-dependent number at runtime").
  * A code is the number of sigma-scaled boundaries <= x_rot/(s+eps) (ties go up), decided in
- * fp32.  An all-zero row gives codes 2^ba/2 and s = 0.
+ * fp32.  An all-zero row gives codes 2^ba/2 and s = 0.  The rotation runs as register
+ * butterflies on the CUDA cores; with the environment variable OQ_K1_PATH=tc (read once per
+ * process) bf16 rows with h <= 256 and d up to about 3.9K use a kernel that runs the block
+ * transform as tcgen05 MMAs instead (same results under the same parity rules).
  * Errors: as oq_quantize_weight. */
 int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype, int T,
                     int d, uint8_t *x_codes, float *s, void *stream);

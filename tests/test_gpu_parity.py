@@ -414,3 +414,18 @@ def test_k1_fused_gelu_rejects_fp32(oq):
     r, cb = oq.oq_build_rpbh(256, 64, 0), oq.oq_lloyd_max(256, 4)
     with pytest.raises(oq.OQError):
         oq.oq_quantize_act(r, cb, torch.zeros(4, 256, device="cuda"), gelu=True)
+
+
+def test_k1_tensor_core_path(oq):
+    """With OQ_K1_PATH=tc, bf16 rows with h <= 256 and d up to ~3.9K go to the tensor-core
+    K1 (block transform as tcgen05.mma); a child process (the variable is read once per
+    process) checks it against the oracle under the same rules, on every supported h and
+    bit width, ragged tiles included."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, OQ_K1_PATH="tc")
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_k1_path_child.py")
+    r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stdout + r.stderr
