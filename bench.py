@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--workload", default="flux_attn_w4a4")
     ap.add_argument("--proj", type=int, default=0, help="projection index within the workload")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--api", choices=("forward", "calls"), default="forward",
+                    help="forward: oq_quantized_linear (one call, codes stay on chip); "
+                         "calls: oq_quantize_act then oq_linear")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -276,10 +279,16 @@ def run_ours(args, p, rank, world, dev):
         })
     torch.cuda.synchronize()
 
+    def run_path(b):
+        if args.api == "forward":
+            oq.oq_quantized_linear(r, ca, cw, b["x"], b["wc"], rn, y=b["y"], s=b["s"],
+                                   gelu=p.fused_gelu)
+        else:
+            oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"], gelu=p.fused_gelu)
+            oq.oq_linear(ca, cw, b["xc"], b["s"], b["wc"], rn, b["y"])
+
     def step(i):
-        b = sets[i % NSETS]
-        oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"], gelu=p.fused_gelu)
-        oq.oq_linear(ca, cw, b["xc"], b["s"], b["wc"], rn, b["y"])
+        run_path(sets[i % NSETS])
 
     def barrier():
         if world > 1:
@@ -354,7 +363,11 @@ def run_ours(args, p, rank, world, dev):
     clock_info = clocks.stop() if clocks else None
     oq.oq_check()
     ms_max = max_over_ranks(g0.elapsed_time(g1), world, dev)
-    launches = 4 * args.steps            # quantize, decode x, decode W, GEMM per step
+    # kernels per step: quantize, decode W, GEMM (+ decode x unless the quantizer writes the
+    # fp16 operand itself: forward path with 2/4/8-bit activations, bf16 x, h <= 256)
+    direct = (args.api == "forward" and p.bits_a in (2, 4, 8) and p.dtype == torch.bfloat16
+              and p.h <= 256)
+    launches = (3 if direct else 4) * args.steps
     del graphs
 
     # end-to-end through the public calls with host buffers (pinned), copies inside timing
@@ -384,8 +397,7 @@ def run_ours(args, p, rank, world, dev):
                 s_comp.wait_event(ev["in"][k])
                 if used[k]:
                     s_comp.wait_event(ev["out"][k])        # y[k] read out by step i - NB
-                oq.oq_quantize_act(r, ca, b["x"], b["xc"], b["s"], gelu=p.fused_gelu)
-                oq.oq_linear(ca, cw, b["xc"], b["s"], b["wc"], rn, b["y"])
+                run_path(b)
                 ev["comp"][k].record(s_comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev["comp"][k])
@@ -437,6 +449,8 @@ def run_ours(args, p, rank, world, dev):
         "dtype": "f16xf16->f32 (gemm), f32 (quantize)",
         "data": "synthetic",
         "config": workload_config(p, world),
+        "api": ("oq_quantized_linear (one call; x_codes stay on chip)" if args.api == "forward"
+                else "oq_quantize_act + oq_linear"),
         "kernels_ms_mean": {"quantize": quant_ms, "decode": dec_ms, "gemm": gemm_ms},
         "roofline": {
             "kernel": "k2_gemm (tcgen05 kind::f16, 128x256x64 tiles)",

@@ -14,6 +14,7 @@
 
 namespace oq {
 
+#if defined(__CUDACC__)
 __device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -38,6 +39,8 @@ __device__ __forceinline__ void decode8(uint32_t w, uint32_t L0, uint32_t L1, ui
     o[2] = prmt_b32(lo_b, hi_b, 0x5140) ^ (prmt_b32(y, nw, 0x6020) & 0x80008000u);
     o[3] = prmt_b32(lo_b, hi_b, 0x7362) ^ (prmt_b32(y, nw, 0x7030) & 0x80008000u);
 }
+
+#endif  // __CUDACC__
 
 // Host: the four permute sources from a 16-entry fp16 LUT; false unless the LUT is exactly
 // odd-symmetric (lut[15-i] == lut[i] ^ 0x8000), the condition decode8 relies on.

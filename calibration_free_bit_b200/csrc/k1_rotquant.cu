@@ -34,6 +34,9 @@
 #include <set>
 #include <tuple>
 
+#include <type_traits>
+
+#include "decode4.cuh"
 #include "oq_internal.h"
 
 namespace oq {
@@ -170,6 +173,48 @@ __device__ __forceinline__ void store_words(uint8_t *dst, const uint32_t (&w)[NW
     }
 }
 
+// 32 codes of one token (NW packed words, LSB-first) -> 32 fp16 unit centroids (16 words)
+// through the shared byte table `dect` (entry e of a byte: the centroids of the 8/BITS codes
+// it holds), stored as four 16-byte pieces.  BITS = 2, 4, 8.
+// 4-bit codes of the (odd-symmetric) codebook use the byte-permute decode instead (no table
+// loads): p.dec_src holds its four sources.
+template <int BITS>
+__device__ __forceinline__ void decode_store(const uint32_t *dect, const uint32_t (&w)[BITS],
+                                             uint4 *dst, const uint32_t (&src)[4]) {
+    uint32_t o[16];
+    if constexpr (BITS == 4) {                       // 8 codes a word -> 4 words of 2 fp16
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t q[4];
+            decode8(w[i], src[0], src[1], src[2], src[3], q);
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                o[4 * i + b] = q[b];
+        }
+    } else if constexpr (BITS == 2) {                // a byte = 4 codes = two words
+        const uint2 *d2 = reinterpret_cast<const uint2 *>(dect);
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const uint2 v = d2[(w[i] >> (8 * b)) & 0xffu];
+                o[8 * i + 2 * b] = v.x;
+                o[8 * i + 2 * b + 1] = v.y;
+            }
+    } else {                                         // a byte = 1 code = one fp16
+        const unsigned short *d16 = reinterpret_cast<const unsigned short *>(dect);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            o[2 * i] = (uint32_t)d16[w[i] & 0xffu] | ((uint32_t)d16[(w[i] >> 8) & 0xffu] << 16);
+            o[2 * i + 1] =
+                (uint32_t)d16[(w[i] >> 16) & 0xffu] | ((uint32_t)d16[w[i] >> 24] << 16);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+}
+
 // Per CTA: NG groups of d/32 threads, each group owns one token pair per round.  bf16 input:
 // the NEXT round's two rows stream into a raw buffer while the current round computes from
 // the interleaved pair buffer.  fp32 input: rows are gathered straight from `stages` raw
@@ -181,9 +226,12 @@ __device__ __forceinline__ float gelu_erf(float x) {
 
 // GELU (bf16 input only): the kernel quantizes R * GELU(x) instead of R * x; GELU is applied
 // to each gathered element before its sign flip (it is elementwise, so it commutes with P).
-template <int BITS, bool IN_F32, int H, bool GELU = false>
+// A16 (bf16 input, BITS = 2, 4, 8): instead of the packed codes, the kernel writes each code's
+// fp16 unit centroid to p.a16 [T, d] (the GEMM's A operand; the codes stay on chip).
+template <int BITS, bool IN_F32, int H, bool GELU = false, bool A16 = false>
 __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     static_assert(!(GELU && IN_F32), "fused GELU is bf16-only");
+    static_assert(!A16 || (!IN_F32 && (BITS == 2 || BITS == 4 || BITS == 8)), "A16 output");
     constexpr int Q = H / kE;                        // threads per h-block
     constexpr bool REPL = (BITS <= 4);               // per-lane table copies (conflict-free)
     constexpr int TSH = REPL ? 7 : 2;                // table row stride: 32 lanes x 4 B, or 4 B
@@ -204,10 +252,11 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     const unsigned wmask = active == 32 ? 0xffffffffu : ((1u << active) - 1u);
     const uint32_t row_in = (uint32_t)d * IN_BYTES;  // bytes of one input row
 
-    // shared memory: [table][entries][partials][mbarriers][raw rows][pair buffers (bf16)]
+    // shared memory: [table][entries][decode table][partials][mbarriers][raw rows][pairs]
     uint32_t *table = reinterpret_cast<uint32_t *>(smem);
     uint32_t *gent = table + p.tbl_words;
-    float2 *red = reinterpret_cast<float2 *>(gent + p.ent_words);
+    uint32_t *dect = gent + p.ent_words;             // A16 only (dec_words = 0 otherwise)
+    float2 *red = reinterpret_cast<float2 *>(dect + p.dec_words);
     unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + NG * kMaxSeg);
     unsigned char *raw = reinterpret_cast<unsigned char *>(bars + 2 * NG + 2);
     unsigned char *myraw = raw + (size_t)grp * nstage * 2 * row_in;
@@ -222,10 +271,12 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     }
     __syncthreads();
     if (tid == 0) {
-        // host-built table and entry images: two bulk copies
-        mbar_expect_tx(setup_bar, 4u * (p.tbl_words + p.ent_words));
+        // host-built table, entry and decode images: bulk copies
+        mbar_expect_tx(setup_bar, 4u * (p.tbl_words + p.ent_words + p.dec_words));
         bulk_copy(smem_u32(table), p.tbl_img, 4u * p.tbl_words, setup_bar);
         bulk_copy(smem_u32(gent), p.ent_img, 4u * p.ent_words, setup_bar);
+        if (p.dec_words > 0)
+            bulk_copy(smem_u32(dect), p.dec_img, 4u * p.dec_words, setup_bar);
     }
 
     // this thread's 32 rotated positions: pos0 + e with pos0 = g * 32
@@ -438,15 +489,22 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             }
         }
         if (valid) {
-            uint8_t *dst0 = p.codes + t0 * row_bytes + pos0 * BITS / 8;
-            store_words<NW>(dst0, w0);
+            if constexpr (A16) {
+                uint4 *a0 = reinterpret_cast<uint4 *>(p.a16 + t0 * d + pos0);
+                const uint32_t src[4] = {p.dec_src[0], p.dec_src[1], p.dec_src[2], p.dec_src[3]};
+                decode_store<BITS>(dect, w0, a0, src);
+                if (has1)
+                    decode_store<BITS>(dect, w1, a0 + d / 8, src);
+            } else {
+                uint8_t *dst0 = p.codes + t0 * row_bytes + pos0 * BITS / 8;
+                store_words<NW>(dst0, w0);
+                if (has1)
+                    store_words<NW>(dst0 + row_bytes, w1);
+            }
             if (g == 0)
                 p.norms[t0] = s0;
-            if (has1) {
-                store_words<NW>(dst0 + row_bytes, w1);
-                if (g == 0)
-                    p.norms[t1] = s1;
-            }
+            if (has1 && g == 0)
+                p.norms[t1] = s1;
         }
     }
 }
@@ -491,7 +549,7 @@ cudaError_t k1_prepare(const void *kern, int threads, size_t smem, int *per_sm) 
     return cudaSuccess;
 }
 
-template <int BITS, bool F32, bool GELU = false>
+template <int BITS, bool F32, bool GELU = false, bool A16 = false>
 cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int threads, size_t smem,
                      int num_sms, cudaStream_t st, std::string *why) {
     auto go = [&](auto kern) -> cudaError_t {
@@ -510,20 +568,30 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
             *why = "k1 launch";
         return e;
     };
-    switch (h) {
-        case 32: return go(k1_rotquant<BITS, F32, 32, GELU>);
-        case 64: return go(k1_rotquant<BITS, F32, 64, GELU>);
-        case 128: return go(k1_rotquant<BITS, F32, 128, GELU>);
-        case 256: return go(k1_rotquant<BITS, F32, 256, GELU>);
-        case 512: return go(k1_rotquant<BITS, F32, 512, GELU>);
-        case 1024: return go(k1_rotquant<BITS, F32, 1024, GELU>);
-        default: *why = "unsupported h"; return cudaErrorInvalidValue;
+    if constexpr (A16) {            // the fp16-output variants are built for h <= 256
+        switch (h) {
+            case 32: return go(k1_rotquant<BITS, F32, 32, GELU, true>);
+            case 64: return go(k1_rotquant<BITS, F32, 64, GELU, true>);
+            case 128: return go(k1_rotquant<BITS, F32, 128, GELU, true>);
+            case 256: return go(k1_rotquant<BITS, F32, 256, GELU, true>);
+            default: *why = "unsupported h for fp16 output"; return cudaErrorInvalidValue;
+        }
+    } else {
+        switch (h) {
+            case 32: return go(k1_rotquant<BITS, F32, 32, GELU>);
+            case 64: return go(k1_rotquant<BITS, F32, 64, GELU>);
+            case 128: return go(k1_rotquant<BITS, F32, 128, GELU>);
+            case 256: return go(k1_rotquant<BITS, F32, 256, GELU>);
+            case 512: return go(k1_rotquant<BITS, F32, 512, GELU>);
+            case 1024: return go(k1_rotquant<BITS, F32, 1024, GELU>);
+            default: *why = "unsupported h"; return cudaErrorInvalidValue;
+        }
     }
 }
 
 size_t k1_smem(const K1Params &p, int in_f32, int NG, int stages) {
     const size_t row_in = (size_t)p.d * (in_f32 ? 4 : 2);
-    size_t b = 4 * (size_t)(p.tbl_words + p.ent_words);    // table + gather entries
+    size_t b = 4 * (size_t)(p.tbl_words + p.ent_words + p.dec_words);   // tables, entries
     b += sizeof(float2) * NG * kMaxSeg;                    // norm partials
     b += 8 * (size_t)(2 * NG + 2);                         // mbarriers
     b += (size_t)NG * stages * 2 * row_in;                 // raw rows
@@ -558,6 +626,22 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     p.stages = stages;
     const int threads = NG * GT;
     const long long ctas_needed = (npairs + NG - 1) / NG;
+    if (p.a16) {
+        if (in_f32) {
+            *why = "fp16 centroid output takes bf16 input";
+            return cudaErrorInvalidValue;
+        }
+        auto go16 = [&](auto gelu_tag) -> cudaError_t {
+            constexpr bool GL = decltype(gelu_tag)::value;
+            switch (bits) {
+                case 2: return launch_h<2, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+                case 4: return launch_h<4, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+                case 8: return launch_h<8, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+                default: *why = "fp16 centroid output: bit width"; return cudaErrorInvalidValue;
+            }
+        };
+        return p.gelu ? go16(std::true_type{}) : go16(std::false_type{});
+    }
     if (p.gelu) {
         if (in_f32) {
             *why = "fused GELU takes bf16 input";

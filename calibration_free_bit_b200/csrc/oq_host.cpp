@@ -13,6 +13,7 @@
 #include <limits>
 #include <new>
 
+#include "decode4.cuh"
 #include "oq_internal.h"
 
 namespace {
@@ -327,8 +328,10 @@ struct oq_codebook {
     double delta = 0.0;
     std::vector<uint32_t> grid;                   // G + 1 words
     std::vector<uint32_t> tbl_img;                // K1 shared-memory image of the table
+    std::vector<uint32_t> dec_img;                // K1 fp16 output: byte -> centroids (b 2,4,8)
     std::mutex mu;
     uint32_t *dev_tbl[oq::kMaxDevices] = {};
+    uint32_t *dev_dec[oq::kMaxDevices] = {};
 };
 
 namespace {
@@ -393,6 +396,8 @@ struct DeviceInfo {
     int checked = 0;       // 0 unknown, 1 ok, -1 unsupported
     int sms = 0;
     cudaMemPool_t pool = nullptr;
+    cudaStream_t side = nullptr;      // oq_quantized_linear: weight decode beside K1
+    cudaEvent_t fork = nullptr, join = nullptr;
 };
 DeviceInfo g_dev[oq::kMaxDevices];
 std::mutex g_dev_mu;
@@ -460,9 +465,11 @@ bool tc_k1_requested() {
     return v;
 }
 
+// K1 for `rows` rows of x: packed codes into `codes`, or (a16 non-null, bits 2/4/8, bf16, h <=
+// 256) the codes' fp16 unit centroids into a16 [rows, d]; norms into `norms`.
 int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dtype, int rows,
                   int d, uint8_t *codes, float *norms, void *stream, float eps,
-                  const char *who, bool gelu = false) {
+                  const char *who, bool gelu = false, uint16_t *a16 = nullptr) {
     if (!r || !cb)
         return fail(OQ_EINVAL, "%s: null handle", who);
     if (check_dims(d, who) != OQ_OK)
@@ -478,9 +485,10 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
         return fail(OQ_EINVAL, "%s: negative row count %d", who, rows);
     if (rows == 0)
         return OQ_OK;
-    if (!x || !codes || !norms)
+    uint8_t *out = a16 ? reinterpret_cast<uint8_t *>(a16) : codes;
+    if (!x || !out || !norms)
         return fail(OQ_EINVAL, "%s: null data pointer", who);
-    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(norms) & 3u))
+    if (!aligned16(x) || !aligned16(out) || (reinterpret_cast<uintptr_t>(norms) & 3u))
         return fail(OQ_EINVAL, "%s: x and codes must be 16-byte aligned, norms 4-byte", who);
     int dev;
     DeviceInfo *di;
@@ -494,7 +502,7 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
     const float Kq = (float)(std::sqrt((double)d / r->h) / (cb->G * cb->delta));
     std::string why;
     cudaStream_t st = (cudaStream_t)stream;
-    if (dtype == OQ_BF16 && !gelu && tc_k1_requested() &&
+    if (dtype == OQ_BF16 && !gelu && !a16 && tc_k1_requested() &&
         oq::k1_tc_supported(d, r->h, cb->bits, (int)cw->tbl_img.size())) {
         // block transform on the tensor cores
         if ((rc = upload(rw->mu, &rw->dev_ent16[dev], rw->ent16, "upload rotation entries")) !=
@@ -540,6 +548,22 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
     p.G = cb->G;
     p.F = cb->F;
     p.gelu = gelu ? 1 : 0;
+    if (a16) {
+        if (!oq::k1_a16_supported(cb->bits, r->h, dtype == OQ_BF16))
+            return fail(OQ_EINVAL, "%s: no fp16 centroid output for bits %d, h %d", who,
+                        cb->bits, r->h);
+        if ((rc = upload(cw->mu, &cw->dev_dec[dev], cw->dec_img, "upload decode table")) != OQ_OK)
+            return rc;
+        p.a16 = a16;
+        if (cb->bits == 4) {
+            if (!oq::decode8_sources(cb->lut, &p.dec_src[0], &p.dec_src[1], &p.dec_src[2],
+                                     &p.dec_src[3]))
+                return fail(OQ_EINVAL, "%s: 4-bit codebook is not odd-symmetric", who);
+        } else {
+            p.dec_img = cw->dev_dec[dev];
+            p.dec_words = (int)cw->dec_img.size();
+        }
+    }
     cudaError_t e = timed(OQ_KERNEL_QUANTIZE, st, [&] {
         return oq::launch_k1(p, cb->bits, r->h, dtype == OQ_F32, st, di->sms, &why);
     });
@@ -566,6 +590,32 @@ cudaMemPool_t device_pool(int dev, DeviceInfo *di, int *rc) {
     cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
     di->pool = pool;
     return pool;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// The library's side stream of a device and the two events oq_quantized_linear forks and joins
+// it with (created once; nullptr and *rc set on failure).
+std::mutex g_side_mu;          // serialises the fork/join enqueues of concurrent callers
+cudaStream_t device_side(DeviceInfo *di, int *rc) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (di->side)
+        return di->side;
+    cudaStream_t st = nullptr;
+    cudaEvent_t a = nullptr, b = nullptr;
+    cudaError_t e = cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking);
+    if (e == cudaSuccess)
+        e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
+    if (e == cudaSuccess)
+        e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+        *rc = fail_cuda(e, "side stream / events");
+        return nullptr;
+    }
+    di->fork = a;
+    di->join = b;
+    di->side = st;
+    return st;
 }
 
 // OQ_LINEAR_PATH=fused decodes 4-bit activation codes inside the GEMM kernel instead of in
@@ -695,6 +745,17 @@ int oq_lloyd_max_marginal(int d, int bits, int marginal, oq_codebook **out) {
     if (!build_grid(cb)) {
         delete cb;
         return fail(OQ_EINVAL, "%s: could not build the quantizer grid", who);
+    }
+    // K1 fp16-output image: entry e (a byte of packed codes) = the fp16 centroids of the
+    // 8/bits codes in it, lowest code first (bits 2: four, 4: two, 8: one per entry)
+    if (bits == 2 || bits == 4 || bits == 8) {
+        const int per = 8 / bits;
+        std::vector<uint16_t> tab((size_t)256 * per);
+        for (int e = 0; e < 256; ++e)
+            for (int i = 0; i < per; ++i)
+                tab[(size_t)e * per + i] = cb->lut[(e >> (i * bits)) & (L - 1)];
+        cb->dec_img.assign((tab.size() / 2 + 3) / 4 * 4, 0u);
+        std::memcpy(cb->dec_img.data(), tab.data(), tab.size() * 2);
     }
     // K1 table image: one copy per lane when bits <= 4 (conflict-free lookups), padded to 16 B
     const int copies = bits <= 4 ? 32 : 1;
@@ -882,6 +943,114 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
     return OQ_OK;
 }
 
+int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebook *cw,
+                        const void *x, int dtype, const uint8_t *W_codes, const float *row_norms,
+                        int T, int d, int out_features, void *y, int out_dtype, float *s,
+                        int flags, void *stream) {
+    const char *who = "oq_quantized_linear";
+    if (!r || !ca || !cw)
+        return fail(OQ_EINVAL, "%s: null handle", who);
+    if (check_dims(d, who) != OQ_OK)
+        return OQ_EINVAL;
+    if (r->d != d || ca->d != d || cw->d != d)
+        return fail(OQ_EINVAL, "%s: d = %d but rotation/codebooks have d = %d / %d / %d", who,
+                    d, r->d, ca->d, cw->d);
+    if (dtype != OQ_F32 && dtype != OQ_BF16)
+        return fail(OQ_EINVAL, "%s: dtype must be OQ_F32 or OQ_BF16", who);
+    if (out_dtype != OQ_F32 && out_dtype != OQ_BF16)
+        return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32 or OQ_BF16", who);
+    if (flags & ~OQ_FORWARD_GELU)
+        return fail(OQ_EINVAL, "%s: unknown flags 0x%x", who, flags);
+    const bool gelu = (flags & OQ_FORWARD_GELU) != 0;
+    if (gelu && dtype != OQ_BF16)
+        return fail(OQ_EINVAL, "%s: OQ_FORWARD_GELU takes bf16 input", who);
+    if (T < 0 || out_features < 1 || out_features % 16 != 0)
+        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
+                               "multiple of 16", who, T, out_features);
+    if (T == 0)
+        return OQ_OK;
+    if (!x || !W_codes || !row_norms || !y)
+        return fail(OQ_EINVAL, "%s: null data pointer", who);
+    if (!aligned16(x) || !aligned16(W_codes) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(row_norms) & 3u) || (reinterpret_cast<uintptr_t>(s) & 3u))
+        return fail(OQ_EINVAL, "%s: x, W_codes and y must be 16-byte aligned, row_norms and s "
+                               "4-byte", who);
+    int dev;
+    DeviceInfo *di;
+    int rc = current_device(&dev, &di);
+    if (rc != OQ_OK)
+        return rc;
+    cudaMemPool_t pool = device_pool(dev, di, &rc);
+    if (!pool)
+        return rc;
+    cudaStream_t side = device_side(di, &rc);
+    if (!side)
+        return rc;
+    // workspace: A16 [T, d] fp16 | B16 [N, d] fp16 | s [T] (if not given) | codes (fallback)
+    const bool direct = oq::k1_a16_supported(ca->bits, r->h, dtype == OQ_BF16);
+    const size_t a_bytes = align_up((size_t)T * d * 2, 1024);
+    const size_t b_bytes = align_up((size_t)out_features * d * 2, 1024);
+    const size_t s_bytes = s ? 0 : align_up((size_t)T * 4, 1024);
+    const size_t c_bytes = direct ? 0 : align_up((size_t)T * d * ca->bits / 8, 1024);
+    void *ws = nullptr;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, a_bytes + b_bytes + s_bytes + c_bytes, pool, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "oq_quantized_linear: workspace allocation");
+    unsigned char *w8 = static_cast<unsigned char *>(ws);
+    uint16_t *A16 = reinterpret_cast<uint16_t *>(w8);
+    uint16_t *B16 = reinterpret_cast<uint16_t *>(w8 + a_bytes);
+    float *sv = s ? s : reinterpret_cast<float *>(w8 + a_bytes + b_bytes);
+    uint8_t *codes = direct ? nullptr : w8 + a_bytes + b_bytes + s_bytes;
+    std::string why;
+    {
+        // the weight decode needs nothing from x: it runs on the side stream beside K1
+        std::lock_guard<std::mutex> lk(g_side_mu);
+        e = cudaEventRecord(di->fork, st);
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(side, di->fork, 0);
+        if (e == cudaSuccess)
+            e = timed(OQ_KERNEL_DECODE, side, [&] {
+                return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, side,
+                                         di->sms, &why);
+            });
+        if (e == cudaSuccess)
+            e = cudaEventRecord(di->join, side);
+    }
+    if (e != cudaSuccess) {
+        cudaFreeAsync(ws, st);
+        return fail_cuda(e, why.empty() ? "oq_quantized_linear: side stream" : why.c_str());
+    }
+    rc = quantize_rows(r, ca, x, dtype, T, d, codes, sv, st, 1e-8f, who, gelu,
+                       direct ? A16 : nullptr);
+    if (rc == OQ_OK && !direct) {
+        e = timed(OQ_KERNEL_DECODE, st, [&] {
+            return oq::launch_decode(ca->bits, codes, A16, T, d, ca->lut, st, di->sms, &why);
+        });
+        if (e != cudaSuccess)
+            rc = fail_cuda(e, why.c_str());
+    }
+    // the GEMM waits for the weight operand (join) whether or not K1 succeeded, so the
+    // workspace is released after every use of it
+    e = cudaStreamWaitEvent(st, di->join, 0);
+    if (rc == OQ_OK && e == cudaSuccess) {
+        e = timed(OQ_KERNEL_GEMM, st, [&] {
+            return oq::launch_gemm(A16, nullptr, nullptr, B16, sv, row_norms, y,
+                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why);
+        });
+        if (e != cudaSuccess)
+            rc = fail_cuda(e, why.c_str());
+    } else if (rc == OQ_OK) {
+        rc = fail_cuda(e, "oq_quantized_linear: join");
+    }
+    cudaError_t e2 = cudaFreeAsync(ws, st);
+    if (rc != OQ_OK)
+        return rc;
+    if (e2 != cudaSuccess)
+        return fail_cuda(e2, "oq_quantized_linear: workspace release");
+    return OQ_OK;
+}
+
 int oq_check(void *stream) {
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaStreamSynchronize(st);
@@ -929,11 +1098,16 @@ void oq_free_codebook(oq_codebook *cb) {
         return;
     int cur = -1;
     cudaGetDevice(&cur);
-    for (int dev = 0; dev < oq::kMaxDevices; ++dev)
+    for (int dev = 0; dev < oq::kMaxDevices; ++dev) {
         if (cb->dev_tbl[dev]) {
             cudaSetDevice(dev);
             cudaFree(cb->dev_tbl[dev]);
         }
+        if (cb->dev_dec[dev]) {
+            cudaSetDevice(dev);
+            cudaFree(cb->dev_dec[dev]);
+        }
+    }
     if (cur >= 0)
         cudaSetDevice(cur);
     delete cb;

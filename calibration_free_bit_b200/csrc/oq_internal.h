@@ -40,7 +40,17 @@ struct K1Params {
     int groups;             // token pairs processed at once per CTA (set by launch_k1)
     int stages;             // raw row buffers per group, fp32 input only (set by launch_k1)
     int gelu;               // 1: quantize R GELU(x) (erf form; bf16 input only)
+    uint16_t *a16;          // non-null: write fp16 unit centroids [T, d] here, not codes
+    const uint32_t *dec_img;   // byte -> centroid table for a16 (bits 2, 8)
+    int dec_words;             // its size in words (multiple of 4; 0 without a16)
+    uint32_t dec_src[4];       // a16 with 4-bit codes: byte-permute decode sources
 };
+// True when K1 can write fp16 centroids itself (launch_k1 with p.a16 set).
+inline bool k1_a16_supported(int bits, int h, bool bf16_in) {
+    return bf16_in && h <= 256 && (bits == 2 || bits == 4 || bits == 8);
+}
+// (4-bit additionally needs an odd-symmetric codebook, which every Lloyd-Max codebook here is;
+// the host checks it when it builds dec_src.)
 
 // Tensor-core K1 (k1_tc.cu): bf16 rows; the block transform as tcgen05.mma.
 struct K1TcParams {

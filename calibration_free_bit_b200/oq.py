@@ -55,6 +55,8 @@ def lib():
     L.oq_quantize_act.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.oq_quantize_act_gelu.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, vp]
     L.oq_linear.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp]
+    L.oq_quantized_linear.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, vp, i32, vp,
+                                      i32, vp]
     L.oq_linear_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, i32, vp]
     L.oq_check.argtypes = [vp]
     L.oq_free_rpbh.argtypes = [vp]
@@ -68,7 +70,7 @@ def lib():
     for name in ("oq_build_rpbh", "oq_build_block_rht", "oq_rpbh_tables", "oq_lloyd_max", "oq_lloyd_max_marginal",
                  "oq_codebook_values",
                  "oq_codebook_grid", "oq_quantize_weight", "oq_quantize_act",
-                 "oq_quantize_act_gelu", "oq_linear",
+                 "oq_quantize_act_gelu", "oq_linear", "oq_quantized_linear",
                  "oq_linear_noalloc", "oq_check", "oq_timing_enable", "oq_timing_collect"):
         getattr(L, name).restype = i32
     _lib = L
@@ -234,6 +236,23 @@ def oq_linear(ca: Codebook, cw: Codebook, x_codes: torch.Tensor, s: torch.Tensor
     y = _out(y, T, N, out_dtype, x_codes.device)
     _check(lib().oq_linear(ca.handle, cw.handle, _ptr(x_codes), _ptr(s), _ptr(W_codes),
                            _ptr(row_norms), T, d, N, _ptr(y), _dtype_code(y), _stream(stream)))
+    return y
+
+
+OQ_FORWARD_GELU = 1
+
+
+def oq_quantized_linear(r: RPBH, ca: Codebook, cw: Codebook, x: torch.Tensor,
+                        W_codes: torch.Tensor, row_norms: torch.Tensor, y=None, s=None,
+                        stream=None, out_dtype=torch.float32, gelu: bool = False):
+    """The online path in one call: y = oq_linear(oq_quantize_act(x)) without x_codes in
+    memory (with gelu=True: of GELU(x)).  Returns y; the norms go to s when given."""
+    T, d, N = x.shape[0], x.shape[1], W_codes.shape[0]
+    y = _out(y, T, N, out_dtype, x.device)
+    _check(lib().oq_quantized_linear(r.handle, ca.handle, cw.handle, _ptr(x), _dtype_code(x),
+                                     _ptr(W_codes), _ptr(row_norms), T, d, N, _ptr(y),
+                                     _dtype_code(y), _ptr(s), OQ_FORWARD_GELU if gelu else 0,
+                                     _stream(stream)))
     return y
 
 

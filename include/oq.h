@@ -157,6 +157,28 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
               const float *s, const uint8_t *W_codes, const float *row_norms, int T, int d,
               int out_features, void *y, int out_dtype, void *stream);
 
+#define OQ_FORWARD_GELU 1u   /* oq_quantized_linear flag: the input is a GELU pre-activation */
+
+/* The whole online path in one call: y = W_hat x_hat with x_hat the activation step of x
+ * ([RCAP] pseudocode, online part, and rotation-cancellation paragraph), i.e. the result of
+ * oq_quantize_act followed by oq_linear, without materialising x_codes: the rotate+quantize
+ * kernel writes each code's fp16 unit centroid straight into the GEMM's A operand (bf16 x,
+ * ba in {2, 4, 8}, h <= 256; otherwise codes and the decode prepass are used inside the
+ * call), and the weight codes are decoded on a library-owned side stream of the device
+ * while x is quantized.  y and s are bit-identical to oq_quantize_act + oq_linear.
+ * x: device [T, d] of dtype; W_codes [out_features, d*bw/8]; row_norms fp32 [out_features];
+ * y: device [T, out_features] of out_dtype (OQ_F32 or OQ_BF16); s: optional device fp32 [T]
+ * receiving the norms (NULL: kept internal).  flags: OQ_FORWARD_GELU quantizes GELU(x)
+ * (as oq_quantize_act_gelu; bf16 x).  Temporary device memory comes from the library's
+ * stream-ordered pool.  The side stream and its fork/join events are per device and shared
+ * by all callers (enqueues are serialised); while a graph capture is open on one host
+ * thread, no other thread may call this function on the same device.
+ * Errors: as oq_quantize_act and oq_linear. */
+int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebook *cw,
+                        const void *x, int dtype, const uint8_t *W_codes, const float *row_norms,
+                        int T, int d, int out_features, void *y, int out_dtype, float *s,
+                        int flags, void *stream);
+
 /* oq_linear for callers that cannot allocate device memory.  The paper has no counterpart;
  * this is a deployment variant of the same computation, with the same arguments, result and
  * errors as oq_linear.

@@ -429,3 +429,39 @@ def test_k1_tensor_core_path(oq):
     r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
                        timeout=900)
     assert r.returncode == 0, r.stdout + r.stderr
+
+
+
+@pytest.mark.parametrize("d,h,ba,bw,T,N,gelu,out", [
+    (3072, 128, 4, 4, 4608, 3072, False, torch.float32),    # the attention projection
+    (384, 128, 4, 2, 37, 272, False, torch.float32),        # ragged T and N
+    (1024, 64, 2, 8, 129, 512, False, torch.bfloat16),
+    (2048, 256, 8, 4, 33, 160, False, torch.float32),
+    (1024, 128, 3, 4, 65, 256, False, torch.float32),       # fallback: codes + decode
+    (2560, 128, 6, 6, 50, 336, False, torch.float32),       # fallback: 6-bit
+    (2048, 512, 4, 4, 40, 128, False, torch.float32),       # fallback: h = 512
+    (3072, 128, 4, 2, 100, 384, True, torch.float32),       # GELU pre-activation
+])
+def test_quantized_linear_matches_the_two_calls(oq, d, h, ba, bw, T, N, gelu, out):
+    """oq_quantized_linear (x -> y, codes never in memory) is bit-identical to
+    oq_quantize_act (or _gelu) followed by oq_linear: y and the norms s."""
+    p = synth.sweep_projection(d, 128, 4, T) if d != 3072 or T != 4608 else \
+        synth.get("flux_attn_w4a4")[0]
+    x = synth.activations(p).cuda()
+    W = (torch.randn(N, d, generator=torch.Generator().manual_seed(d + N)) /
+         math.sqrt(d)).cuda()
+    r = oq.oq_build_rpbh(d, h, 0)
+    ca, cw = oq.oq_lloyd_max(d, ba), oq.oq_lloyd_max(d, bw)
+    wc, rn = oq.oq_quantize_weight(r, cw, W)
+    xc, s_ref = oq.oq_quantize_act(r, ca, x, gelu=gelu)
+    y_ref = oq.oq_linear(ca, cw, xc, s_ref, wc, rn, out_dtype=out)
+    s = torch.empty(T, device="cuda")
+    y = oq.oq_quantized_linear(r, ca, cw, x, wc, rn, s=s, out_dtype=out, gelu=gelu)
+    oq.oq_check()
+    assert torch.equal(s, s_ref)
+    assert torch.equal(y.view(torch.int32 if out == torch.float32 else torch.int16),
+                       y_ref.view(torch.int32 if out == torch.float32 else torch.int16))
+    # and without the norms output (kept internal)
+    y2 = oq.oq_quantized_linear(r, ca, cw, x, wc, rn, out_dtype=out, gelu=gelu)
+    oq.oq_check()
+    assert torch.equal(y2, y)

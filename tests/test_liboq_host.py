@@ -85,6 +85,29 @@ def test_exact_marginal_codebook_matches_oracle(d, bits, tol):
     assert np.all(np.abs(c) < 1.0) and np.all(np.diff(c) > 0)
 
 
+def test_quantized_linear_validation_without_a_gpu():
+    L = oq.lib()
+    r = oq.oq_build_rpbh(3072, 128)
+    ca = oq.oq_lloyd_max(3072, 4)
+    c_other = oq.oq_lloyd_max(1024, 4)
+    fake = 1 << 20
+    args = lambda **kw: dict(dict(r=r.handle, ca=ca.handle, cw=ca.handle, x=fake,    # noqa
+                                  dtype=oq.OQ_BF16, wc=fake, rn=fake, T=8, d=3072, N=128,
+                                  y=fake, od=oq.OQ_F32, s=None, flags=0), **kw)
+
+    def call(a):
+        return L.oq_quantized_linear(a["r"], a["ca"], a["cw"], a["x"], a["dtype"], a["wc"],
+                                     a["rn"], a["T"], a["d"], a["N"], a["y"], a["od"], a["s"],
+                                     a["flags"], None)
+    assert call(args(flags=4)) == oq.OQ_EINVAL                        # unknown flag
+    assert call(args(flags=1, dtype=oq.OQ_F32)) == oq.OQ_EINVAL       # GELU needs bf16
+    assert call(args(cw=c_other.handle)) == oq.OQ_EINVAL              # d mismatch
+    assert call(args(N=100)) == oq.OQ_EINVAL                          # N not a multiple of 16
+    assert call(args(x=fake + 4)) == oq.OQ_EINVAL                     # misaligned x
+    assert call(args(s=fake + 2)) == oq.OQ_EINVAL                     # misaligned s
+    assert call(args(T=0, x=None, wc=None, rn=None, y=None)) == oq.OQ_OK
+
+
 def test_exact_marginal_rejects_small_d():
     h = C.c_void_p()
     assert oq.lib().oq_lloyd_max_marginal(2, 4, 1, C.byref(h)) == oq.OQ_EINVAL
