@@ -437,7 +437,10 @@ def run_ours(args, p, rank, world, dev):
     gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
     traffic, traffic_src = profile_traffic(f"k2_gemm_{p.name}.md", GEMM_SOURCES)
     in_bytes = 2 if p.dtype == torch.bfloat16 else 4
-    q_bytes = p.T * (in_bytes * p.d + p.d * p.bits_a // 8 + 4)
+    # K1's algorithmic bytes: x in, then the packed codes, or on the one-call path the fp16
+    # centroids it writes for the GEMM instead, and s
+    out_bytes = 2 * p.d if direct else p.d * p.bits_a // 8
+    q_bytes = p.T * (in_bytes * p.d + out_bytes + 4)
     q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
@@ -463,7 +466,8 @@ def run_ours(args, p, rank, world, dev):
             "algorithmic_per_launch": flops,
         },
         "roofline_quantize": {
-            "kernel": "k1_rotquant", "bound": "hbm", "achieved": q_gbs,
+            "kernel": "k1_rotquant (fp16-operand output)" if direct else "k1_rotquant",
+            "bound": "hbm", "achieved": q_gbs,
             "peak": pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "unit": "GB/s",
             "frac": q_gbs / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
             "frac_of_8TBps_nominal": q_gbs / 8000.0,
@@ -472,7 +476,9 @@ def run_ours(args, p, rank, world, dev):
         "gpu_launches": launches,
         "timing": f"value/ms_per_step: {timing_mode} of the step; kernels_ms_mean and the "
                   f"rooflines: CUDA events around each kernel of {n_k} eager steps queued "
-                  "behind a GPU spin (device time, not host gaps)",
+                  "behind a GPU spin (device time, not host gaps); on the one-call path the "
+                  "decode (weights) runs on a side stream beside K1, so its event time "
+                  "includes that overlap",
         "eager_ms_per_step": eager_ms / args.steps,
         "host_ms_per_step_eager": host_ms / args.steps,
         "clocks": clock_info,
