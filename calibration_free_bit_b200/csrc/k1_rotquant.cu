@@ -228,9 +228,14 @@ __device__ __forceinline__ float gelu_erf(float x) {
 // to each gathered element before its sign flip (it is elementwise, so it commutes with P).
 // A16 (bf16 input, BITS = 2, 4, 8): instead of the packed codes, the kernel writes each code's
 // fp16 unit centroid to p.a16 [T, d] (the GEMM's A operand; the codes stay on chip).
-template <int BITS, bool IN_F32, int H, bool GELU = false, bool A16 = false>
+// NAMED (bf16 input, groups of whole warps): each group synchronises on its own named barrier
+// and takes pairs from a shared counter; the kernel then reserves all 16 barriers of the SM's
+// CTA slot, so it is launched one CTA per SM.  Otherwise the CTA synchronises as a whole and
+// its groups step through the CTA's pairs in lockstep.
+template <int BITS, bool IN_F32, int H, bool GELU = false, bool A16 = false, bool NAMED = false>
 __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     static_assert(!(GELU && IN_F32), "fused GELU is bf16-only");
+    static_assert(!(NAMED && IN_F32), "named-barrier groups are bf16-only");
     static_assert(!A16 || (!IN_F32 && (BITS == 2 || BITS == 4 || BITS == 8)), "A16 output");
     constexpr int Q = H / kE;                        // threads per h-block
     constexpr bool REPL = (BITS <= 4);               // per-lane table copies (conflict-free)
@@ -251,14 +256,22 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     const int active = min(32, (int)blockDim.x - warp_start);
     const unsigned wmask = active == 32 ? 0xffffffffu : ((1u << active) - 1u);
     const uint32_t row_in = (uint32_t)d * IN_BYTES;  // bytes of one input row
+    // NAMED: a group waits only for its own threads (named barrier 1 + grp, GT threads)
+    auto group_sync = [&]() {
+        if constexpr (NAMED)
+            asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(GT) : "memory");
+        else
+            __syncthreads();
+    };
 
     // shared memory: [table][entries][decode table][partials][mbarriers][raw rows][pairs]
     uint32_t *table = reinterpret_cast<uint32_t *>(smem);
     uint32_t *gent = table + p.tbl_words;
     uint32_t *dect = gent + p.ent_words;             // A16 only (dec_words = 0 otherwise)
     float2 *red = reinterpret_cast<float2 *>(dect + p.dec_words);
-    unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + NG * kMaxSeg);
-    unsigned char *raw = reinterpret_cast<unsigned char *>(bars + 2 * NG + 2);
+    unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + 2 * NG * kMaxSeg);
+    int *sched = reinterpret_cast<int *>(bars + 2 * NG + 2);   // [0] next pair, [1 + grp]
+    unsigned char *raw = reinterpret_cast<unsigned char *>(sched + 16);
     unsigned char *myraw = raw + (size_t)grp * nstage * 2 * row_in;
     unsigned char *pairs = raw + (size_t)NG * nstage * 2 * row_in;
     unsigned char *mypairs = pairs + (size_t)grp * d * 4;
@@ -267,6 +280,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     if (tid == 0) {
         for (int b = 0; b < 2 * NG + 1; ++b)
             mbar_init(smem_u32(&bars[b]), 1);
+        sched[0] = NG;                               // pairs lo .. lo + NG - 1 start the groups
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -294,14 +308,23 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     const int nslots = 1 + ((grp * GT + GT - 1) / 32 - (grp * GT) / 32);
     const int row_bytes = d * BITS / 8;
     const long long npairs = ((long long)p.T + 1) / 2;
-    const long long stride = (long long)gridDim.x * NG;
+    // The group's pairs are lo + my for my < cnt.  NAMED: the CTA owns an equal contiguous
+    // share of all pairs and its groups take them from a shared counter (a group that finishes
+    // early takes the next one).  Otherwise all groups of all CTAs step through the pairs in
+    // lockstep rounds of gridDim.x * NG, and a CTA leaves once its next round is empty.
+    constexpr bool dyn = NAMED;
+    const long long lo = dyn ? (long long)blockIdx.x * npairs / gridDim.x
+                             : (long long)blockIdx.x * NG;
+    const int cnt = (int)(dyn ? ((long long)blockIdx.x + 1) * npairs / gridDim.x - lo
+                              : npairs - lo);
+    const int step = dyn ? NG : (int)gridDim.x * NG;
     const unsigned char *xb = static_cast<const unsigned char *>(p.x);
 
-    // the two rows of pair `pr` into raw stage `s` (one thread per group issues)
-    auto issue = [&](long long pr, int s) {
-        if (g != 0 || pr >= npairs)
+    // the two rows of pair lo + i into raw stage `s` (one thread per group issues)
+    auto issue = [&](int i, int s) {
+        if (g != 0 || i >= cnt)
             return;
-        const long long t0 = 2 * pr;
+        const long long t0 = 2 * (lo + i);
         const bool two = t0 + 1 < p.T;
         const uint32_t bar = smem_u32(&bars[2 * grp + s]);
         const uint32_t dst = smem_u32(myraw + (size_t)s * 2 * row_in);
@@ -311,14 +334,16 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             bulk_copy(dst + row_in, xb + (t0 + 1) * row_in, row_in, bar);
     };
 
-    issue((long long)blockIdx.x * NG + grp, 0);
+    issue(grp, 0);
     if (!mbar_wait(setup_bar, 0))
         atomicOr(&g_k1_err, K1_ERR_COPY_WAIT);
 
-    int round = 0;
-    for (long long base = (long long)blockIdx.x * NG; base < npairs; base += stride, ++round) {
-        const long long pr = base + grp;
-        bool valid = pr < npairs;
+    int my = grp;                                      // this round's pair: lo + my
+    for (int round = 0;; ++round) {
+        if (dyn ? my >= cnt : my - grp >= cnt)
+            break;                                     // uniform across the group / the CTA
+        const long long pr = lo + my;
+        bool valid = my < cnt;
         const long long t0 = 2 * pr, t1 = 2 * pr + 1;
         const int stage = round % nstage;
         const uint32_t parity = (uint32_t)(round / nstage) & 1u;
@@ -347,11 +372,19 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
                                        prmt(a.w, b.w, 0x5410), prmt(a.w, b.w, 0x7632));
                 }
             }
-            __syncthreads();
-            issue(pr + stride, 0);                         // raw is free: fetch next round
+            group_sync();
+            if (dyn) {                                     // raw is free: fetch the next pair
+                if (g == 0) {
+                    const int nx = atomicAdd(&sched[0], 1);
+                    sched[1 + grp] = nx;
+                    issue(nx, 0);
+                }
+            } else {
+                issue(my + step, 0);
+            }
         } else {
             if (nstage > 1)
-                issue(pr + stride, (round + 1) % nstage);  // the other stage is free
+                issue(my + step, (round + 1) % nstage);    // the other stage is free
         }
 
         // ---- gather y[i] = sign[i] * x[perm[i]] for both tokens ------------------------------
@@ -427,15 +460,20 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             }
         }
         if (seg_head)
-            red[grp * kMaxSeg + seg_slot] = acc;
-        __syncthreads();
+            red[((round & 1) * NG + grp) * kMaxSeg + seg_slot] = acc;
+        group_sync();
         if constexpr (IN_F32) {
             if (nstage == 1)
-                issue(pr + stride, 0);                     // gathers are done: refill
+                issue(my + step, 0);                       // gathers are done: refill
         }
-        float2 ss = red[grp * kMaxSeg];
+        // partials alternate between two buffers by round: a round's writes never meet the
+        // previous round's reads, which the barrier of that round separates
+        const float2 *myred = red + ((round & 1) * NG + grp) * kMaxSeg;
+        // the group's next pair (its leader wrote the index before the barrier above)
+        const int nxt = dyn ? sched[1 + grp] : my + step;
+        float2 ss = myred[0];
         for (int i = 1; i < nslots; ++i) {
-            const float2 o = red[grp * kMaxSeg + i];
+            const float2 o = myred[i];
             ss.x += o.x;
             ss.y += o.y;
         }
@@ -506,6 +544,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             if (has1 && g == 0)
                 p.norms[t1] = s1;
         }
+        my = nxt;
     }
 }
 
@@ -551,7 +590,7 @@ cudaError_t k1_prepare(const void *kern, int threads, size_t smem, int *per_sm) 
 
 template <int BITS, bool F32, bool GELU = false, bool A16 = false>
 cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int threads, size_t smem,
-                     int num_sms, cudaStream_t st, std::string *why) {
+                     int num_sms, cudaStream_t st, std::string *why, bool named) {
     auto go = [&](auto kern) -> cudaError_t {
         int per_sm = 0;
         cudaError_t e = k1_prepare((const void *)kern, threads, smem, &per_sm);
@@ -568,22 +607,24 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
             *why = "k1 launch";
         return e;
     };
+    // the named-barrier form exists for bf16 input only (F32 picks the same kernel twice)
+    auto pick = [&](auto kn, auto kl) { return named ? go(kn) : go(kl); };
     if constexpr (A16) {            // the fp16-output variants are built for h <= 256
         switch (h) {
-            case 32: return go(k1_rotquant<BITS, F32, 32, GELU, true>);
-            case 64: return go(k1_rotquant<BITS, F32, 64, GELU, true>);
-            case 128: return go(k1_rotquant<BITS, F32, 128, GELU, true>);
-            case 256: return go(k1_rotquant<BITS, F32, 256, GELU, true>);
+            case 32: return pick(k1_rotquant<BITS, F32, 32, GELU, true, !F32>, k1_rotquant<BITS, F32, 32, GELU, true>);
+            case 64: return pick(k1_rotquant<BITS, F32, 64, GELU, true, !F32>, k1_rotquant<BITS, F32, 64, GELU, true>);
+            case 128: return pick(k1_rotquant<BITS, F32, 128, GELU, true, !F32>, k1_rotquant<BITS, F32, 128, GELU, true>);
+            case 256: return pick(k1_rotquant<BITS, F32, 256, GELU, true, !F32>, k1_rotquant<BITS, F32, 256, GELU, true>);
             default: *why = "unsupported h for fp16 output"; return cudaErrorInvalidValue;
         }
     } else {
         switch (h) {
-            case 32: return go(k1_rotquant<BITS, F32, 32, GELU>);
-            case 64: return go(k1_rotquant<BITS, F32, 64, GELU>);
-            case 128: return go(k1_rotquant<BITS, F32, 128, GELU>);
-            case 256: return go(k1_rotquant<BITS, F32, 256, GELU>);
-            case 512: return go(k1_rotquant<BITS, F32, 512, GELU>);
-            case 1024: return go(k1_rotquant<BITS, F32, 1024, GELU>);
+            case 32: return pick(k1_rotquant<BITS, F32, 32, GELU, false, !F32>, k1_rotquant<BITS, F32, 32, GELU>);
+            case 64: return pick(k1_rotquant<BITS, F32, 64, GELU, false, !F32>, k1_rotquant<BITS, F32, 64, GELU>);
+            case 128: return pick(k1_rotquant<BITS, F32, 128, GELU, false, !F32>, k1_rotquant<BITS, F32, 128, GELU>);
+            case 256: return pick(k1_rotquant<BITS, F32, 256, GELU, false, !F32>, k1_rotquant<BITS, F32, 256, GELU>);
+            case 512: return pick(k1_rotquant<BITS, F32, 512, GELU, false, !F32>, k1_rotquant<BITS, F32, 512, GELU>);
+            case 1024: return pick(k1_rotquant<BITS, F32, 1024, GELU, false, !F32>, k1_rotquant<BITS, F32, 1024, GELU>);
             default: *why = "unsupported h"; return cudaErrorInvalidValue;
         }
     }
@@ -592,8 +633,9 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
 size_t k1_smem(const K1Params &p, int in_f32, int NG, int stages) {
     const size_t row_in = (size_t)p.d * (in_f32 ? 4 : 2);
     size_t b = 4 * (size_t)(p.tbl_words + p.ent_words + p.dec_words);   // tables, entries
-    b += sizeof(float2) * NG * kMaxSeg;                    // norm partials
+    b += sizeof(float2) * 2 * NG * kMaxSeg;                // norm partials, two buffers
     b += 8 * (size_t)(2 * NG + 2);                         // mbarriers
+    b += 4 * 16;                                           // pair scheduling words
     b += (size_t)NG * stages * 2 * row_in;                 // raw rows
     if (!in_f32)
         b += (size_t)NG * p.d * 4;                         // interleaved pairs
@@ -610,13 +652,35 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     int stages = in_f32 ? 2 : 1;
     if (in_f32 && k1_smem(p, in_f32, 1, 2) > 200 * 1024)
         stages = 1;
-    int NG = 256 / GT;
-    if (NG < 1)
-        NG = 1;
-    if (NG > npairs)
-        NG = (int)npairs;
-    while (NG > 1 && k1_smem(p, in_f32, NG, stages) > 72 * 1024)
-        --NG;
+    long long ctas_needed;
+    int NG;
+    const bool named = GT % 32 == 0 && !in_f32;
+    if (named) {
+        // Groups of whole warps: one CTA per SM with as many groups as the register file
+        // holds (96 registers a thread; at most 15 named barriers and 1024 threads), each CTA
+        // an equal share of the pairs.  The group count is the smallest that takes the share
+        // in the same number of rounds, so the rounds stay full.
+        ctas_needed = std::min<long long>(num_sms, npairs);
+        const long long share = (npairs + ctas_needed - 1) / ctas_needed;
+        // registers: each of the SM's four 16K-register partitions holds 5 warps of 96
+        constexpr int kWarpsPerSm = 4 * ((65536 / 4) / (96 * 32));
+        int ng_max = std::min(std::min(15, 1024 / GT), kWarpsPerSm * 32 / GT);
+        while (ng_max > 1 && k1_smem(p, in_f32, ng_max, stages) > 220 * 1024)
+            --ng_max;
+        ng_max = (int)std::max(1LL, std::min<long long>(ng_max, share));
+        const long long rounds = (share + ng_max - 1) / ng_max;
+        NG = (int)((share + rounds - 1) / rounds);
+    } else {
+        // Groups that share warps run in lockstep: several smaller CTAs per SM.
+        NG = 256 / GT;
+        if (NG < 1)
+            NG = 1;
+        if (NG > npairs)
+            NG = (int)npairs;
+        while (NG > 1 && k1_smem(p, in_f32, NG, stages) > 72 * 1024)
+            --NG;
+        ctas_needed = (npairs + NG - 1) / NG;
+    }
     const size_t smem = k1_smem(p, in_f32, NG, stages);
     if (smem > 227 * 1024) {
         *why = "k1 shared memory exceeds the per-CTA limit";
@@ -625,7 +689,6 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     p.groups = NG;
     p.stages = stages;
     const int threads = NG * GT;
-    const long long ctas_needed = (npairs + NG - 1) / NG;
     if (p.a16) {
         if (in_f32) {
             *why = "fp16 centroid output takes bf16 input";
@@ -634,9 +697,9 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
         auto go16 = [&](auto gelu_tag) -> cudaError_t {
             constexpr bool GL = decltype(gelu_tag)::value;
             switch (bits) {
-                case 2: return launch_h<2, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-                case 4: return launch_h<4, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-                case 8: return launch_h<8, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+                case 2: return launch_h<2, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+                case 4: return launch_h<4, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+                case 8: return launch_h<8, false, GL, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
                 default: *why = "fp16 centroid output: bit width"; return cudaErrorInvalidValue;
             }
         };
@@ -648,25 +711,25 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
             return cudaErrorInvalidValue;
         }
         switch (bits) {
-            case 2: return launch_h<2, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-            case 3: return launch_h<3, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-            case 4: return launch_h<4, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-            case 6: return launch_h<6, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-            case 8: return launch_h<8, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+            case 2: return launch_h<2, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+            case 3: return launch_h<3, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+            case 4: return launch_h<4, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+            case 6: return launch_h<6, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+            case 8: return launch_h<8, false, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
             default: *why = "unsupported bit width"; return cudaErrorInvalidValue;
         }
     }
     switch (bits * 2 + (in_f32 ? 1 : 0)) {
-        case 4: return launch_h<2, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 5: return launch_h<2, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 6: return launch_h<3, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 7: return launch_h<3, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 8: return launch_h<4, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 9: return launch_h<4, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 12: return launch_h<6, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 13: return launch_h<6, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 16: return launch_h<8, false>(p, h, ctas_needed, threads, smem, num_sms, st, why);
-        case 17: return launch_h<8, true>(p, h, ctas_needed, threads, smem, num_sms, st, why);
+        case 4: return launch_h<2, false>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 5: return launch_h<2, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 6: return launch_h<3, false>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 7: return launch_h<3, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 8: return launch_h<4, false>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 9: return launch_h<4, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 12: return launch_h<6, false>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 13: return launch_h<6, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 16: return launch_h<8, false>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
+        case 17: return launch_h<8, true>(p, h, ctas_needed, threads, smem, num_sms, st, why, named);
         default: *why = "unsupported bit width"; return cudaErrorInvalidValue;
     }
 }
