@@ -18,6 +18,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "decode4.cuh"
@@ -353,6 +354,233 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
 }
 
 // ------------------------------------------------------------------------------------------
+// CTA-pair GEMM (cluster of two CTAs on neighbouring SMs, tcgen05 .cta_group::2).  A pair
+// computes a 256 x 256 output tile: per k-block each CTA loads its own 128 rows of A and its
+// own 128 rows of B (outputs n0 + 128 * rank ...), and the leader CTA (rank 0) issues
+// M = 256, N = 256 MMAs that read both CTAs' tiles, each CTA's tensor memory receiving its 128
+// rows of the tile.  Per SM a k-block then brings in 32 KB instead of 48 KB for the same MMA
+// time, and the ring holds 6 stages.  Barriers: the leader's full barrier counts both CTAs'
+// TMA bytes (only the leader arms it); the leader's MMA commits release both CTAs' stages and
+// signal both CTAs' accumulator-full barriers (multicast commit); every epilogue warp of both
+// CTAs arrives on the leader's accumulator-empty barrier.  TMA loads carry no multicast.
+// ------------------------------------------------------------------------------------------
+constexpr int P_STAGES = 6;
+constexpr int P_BM = 256, P_BN = 256;                    // pair tile
+constexpr int P_A_BYTES = 128 * BK * 2;                  // 16 KB: this CTA's 128 rows of A
+constexpr int P_B_BYTES = 128 * BK * 2;                  // 16 KB: this CTA's 128 rows of B
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr int kPairNumBars = 2 * P_STAGES + 5;
+constexpr int kPairThreads = 32 * (2 + kEpiWarps);
+constexpr uint32_t kIdescPair = idesc_f16(P_BM, P_BN);
+
+__host__ __device__ constexpr size_t gemm_pair_smem() {
+    return 1024 + (size_t)P_STAGES * P_STAGE_BYTES + (size_t)kEpiWarps * 2 * kStageOut +
+           8 * kPairNumBars + 8 + kEpiWarps * 64 * sizeof(float) + 64;
+}
+static_assert(gemm_pair_smem() <= 227 * 1024, "shared memory budget (pair)");
+
+// Warp roles as in k2_gemm: warp 0 lane 0 loads (both CTAs), warp 1 owns tensor memory (both
+// CTAs allocate the same columns) and its lane 0 issues the MMAs (leader only), warps 2..5
+// are the epilogue (both CTAs, each its own 128 rows).  Pair p takes tiles p, p + #pairs, ...
+template <bool BF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    k2_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;                 // same offsets in both CTAs
+    unsigned char *basep = smem_raw + (base - raw);
+    const uint32_t sA = base, sB = base + P_STAGES * P_A_BYTES;
+    const uint32_t sOut = sB + P_STAGES * P_B_BYTES;              // [4 warps][2][4 KB]
+    const uint32_t bars = sOut + kEpiWarps * 2 * kStageOut;
+    auto full_bar = [&](int s) { return bars + 8u * s; };                   // leader's is used
+    auto empty_bar = [&](int s) { return bars + 8u * (P_STAGES + s); };
+    auto tfull_bar = [&](int a) { return bars + 8u * (2 * P_STAGES + a); };
+    auto tempty_bar = [&](int a) { return bars + 8u * (2 * P_STAGES + 2 + a); };   // leader's
+    const uint32_t drain_bar = bars + 8u * (2 * P_STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain_bar + 8u - base));
+    float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][64]
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();                      // 0: the leader
+    const int pair0 = (int)cluster_id_x(), npair = (int)cluster_count_x();
+    const int n_tiles = (p.N + P_BN - 1) / P_BN;
+    const int num_tiles = ((p.M + P_BM - 1) / P_BM) * n_tiles;
+    const int num_kb = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 2 * kEpiWarps);
+        }
+        mbar_init(drain_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        abort_flag = 0;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync_all();                 // both CTAs' barriers initialised, tensor memory held
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
+    auto give_up = [&](unsigned bit) {
+        atomicOr(&g_k2_err, bit);
+        atomicExch(&abort_flag, 1);
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int tile = pair0; tile < num_tiles && !aborted(); tile += npair) {
+                const int m0 = (tile / n_tiles) * P_BM + (int)rank * 128;
+                const int n0 = (tile % n_tiles) * P_BN + (int)rank * 128;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % P_STAGES;
+                    if (it >= P_STAGES &&
+                        !mbar_wait(empty_bar(s), ((it / P_STAGES) & 1) ^ 1)) {
+                        give_up(ERR_WAIT_EMPTY);
+                        break;
+                    }
+                    if (aborted())
+                        break;
+                    if (rank == 0)
+                        mbar_expect_tx(full_bar(s), 2 * P_STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(full_bar(s), 0);
+                    tma_load_2d_pair(sA + s * P_A_BYTES, &tmA, kb * BK, m0, fb);
+                    tma_load_2d_pair(sB + s * P_B_BYTES, &tmB, kb * BK, n0, fb);
+                }
+            }
+            if (aborted() && rank == 0) {
+                // let the loads already issued land before the pair can exit
+                const uint32_t from = it > (uint32_t)P_STAGES ? it - P_STAGES : 0;
+                for (uint32_t j = from; j < it; ++j)
+                    mbar_wait(full_bar(j % P_STAGES), (j / P_STAGES) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (leader) ----------------
+        if (lane == 0 && rank == 0) {
+            uint32_t it = 0;
+            int i = 0;
+            for (int tile = pair0; tile < num_tiles && !aborted(); tile += npair, ++i) {
+                const int acc = i & 1;
+                if (i >= 2 && !mbar_wait(tempty_bar(acc), ((i >> 1) & 1) ^ 1)) {
+                    give_up(ERR_WAIT_EMPTY);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * kAccCols);
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                    const int s = it % P_STAGES;
+                    if (!mbar_wait(full_bar(s), (it / P_STAGES) & 1)) {
+                        give_up(ERR_WAIT_FULL);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t da = sw128_desc(sA + s * P_A_BYTES);
+                    const uint64_t db = sw128_desc(sB + s * P_B_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        mma_ss_pair(d_tmem, da + 2 * kk, db + 2 * kk, kIdescPair, (kb | kk) != 0);
+                    mma_commit_pair_mc(empty_bar(s), 0x3);
+                }
+                if (!ok)
+                    break;
+                mma_commit_pair_mc(tfull_bar(acc), 0x3);
+            }
+            mma_commit_pair_mc(drain_bar, 0x1);
+            if (!mbar_wait(drain_bar, 0))
+                atomicOr(&g_k2_err, ERR_WAIT_ACCUM);
+        }
+    } else {
+        // ---------------- epilogue (both CTAs): this CTA's 128 rows of the tile ----------
+        const int q = warp & 3;                               // TMEM lane quarter
+        float *rn_w = rn_s + (warp - 2) * 64;
+        const uint32_t out0 = sOut + (uint32_t)((warp - 2) * 2 * kStageOut);
+        unsigned char *out0p = basep + (out0 - base);
+        uint32_t u = 0;
+        int i = 0;
+        for (int tile = pair0; tile < num_tiles; tile += npair, ++i) {
+            const int acc = i & 1;
+            const int m0 = (tile / n_tiles) * P_BM + (int)rank * 128;
+            const int n0 = (tile % n_tiles) * P_BN;
+            const int row = m0 + q * 32 + lane;
+            const float srow = (row < p.M) ? p.s[row] * p.inv_d : 0.f;
+            float rnv[P_BN / 32];
+#pragma unroll
+            for (int c = 0; c < P_BN / 32; ++c) {
+                const int col = n0 + c * 32 + lane;
+                rnv[c] = (col < p.N) ? p.rn[col] : 0.f;
+            }
+            const bool ok = mbar_wait(tfull_bar(acc), (i >> 1) & 1);
+            if (!__all_sync(0xffffffffu, ok && !aborted())) {
+                if (!ok)
+                    give_up(ERR_WAIT_ACCUM);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t t_base =
+                tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * kAccCols);
+            const bool rows_in = m0 + q * 32 < p.M;
+            constexpr int kCW = BF16 ? 64 : 32;
+#pragma unroll
+            for (int c = 0; c < P_BN / kCW; ++c) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(t_base + (uint32_t)(c * kCW), r0);
+                if constexpr (BF16)
+                    tmem_ld32(t_base + (uint32_t)(c * kCW + 32), r1);
+                if (!rows_in || n0 + c * kCW >= p.N)
+                    continue;
+                const uint32_t b = u & 1;
+                if (lane == 0)
+                    bulk_wait_read<1>();
+                __syncwarp();
+                if constexpr (BF16) {
+                    rn_w[lane] = rnv[2 * c];
+                    rn_w[32 + lane] = rnv[2 * c + 1];
+                } else {
+                    rn_w[lane] = rnv[c];
+                }
+                __syncwarp();
+                if constexpr (BF16)
+                    store_chunk_bf16(&tmY, out0p + b * kStageOut, out0 + b * kStageOut, r0, r1,
+                                     srow, rn_w, lane, n0 + c * kCW, m0 + q * 32);
+                else
+                    store_chunk(&tmY, out0p + b * kStageOut, out0 + b * kStageOut, r0, srow,
+                                rn_w, lane, n0 + c * kCW, m0 + q * 32);
+                ++u;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+        }
+        if (lane == 0)
+            bulk_wait_all();
+    }
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();                 // no MMA, load or arrive of the pair is still pending
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                     ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 // Host side.
 // ------------------------------------------------------------------------------------------
 // fp16 [rows, K] row-major -> tiles of box_rows x 64 with 128-byte swizzle.
@@ -458,6 +686,61 @@ cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const CU
     return e;
 }
 
+// Pairs of the CTA-pair GEMM that fit on the device at once (0: the form is unavailable),
+// once per device and instantiation.
+template <bool BF16>
+int gemm_pair_slots() {
+    static std::mutex mu;
+    static int slots[kMaxDevices];
+    static bool done[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done[dev]) {
+        done[dev] = true;
+        slots[dev] = 0;
+        auto kern = k2_gemm_pair<BF16>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gemm_pair_smem()) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2, 1, 1);
+        cfg.blockDim = dim3(kPairThreads, 1, 1);
+        cfg.dynamicSmemBytes = gemm_pair_smem();
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        slots[dev] = n;
+    }
+    return slots[dev];
+}
+
+template <bool BF16>
+cudaError_t launch_gemm_pair_t(const CUtensorMap &ma, const CUtensorMap &mb,
+                               const CUtensorMap &my, const GemmParams &gp, int pairs,
+                               cudaStream_t st, std::string *why) {
+    k2_gemm_pair<BF16><<<2 * pairs, kPairThreads, gemm_pair_smem(), st>>>(ma, mb, my, gp);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        *why = "k2_gemm_pair launch";
+    return e;
+}
+
+// The CTA-pair GEMM is used when the device can hold it; OQ_GEMM_PAIR=0 selects the
+// single-CTA kernel (read once per process).
+bool gemm_pair_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("OQ_GEMM_PAIR");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
@@ -479,6 +762,20 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
         return cudaErrorInvalidValue;
     }
     CUtensorMap ma, mb, my;
+    if (!acodes && gemm_pair_enabled()) {
+        const int slots = y_bf16 ? gemm_pair_slots<true>() : gemm_pair_slots<false>();
+        if (slots > 0) {
+            if (!make_map(&ma, A16, T, d, 128) || !make_map(&mb, B16, N, d, 128) ||
+                !make_out_map(&my, y, T, N, y_bf16)) {
+                *why = "cuTensorMapEncodeTiled failed";
+                return cudaErrorInvalidValue;
+            }
+            const int tiles = ((N + P_BN - 1) / P_BN) * ((T + P_BM - 1) / P_BM);
+            const int pairs = tiles < slots ? tiles : slots;
+            return y_bf16 ? launch_gemm_pair_t<true>(ma, mb, my, gp, pairs, st, why)
+                          : launch_gemm_pair_t<false>(ma, mb, my, gp, pairs, st, why);
+        }
+    }
     const bool a_ok = acodes ? make_code_map(&ma, x_codes4, T, d) : make_map(&ma, A16, T, d, BM);
     if (!a_ok || !make_map(&mb, B16, N, d, BN) || !make_out_map(&my, y, T, N, y_bf16)) {
         *why = "cuTensorMapEncodeTiled failed";

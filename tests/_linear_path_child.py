@@ -1,5 +1,6 @@
-"""Child process for the oq_linear path test: OQ_LINEAR_PATH is read once per process, so each
-path for 4-bit activation codes (in-GEMM decode, prepass) is exercised in a process of its own.  Checks oq_linear on uniform
+"""Child process for the oq_linear path test: OQ_LINEAR_PATH and OQ_GEMM_PAIR are read once per
+process, so each GEMM form (in-GEMM decode of 4-bit activation codes; fp16 prepass into the
+CTA-pair or the single-CTA GEMM) is exercised in a process of its own.  Checks oq_linear on uniform
 random codes (every centroid used, ragged M and N tails) against the fp64 oracle, and the bf16
 output against the fp32 output rounded to nearest even; exits non-zero on any failure."""
 import os
@@ -20,7 +21,8 @@ LINEAR_RTOL = 1e-3
 def main():
     worst = 0.0
     for ba, bw in [(4, 4), (4, 2), (4, 3), (4, 8)]:
-        for T, N, d in [(200, 272, 384), (1, 16, 128), (129, 512, 1024), (300, 784, 3072)]:
+        for T, N, d in [(200, 272, 384), (1, 16, 128), (129, 512, 1024), (300, 784, 3072),
+                        (520, 528, 256)]:
             rng = np.random.default_rng(T * 7 + N + ba * 100 + bw + 5)
             xc = O.pack(rng.integers(0, 1 << ba, (T, d)).astype(np.uint8), ba)
             wc = O.pack(rng.integers(0, 1 << bw, (N, d)).astype(np.uint8), bw)

@@ -334,18 +334,22 @@ def test_linear_video_ffn_up_full_size(oq, variant):
     _sampled_linear(oq, p, rows, cols)
 
 
-@pytest.mark.parametrize("path", ["fused", "default"])
+@pytest.mark.parametrize("path", ["fused", "default", "single"])
 def test_linear_path_selection(oq, path):
-    """Both oq_linear paths for 4-bit activation codes (the fp16 prepass by default; decoded
-    inside the GEMM with OQ_LINEAR_PATH=fused) against the oracle; each runs in a child
-    process because the variable is read once per process."""
+    """Every oq_linear GEMM form against the oracle: the fp16 prepass feeding the CTA-pair
+    GEMM (default), the same prepass feeding the single-CTA GEMM (OQ_GEMM_PAIR=0), and 4-bit
+    activation codes decoded inside the GEMM (OQ_LINEAR_PATH=fused); each runs in a child
+    process because the variables are read once per process."""
     import os
     import subprocess
     import sys
     env = dict(os.environ)
     env.pop("OQ_LINEAR_PATH", None)
+    env.pop("OQ_GEMM_PAIR", None)
     if path == "fused":
         env["OQ_LINEAR_PATH"] = "fused"
+    if path == "single":
+        env["OQ_GEMM_PAIR"] = "0"
     child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_linear_path_child.py")
     r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
                        timeout=600)
