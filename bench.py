@@ -456,7 +456,8 @@ def run_ours(args, p, rank, world, dev):
                 else "oq_quantize_act + oq_linear"),
         "kernels_ms_mean": {"quantize": quant_ms, "decode": dec_ms, "gemm": gemm_ms},
         "roofline": {
-            "kernel": "k2_gemm (tcgen05 kind::f16, 128x256x64 tiles)",
+            "kernel": ("k2_gemm_pair (tcgen05 cta_group::2 kind::f16, 256x256x64 tiles per "
+                       "CTA pair)"),
             "bound": "tensor", "achieved": gemm_tf,
             "peak": pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
             "peak_note": f"{pk_kind} dense bf16 burst (fp16 kind::f16 runs at the bf16 rate)",
