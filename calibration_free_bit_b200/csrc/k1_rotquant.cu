@@ -277,6 +277,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     unsigned char *mypairs = pairs + (size_t)grp * d * 4;
     const uint32_t setup_bar = smem_u32(&bars[2 * NG]);
 
+    pdl_trigger();
     if (tid == 0) {
         for (int b = 0; b < 2 * NG + 1; ++b)
             mbar_init(smem_u32(&bars[b]), 1);
@@ -334,6 +335,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             bulk_copy(dst + row_in, xb + (t0 + 1) * row_in, row_in, bar);
     };
 
+    pdl_wait();                                        // x, codes, norms: earlier work done
     issue(grp, 0);
     if (!mbar_wait(setup_bar, 0))
         atomicOr(&g_k1_err, K1_ERR_COPY_WAIT);
@@ -601,8 +603,7 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
         long long grid = (long long)num_sms * per_sm;
         if (grid > ctas_needed)
             grid = ctas_needed;
-        kern<<<(unsigned)grid, threads, smem, st>>>(p);
-        e = cudaGetLastError();
+        e = launch_pdl(kern, dim3((unsigned)grid), dim3(threads), smem, st, p);
         if (e != cudaSuccess)
             *why = "k1 launch";
         return e;

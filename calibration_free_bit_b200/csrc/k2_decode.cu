@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(kDecThreads) k2_decode(const __grid_constant__
     constexpr int ENTRIES = 1 << IDX_BITS;
     static_assert(!SYM || BITS == 4, "byte-permute decode is 4-bit only");
     __shared__ __align__(16) uint16_t tab[SYM ? 8 : (ENTRIES * PER < 512 ? 512 : ENTRIES * PER)];
+    pdl_trigger();
     if constexpr (!SYM) {
         for (int e = threadIdx.x; e < ENTRIES; e += blockDim.x)
 #pragma unroll
@@ -95,6 +96,7 @@ __global__ void __launch_bounds__(kDecThreads) k2_decode(const __grid_constant__
                 tab[e * PER + i] = p.lut[(e >> (i * BITS)) & ((1 << BITS) - 1)];
         __syncthreads();
     }
+    pdl_wait();                                        // codes, out: earlier work done
     const uint32_t *tab32 = reinterpret_cast<const uint32_t *>(tab);
     const long long stride = (long long)gridDim.x * blockDim.x;
     uint4 *out = reinterpret_cast<uint4 *>(p.out);
@@ -130,8 +132,7 @@ cudaError_t decode(const DecodeParams &dp, cudaStream_t st, int num_sms) {
         blocks = cap;
     if (blocks < 1)
         blocks = 1;
-    k2_decode<BITS, SYM><<<(unsigned)blocks, kDecThreads, 0, st>>>(dp);
-    return cudaGetLastError();
+    return launch_pdl(k2_decode<BITS, SYM>, dim3((unsigned)blocks), dim3(kDecThreads), 0, st, dp);
 }
 
 }  // namespace

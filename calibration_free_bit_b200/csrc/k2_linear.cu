@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
     const int num_tiles = ((p.M + BM - 1) / BM) * n_tiles;
     const int num_kb = p.K / BK;
 
+    pdl_trigger();
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), 1);
@@ -152,6 +153,7 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();                         // operands, s, rn and y: earlier work of the stream done
     auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
     auto give_up = [&](unsigned bit) {
         atomicOr(&g_k2_err, bit);
@@ -409,6 +411,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int num_tiles = ((p.M + P_BM - 1) / P_BM) * n_tiles;
     const int num_kb = p.K / BK;
 
+    pdl_trigger();
     if (threadIdx.x == 0) {
         for (int s = 0; s < P_STAGES; ++s) {
             mbar_init(full_bar(s), 1);
@@ -431,6 +434,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     cluster_sync_all();                 // both CTAs' barriers initialised, tensor memory held
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();                         // operands, s, rn and y: earlier work of the stream done
     auto aborted = [&]() { return *(volatile int *)&abort_flag != 0; };
     auto give_up = [&](unsigned bit) {
         atomicOr(&g_k2_err, bit);
@@ -679,8 +683,8 @@ cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const CU
         *why = "cudaFuncSetAttribute(k2_gemm)";
         return e;
     }
-    kern<<<grid, gemm_threads<ACODES>(), gemm_smem<ACODES>(), st>>>(ma, mb, my, gp);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3(grid), dim3(gemm_threads<ACODES>()), gemm_smem<ACODES>(), st, ma, mb,
+                   my, gp);
     if (e != cudaSuccess)
         *why = "k2_gemm launch";
     return e;
@@ -724,8 +728,8 @@ template <bool BF16>
 cudaError_t launch_gemm_pair_t(const CUtensorMap &ma, const CUtensorMap &mb,
                                const CUtensorMap &my, const GemmParams &gp, int pairs,
                                cudaStream_t st, std::string *why) {
-    k2_gemm_pair<BF16><<<2 * pairs, kPairThreads, gemm_pair_smem(), st>>>(ma, mb, my, gp);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(k2_gemm_pair<BF16>, dim3(2 * pairs), dim3(kPairThreads),
+                                     gemm_pair_smem(), st, ma, mb, my, gp);
     if (e != cudaSuccess)
         *why = "k2_gemm_pair launch";
     return e;

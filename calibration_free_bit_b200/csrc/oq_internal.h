@@ -15,6 +15,37 @@ namespace oq {
 
 constexpr int kMaxDevices = 32;
 
+// Programmatic dependent launch.  liboq launches every kernel of the hot path so that it may
+// start while the previous kernel of its stream is finishing: the kernel signals at once that
+// its own successor may start (pdl_trigger), does its set-up from data no earlier work writes
+// (barriers, tensor memory, its host-built tables), and waits for all earlier work of the
+// stream before it reads or writes anything else (pdl_wait; a no-op for a launch without a
+// programmatic dependency).
+#if defined(__CUDACC__)
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+#endif
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // Shared-memory images of K1, built on the host (oq_host.cpp) and bulk-copied per CTA.
 //   Gather entries: d/32 rows of kK1EntStride words; row g holds, for positions g*32+e,
 //   (byte offset of x[perm[pos]] in the staged row data) | (sign[pos] < 0) << 31.  For fp32
