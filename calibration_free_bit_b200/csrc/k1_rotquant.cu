@@ -12,8 +12,9 @@
 //     (cp.async.bulk, mbarrier completion, no multicast) one round ahead of the compute.
 //   * bf16 rows are interleaved into 32-bit words (x_t0[j], x_t1[j]), so one 4-byte gather
 //     load serves both tokens and the butterfly runs on packed fp32x2 (add/sub/fma .f32x2,
-//     new on sm_100).  The low and high halves of each 8-element chunk go to separate
-//     regions, so the interleave stores of consecutive threads are contiguous.
+//     new on sm_100).  Each half of an 8-element chunk goes to a 16-byte slot the host
+//     chose: the eight stores of a quarter-warp cover all banks, and the slots' bank groups
+//     are arranged so that the 32 lanes of a random gather meet on fewer banks.
 //   * Thread g holds the 32 consecutive rotated positions g*32 .. g*32+31 (h/32 threads per
 //     h-block).  Its gather offsets and signs (pair-buffer byte offset of perm[i] | sign<<31)
 //     are converted once per CTA into a shared table, padded to 36 words per thread so the
@@ -362,16 +363,21 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             if (valid) {
                 const uint4 *r0 = reinterpret_cast<const uint4 *>(cur);
                 const uint4 *r1 = reinterpret_cast<const uint4 *>(cur + row_in);
-                uint4 *lo = reinterpret_cast<uint4 *>(mypairs);
-                uint4 *hi = reinterpret_cast<uint4 *>(mypairs + 2 * d);
+                uint4 *slots = reinterpret_cast<uint4 *>(mypairs);
+                // the 16-byte slots of this thread's eight half-chunks (host-chosen so that
+                // the random gather below spreads over the banks)
+                const uint4 sl = myent[kE / 4];
+                const uint32_t slw[4] = {sl.x, sl.y, sl.z, sl.w};
 #pragma unroll
                 for (int k = 0; k < kE / 8; ++k) {
                     const int c = g + k * GT;              // elements 8c..8c+7
                     const uint4 a = r0[c], b = r1[c];
-                    lo[c] = make_uint4(prmt(a.x, b.x, 0x5410), prmt(a.x, b.x, 0x7632),
-                                       prmt(a.y, b.y, 0x5410), prmt(a.y, b.y, 0x7632));
-                    hi[c] = make_uint4(prmt(a.z, b.z, 0x5410), prmt(a.z, b.z, 0x7632),
-                                       prmt(a.w, b.w, 0x5410), prmt(a.w, b.w, 0x7632));
+                    slots[slw[k] & 0xffffu] =
+                        make_uint4(prmt(a.x, b.x, 0x5410), prmt(a.x, b.x, 0x7632),
+                                   prmt(a.y, b.y, 0x5410), prmt(a.y, b.y, 0x7632));
+                    slots[slw[k] >> 16] =
+                        make_uint4(prmt(a.z, b.z, 0x5410), prmt(a.z, b.z, 0x7632),
+                                   prmt(a.w, b.w, 0x5410), prmt(a.w, b.w, 0x7632));
                 }
             }
             group_sync();

@@ -5,6 +5,8 @@
 // flips, block Walsh-Hadamard) and lloyd_max(f_d, b) (change-of-basis paragraph: the standard
 // Lloyd-Max quantizer for the fixed marginal, read as N(0, 1/d)).  The generator and draw
 // order are the ones documented in include/oq.h.
+#include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -639,6 +641,86 @@ extern "C" {
 namespace {
 
 // RPBH tables (permute = true) or Block-RHT tables (the same draws, identity permutation).
+// Pair-buffer slot colours for the bf16 K1 (layout in oq_internal.h).  The staged token pair
+// lives in 16-byte slots of 4 positions; thread g's interleave writes the two halves of chunks
+// c = g + k*GT (k = 0..3, GT = d/32) to slot (2k + lh)*GT + (g & ~7) + colour, where the colours
+// of each octet of threads are a permutation of 0..7 (so every quarter-warp store covers all
+// banks).  The gather of rotated position i reads slot word (j & 3) of j = perm[i] with the
+// 32 lanes of a warp at the same step e reading positions perm[32g + e]; its bank is
+// 4 * colour + (j & 3).  A local search over colour swaps inside each octet lowers the sum
+// over (warp, step) of the largest number of lanes on one bank (for a random permutation
+// from about 3.6 to about 2.1 per load; for the identity, from 16 to 4).  Groups whose
+// threads do not fill whole warps keep colour = g & 7.
+std::vector<uint8_t> pair_slot_colours(const std::vector<int32_t> &perm, int d) {
+    const int GT = d / 32, NH = d / 4;
+    std::vector<uint8_t> col(NH);
+    for (int h = 0; h < NH; ++h) {
+        const int c = h >> 1, g = c % GT;
+        col[h] = (uint8_t)(((g & ~7) + 8 <= GT) ? ((g + (c / GT) * 3) & 7) : (g & 7));
+    }
+    if (GT % 32 != 0)
+        return col;
+    // reads of each half-chunk: (event = warp * 32 + step, j & 3)
+    std::vector<std::array<std::pair<int, int>, 4>> reads(NH);
+    std::vector<int> nread(NH, 0);
+    for (int i = 0; i < d; ++i) {
+        const int j = perm[i], g = i >> 5, e = i & 31;
+        reads[j >> 2][nread[j >> 2]++] = {(g >> 5) * 32 + e, j & 3};
+    }
+    const int NE = (GT / 32) * 32;
+    std::vector<int> cnt((size_t)NE * 32, 0);
+    for (int h = 0; h < NH; ++h)
+        for (int t = 0; t < 4; ++t)
+            ++cnt[(size_t)reads[h][t].first * 32 + 4 * col[h] + reads[h][t].second];
+    auto evmax = [&](int ev) {
+        int m = 0;
+        for (int b = 0; b < 32; ++b)
+            m = std::max(m, cnt[(size_t)ev * 32 + b]);
+        return m;
+    };
+    auto move = [&](int h, int from, int to) {
+        for (int t = 0; t < 4; ++t) {
+            const size_t base = (size_t)reads[h][t].first * 32 + reads[h][t].second;
+            --cnt[base + 4 * from];
+            ++cnt[base + 4 * to];
+        }
+    };
+    SplitMix64 rng{0x5eedULL + (uint64_t)d};
+    const long long iters = std::min(60LL * NH, 200000LL);
+    int evs[8];
+    for (long long it = 0; it < iters; ++it) {
+        // a random octet (g0, k, lh) and two of its members
+        const int oct = (int)rng.below((uint64_t)(GT / 8) * 8);
+        const int g0 = (oct >> 3) * 8, k = (oct >> 1) & 3, lh = oct & 1;
+        const int a = (int)rng.below(8), b = (int)rng.below(7);
+        const int ha = 2 * (g0 + a + k * GT) + lh;
+        const int hb = 2 * (g0 + (b >= a ? b + 1 : b) + k * GT) + lh;
+        int ne = 0;
+        for (int t = 0; t < 4; ++t) {
+            evs[ne++] = reads[ha][t].first;
+            evs[ne++] = reads[hb][t].first;
+        }
+        std::sort(evs, evs + ne);
+        ne = (int)(std::unique(evs, evs + ne) - evs);
+        int before = 0, after = 0;
+        for (int q = 0; q < ne; ++q)
+            before += evmax(evs[q]);
+        const int ca = col[ha], cb = col[hb];
+        move(ha, ca, cb);
+        move(hb, cb, ca);
+        for (int q = 0; q < ne; ++q)
+            after += evmax(evs[q]);
+        if (after <= before) {
+            col[ha] = (uint8_t)cb;
+            col[hb] = (uint8_t)ca;
+        } else {
+            move(ha, cb, ca);
+            move(hb, ca, cb);
+        }
+    }
+    return col;
+}
+
 int build_rotation(int d, int h, uint64_t seed, bool permute, oq_rpbh **out, const char *who) {
     if (!out)
         return fail(OQ_EINVAL, "%s: out is NULL", who);
@@ -672,15 +754,33 @@ int build_rotation(int d, int h, uint64_t seed, bool permute, oq_rpbh **out, con
     for (int i = 0; i < d; ++i)
         r->ent16[i] = (uint16_t)(r->perm[i] | (r->sign[i] < 0 ? 0x8000 : 0));
     // K1 gather-entry images (layout documented in oq_internal.h)
+    const std::vector<uint8_t> colour = pair_slot_colours(r->perm, d);
+    auto slot_of = [&](int g, int k, int lh) {               // 16-byte slot of a half-chunk
+        const int GT = d / 32;
+        return (2 * k + lh) * GT + (g & ~7) + colour[(size_t)2 * (g + k * GT) + lh];
+    };
     for (int f = 0; f < 2; ++f) {
         r->ent_img[f].assign((size_t)(d / 32) * oq::kK1EntStride, 0u);
         for (int i = 0; i < d; ++i) {
             const uint32_t j = (uint32_t)r->perm[i];
-            const uint32_t word = (j & 4u) ? (uint32_t)d / 2 + (j >> 3) * 4 + (j & 3u)
-                                           : (j >> 3) * 4 + (j & 3u);
+            const int c = (int)(j >> 3), GT = d / 32;
+            const uint32_t word = 4u * (uint32_t)slot_of(c % GT, c / GT, (int)(j >> 2) & 1) +
+                                  (j & 3u);
             const uint32_t off = (f == 1) ? 4u * j : 4u * word;
             r->ent_img[f][(size_t)(i >> 5) * oq::kK1EntStride + (i & 31)] =
                 off | (r->sign[i] < 0 ? 0x80000000u : 0u);
+        }
+        if (f == 0) {
+            // words 32..35 of row g: the 16-byte slots its interleave stores go to, as 16-bit
+            // indices (k, lh) -> halfword 2k + lh
+            for (int g = 0; g < d / 32; ++g)
+                for (int k = 0; k < 4; ++k)
+                    for (int lh = 0; lh < 2; ++lh) {
+                        const uint32_t slot = (uint32_t)slot_of(g, k, lh);
+                        const int hw = 2 * k + lh;
+                        r->ent_img[0][(size_t)g * oq::kK1EntStride + 32 + hw / 2] |=
+                            slot << (16 * (hw & 1));
+                    }
         }
     }
     *out = r;

@@ -49,9 +49,13 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // Shared-memory images of K1, built on the host (oq_host.cpp) and bulk-copied per CTA.
 //   Gather entries: d/32 rows of kK1EntStride words; row g holds, for positions g*32+e,
 //   (byte offset of x[perm[pos]] in the staged row data) | (sign[pos] < 0) << 31.  For fp32
-//   input the offset is 4*perm[pos]; for bf16 input it is 4*pair_word(perm[pos]) with
-//   pair_word(j) = (j & 4) ? d/2 + (j>>3)*4 + (j&3) : (j>>3)*4 + (j&3) (the kernel's interleave
-//   writes the low/high halves of each 8-element chunk into separate regions).
+//   input the offset is 4*perm[pos].  For bf16 input the staged pair lives in 16-byte slots
+//   of four 32-bit words (x_t0[j], x_t1[j]): element j is word j & 3 of the slot of half-chunk
+//   (c = j >> 3, lh = (j >> 2) & 1), slot(g, k, lh) = (2k + lh)*GT + (g & ~7) + colour with
+//   GT = d/32, c = g + k*GT, and the colours of each octet of threads a permutation of 0..7
+//   chosen on the host (oq_host.cpp, pair_slot_colours); the offset is 16*slot + 4*(j & 3).
+//   Words 32..35 of row g (bf16 image) hold the slots of that thread's interleave stores as
+//   16-bit values, half-word 2k + lh.
 //   Quantizer table: G+1 words, each repeated 32 times (one copy per lane, k*32 + lane) when
 //   bits <= 4, else stored once; padded to a multiple of 4 words.
 constexpr int kK1EntStride = 36;
