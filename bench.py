@@ -329,6 +329,8 @@ def run_ours(args, p, rank, world, dev):
     per_kernel = {}
     for name, t in oq.oq_timing_collect():
         per_kernel.setdefault(name, []).append(t)
+    # liboq kernel launches per step, counted from the timing records of the n_k eager steps
+    launches_per_step = round(sum(len(v) for v in per_kernel.values()) / n_k)
 
     # (3) headline region: the step captured once per buffer set in a CUDA graph and replayed,
     #     so host launch cost does not pace the device
@@ -363,11 +365,11 @@ def run_ours(args, p, rank, world, dev):
     clock_info = clocks.stop() if clocks else None
     oq.oq_check()
     ms_max = max_over_ranks(g0.elapsed_time(g1), world, dev)
-    # kernels per step: quantize, decode W, GEMM (+ decode x unless the quantizer writes the
-    # fp16 operand itself: forward path with 2/4/8-bit activations, bf16 x, h <= 256)
+    # the quantizer writes the fp16 operand itself on the forward path with 2/4/8-bit
+    # activations, bf16 x and h <= 256 (and, for 4-bit weights, decodes the weights too)
     direct = (args.api == "forward" and p.bits_a in (2, 4, 8) and p.dtype == torch.bfloat16
               and p.h <= 256)
-    launches = (3 if direct else 4) * args.steps
+    launches = launches_per_step * args.steps
     del graphs
 
     # end-to-end through the public calls with host buffers (pinned), copies inside timing
@@ -432,7 +434,7 @@ def run_ours(args, p, rank, world, dev):
     pk, pk_kind = peaks()
     gemm_ms = statistics.mean(per_kernel.get("gemm", [float("nan")]))
     quant_ms = statistics.mean(per_kernel.get("quantize", [float("nan")]))
-    dec_ms = statistics.mean(per_kernel.get("decode", [float("nan")]))
+    dec_ms = statistics.mean(per_kernel["decode"]) if "decode" in per_kernel else None
     flops = 2.0 * p.T * p.d * p.out
     gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
     traffic, traffic_src = profile_traffic(f"k2_gemm_{p.name}.md", GEMM_SOURCES)
@@ -441,6 +443,10 @@ def run_ours(args, p, rank, world, dev):
     # centroids it writes for the GEMM instead, and s
     out_bytes = 2 * p.d if direct else p.d * p.bits_a // 8
     q_bytes = p.T * (in_bytes * p.d + out_bytes + 4)
+    # with 4-bit weights the one-call path's K1 also decodes the weight codes (no decode launch)
+    fused_dec = direct and dec_ms is None
+    if fused_dec:
+        q_bytes += p.out * p.d * (p.bits_w / 8 + 2)
     q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
@@ -467,7 +473,8 @@ def run_ours(args, p, rank, world, dev):
             "algorithmic_per_launch": flops,
         },
         "roofline_quantize": {
-            "kernel": "k1_rotquant (fp16-operand output)" if direct else "k1_rotquant",
+            "kernel": ("k1_rotquant (fp16-operand output + fused weight decode)" if fused_dec
+                       else "k1_rotquant (fp16-operand output)" if direct else "k1_rotquant"),
             "bound": "hbm", "achieved": q_gbs,
             "peak": pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "unit": "GB/s",
             "frac": q_gbs / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
@@ -477,9 +484,10 @@ def run_ours(args, p, rank, world, dev):
         "gpu_launches": launches,
         "timing": f"value/ms_per_step: {timing_mode} of the step; kernels_ms_mean and the "
                   f"rooflines: CUDA events around each kernel of {n_k} eager steps queued "
-                  "behind a GPU spin (device time, not host gaps); on the one-call path the "
-                  "decode (weights) runs on a side stream beside K1, so its event time "
-                  "includes that overlap",
+                  "behind a GPU spin (device time, not host gaps); on the one-call path "
+                  + ("K1 also decodes the 4-bit weights (no decode launch)" if fused_dec else
+                     "the decode (weights) runs on a side stream beside K1, so its event "
+                     "time includes that overlap"),
         "eager_ms_per_step": eager_ms / args.steps,
         "host_ms_per_step_eager": host_ms / args.steps,
         "clocks": clock_info,

@@ -271,8 +271,10 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     uint32_t *dect = gent + p.ent_words;             // A16 only (dec_words = 0 otherwise)
     float2 *red = reinterpret_cast<float2 *>(dect + p.dec_words);
     unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + 2 * NG * kMaxSeg);
-    int *sched = reinterpret_cast<int *>(bars + 2 * NG + 2);   // [0] next pair, [1 + grp]
-    unsigned char *raw = reinterpret_cast<unsigned char *>(sched + 16);
+    // [0] next pair, [1 + grp] a group's next pair, [16] next decode chunk, [17 + grp] a
+    // group's decode chunk
+    int *sched = reinterpret_cast<int *>(bars + 2 * NG + 2);
+    unsigned char *raw = reinterpret_cast<unsigned char *>(sched + 32);
     unsigned char *myraw = raw + (size_t)grp * nstage * 2 * row_in;
     unsigned char *pairs = raw + (size_t)NG * nstage * 2 * row_in;
     unsigned char *mypairs = pairs + (size_t)grp * d * 4;
@@ -283,6 +285,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
         for (int b = 0; b < 2 * NG + 1; ++b)
             mbar_init(smem_u32(&bars[b]), 1);
         sched[0] = NG;                               // pairs lo .. lo + NG - 1 start the groups
+        sched[16] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -554,6 +557,42 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
         }
         my = nxt;
     }
+
+    if constexpr (NAMED && A16) {
+        // ---- fused weight decode: this CTA's share of the code words, in chunks of GT * 8 ---
+        if (p.wdec_groups > 0) {
+            const long long dlo = (long long)blockIdx.x * p.wdec_groups / gridDim.x;
+            const long long dcnt = ((long long)blockIdx.x + 1) * p.wdec_groups / gridDim.x - dlo;
+            const uint32_t *wc = p.wdec_codes + dlo;
+            uint4 *wo = p.wdec_out + dlo;
+            constexpr int kU = 8;                          // code words per thread and chunk
+            for (;;) {
+                if (g == 0)
+                    sched[17 + grp] = atomicAdd(&sched[16], 1);
+                group_sync();
+                const long long c0 = (long long)sched[17 + grp] * GT * kU;
+                group_sync();                              // read before the next claim
+                if (c0 >= dcnt)
+                    break;
+                uint32_t wv[kU];
+#pragma unroll
+                for (int j = 0; j < kU; ++j) {
+                    const long long i = c0 + g + (long long)j * GT;
+                    wv[j] = i < dcnt ? __ldg(wc + i) : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < kU; ++j) {
+                    const long long i = c0 + g + (long long)j * GT;
+                    if (i < dcnt) {
+                        uint32_t o[4];
+                        decode8(wv[j], p.wdec_src[0], p.wdec_src[1], p.wdec_src[2],
+                                p.wdec_src[3], o);
+                        wo[i] = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+            }
+        }
+    }
 }
 
 // Shared-memory attributes are set once per kernel and device, and occupancy is cached per
@@ -642,7 +681,7 @@ size_t k1_smem(const K1Params &p, int in_f32, int NG, int stages) {
     size_t b = 4 * (size_t)(p.tbl_words + p.ent_words + p.dec_words);   // tables, entries
     b += sizeof(float2) * 2 * NG * kMaxSeg;                // norm partials, two buffers
     b += 8 * (size_t)(2 * NG + 2);                         // mbarriers
-    b += 4 * 16;                                           // pair scheduling words
+    b += 4 * 32;                                           // pair and decode scheduling words
     b += (size_t)NG * stages * 2 * row_in;                 // raw rows
     if (!in_f32)
         b += (size_t)NG * p.d * 4;                         // interleaved pairs
@@ -662,21 +701,32 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     long long ctas_needed;
     int NG;
     const bool named = GT % 32 == 0 && !in_f32;
+    if (p.wdec_groups > 0 && !(named && p.a16)) {
+        *why = "fused weight decode needs fp16 output and whole-warp groups";
+        return cudaErrorInvalidValue;
+    }
     if (named) {
         // Groups of whole warps: one CTA per SM with as many groups as the register file
         // holds (96 registers a thread; at most 15 named barriers and 1024 threads), each CTA
         // an equal share of the pairs.  The group count is the smallest that takes the share
         // in the same number of rounds, so the rounds stay full.
-        ctas_needed = std::min<long long>(num_sms, npairs);
+        // With a fused weight decode every SM takes a share of the decode with all the groups
+        // it holds, whatever the number of pairs.
+        const bool wdec = p.wdec_groups > 0;
+        ctas_needed = wdec ? num_sms : std::min<long long>(num_sms, npairs);
         const long long share = (npairs + ctas_needed - 1) / ctas_needed;
         // registers: each of the SM's four 16K-register partitions holds 5 warps of 96
         constexpr int kWarpsPerSm = 4 * ((65536 / 4) / (96 * 32));
         int ng_max = std::min(std::min(15, 1024 / GT), kWarpsPerSm * 32 / GT);
         while (ng_max > 1 && k1_smem(p, in_f32, ng_max, stages) > 220 * 1024)
             --ng_max;
-        ng_max = (int)std::max(1LL, std::min<long long>(ng_max, share));
-        const long long rounds = (share + ng_max - 1) / ng_max;
-        NG = (int)((share + rounds - 1) / rounds);
+        if (wdec) {
+            NG = ng_max;
+        } else {
+            ng_max = (int)std::max(1LL, std::min<long long>(ng_max, share));
+            const long long rounds = (share + ng_max - 1) / ng_max;
+            NG = (int)((share + rounds - 1) / rounds);
+        }
     } else {
         // Groups that share warps run in lockstep: several smaller CTAs per SM.
         NG = 256 / GT;

@@ -469,9 +469,19 @@ bool tc_k1_requested() {
 
 // K1 for `rows` rows of x: packed codes into `codes`, or (a16 non-null, bits 2/4/8, bf16, h <=
 // 256) the codes' fp16 unit centroids into a16 [rows, d]; norms into `norms`.
+// A weight decode that K1 takes on (fp16 output, whole-warp groups, 4-bit weights of an
+// odd-symmetric codebook): the codes of `rows` weight rows into fp16 unit centroids.
+struct FusedDecode {
+    const oq_codebook *cb = nullptr;
+    const uint8_t *codes = nullptr;
+    uint16_t *out = nullptr;
+    long long rows = 0;
+};
+
 int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dtype, int rows,
                   int d, uint8_t *codes, float *norms, void *stream, float eps,
-                  const char *who, bool gelu = false, uint16_t *a16 = nullptr) {
+                  const char *who, bool gelu = false, uint16_t *a16 = nullptr,
+                  const FusedDecode *fd = nullptr) {
     if (!r || !cb)
         return fail(OQ_EINVAL, "%s: null handle", who);
     if (check_dims(d, who) != OQ_OK)
@@ -564,6 +574,14 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
         } else {
             p.dec_img = cw->dev_dec[dev];
             p.dec_words = (int)cw->dec_img.size();
+        }
+        if (fd && fd->rows > 0) {
+            if (!oq::decode8_sources(fd->cb->lut, &p.wdec_src[0], &p.wdec_src[1],
+                                     &p.wdec_src[2], &p.wdec_src[3]))
+                return fail(OQ_EINVAL, "%s: 4-bit weight codebook is not odd-symmetric", who);
+            p.wdec_codes = reinterpret_cast<const uint32_t *>(fd->codes);
+            p.wdec_out = reinterpret_cast<uint4 *>(fd->out);
+            p.wdec_groups = fd->rows * (long long)d / 8;
         }
     }
     cudaError_t e = timed(OQ_KERNEL_QUANTIZE, st, [&] {
@@ -1103,6 +1121,36 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     float *sv = s ? s : reinterpret_cast<float *>(w8 + a_bytes + b_bytes);
     uint8_t *codes = direct ? nullptr : w8 + a_bytes + b_bytes + s_bytes;
     std::string why;
+    // 4-bit weights of an odd-symmetric codebook with the one-CTA-per-SM K1: the K1 groups
+    // that run out of token pairs decode the weights (no second kernel, no side stream)
+    uint32_t src_probe[4];
+    const bool fuse = direct && cw->bits == 4 && !tc_k1_requested() &&
+                      oq::k1_named(d, dtype == OQ_BF16) &&
+                      oq::decode8_sources(cw->lut, &src_probe[0], &src_probe[1], &src_probe[2],
+                                          &src_probe[3]);
+    if (fuse) {
+        FusedDecode fd;
+        fd.cb = cw;
+        fd.codes = W_codes;
+        fd.out = B16;
+        fd.rows = out_features;
+        rc = quantize_rows(r, ca, x, dtype, T, d, nullptr, sv, st, 1e-8f, who, gelu, A16, &fd);
+        if (rc == OQ_OK) {
+            e = timed(OQ_KERNEL_GEMM, st, [&] {
+                return oq::launch_gemm(A16, nullptr, nullptr, B16, sv, row_norms, y,
+                                       out_dtype == OQ_BF16, T, out_features, d, st, di->sms,
+                                       &why);
+            });
+            if (e != cudaSuccess)
+                rc = fail_cuda(e, why.c_str());
+        }
+        cudaError_t e2 = cudaFreeAsync(ws, st);
+        if (rc != OQ_OK)
+            return rc;
+        if (e2 != cudaSuccess)
+            return fail_cuda(e2, "oq_quantized_linear: workspace release");
+        return OQ_OK;
+    }
     {
         // the weight decode needs nothing from x: it runs on the side stream beside K1
         std::lock_guard<std::mutex> lk(g_side_mu);

@@ -79,11 +79,21 @@ struct K1Params {
     const uint32_t *dec_img;   // byte -> centroid table for a16 (bits 2, 8)
     int dec_words;             // its size in words (multiple of 4; 0 without a16)
     uint32_t dec_src[4];       // a16 with 4-bit codes: byte-permute decode sources
+    // Fused weight decode (a16, groups of whole warps): once a group has no token pair left it
+    // decodes 4-bit weight codes of an odd-symmetric codebook into fp16 unit centroids, each
+    // CTA an equal share of the wdec_groups groups of 8 codes (one 32-bit code word -> 16 bytes).
+    const uint32_t *wdec_codes;   // [wdec_groups] code words (W_codes [N, d/2] as words)
+    uint4 *wdec_out;              // [wdec_groups] fp16 x 8 (B16 [N, d])
+    long long wdec_groups;        // 0: no fused decode
+    uint32_t wdec_src[4];         // byte-permute decode sources of the weight codebook
 };
 // True when K1 can write fp16 centroids itself (launch_k1 with p.a16 set).
 inline bool k1_a16_supported(int bits, int h, bool bf16_in) {
     return bf16_in && h <= 256 && (bits == 2 || bits == 4 || bits == 8);
 }
+// True when K1 runs as one CTA per SM with named-barrier groups (bf16 rows, d/32 threads per
+// token pair a whole number of warps); the fused weight decode needs it.
+inline bool k1_named(int d, bool bf16_in) { return bf16_in && (d / 32) % 32 == 0; }
 // (4-bit additionally needs an odd-symmetric codebook, which every Lloyd-Max codebook here is;
 // the host checks it when it builds dec_src.)
 
