@@ -58,6 +58,9 @@ def parse():
                     help="forward: oq_quantized_linear (one call, codes stay on chip); "
                          "calls: oq_quantize_act then oq_linear")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time K1 (oq_quantize_act, codes output) over the activation sweep "
+                         "(d x h x bits x T) and print one JSON line per point, then a summary")
     return ap.parse_args()
 
 
@@ -497,6 +500,59 @@ def run_ours(args, p, rank, world, dev):
     return out
 
 
+def run_sweep(args, dev):
+    """K1 over the activation sweep: d x h x activation bits x T, bf16 N(0,1) rows with 1 %
+    channels x50.  Rows are a 4096-row synthetic block tiled to T (K1's cost does not depend
+    on the values), rotated over buffer sets larger than the L2 when they fit in 8 GB; the
+    time per launch is the CUDA-event mean over `steps` launches after `warmup`."""
+    from calibration_free_bit_b200 import build as B
+    B.build()
+    from calibration_free_bit_b200 import oq
+
+    pk, pk_kind = peaks()
+    hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    rows_out = []
+    blocks = {}
+    for sp in synth.sweep_points():
+        d, h, bits, T = sp.d, sp.h, sp.bits_a, sp.T
+        if d not in blocks:
+            blocks[d] = synth.activations(synth.sweep_projection(d, 128, 4, 4096)).to(dev)
+        blk = blocks[d]
+        x = blk.repeat((T + blk.shape[0] - 1) // blk.shape[0], 1)[:T].contiguous()
+        one = T * d * 2
+        nb = 1 if one > 2e9 else max(1, min(8, int(400e6 // max(one, 1)) + 1))
+        xs = [x] + [x.clone() for _ in range(nb - 1)]
+        r = oq.oq_build_rpbh(d, h, 0)
+        ca = oq.oq_lloyd_max(d, bits)
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=dev)
+        s = torch.empty(T, device=dev)
+        n = max(3, min(args.steps, 50 if T >= 4096 else 200))
+        for i in range(max(3, min(args.warmup, 5))):
+            oq.oq_quantize_act(r, ca, xs[i % nb], codes, s)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(n):
+            oq.oq_quantize_act(r, ca, xs[i % nb], codes, s)
+        e1.record()
+        torch.cuda.synchronize()
+        oq.oq_check()
+        us = e0.elapsed_time(e1) / n * 1e3
+        byts = T * (2 * d + d * bits // 8 + 4)
+        gbs = byts / (us * 1e-6) / 1e9
+        row = {"d": d, "h": h, "bits_a": bits, "T": T, "k1_us": round(us, 3),
+               "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4), "tokens_per_s": T / (us * 1e-6)}
+        rows_out.append(row)
+        print(json.dumps(row), flush=True)
+        del xs, x, codes, s
+    big = [r_ for r_ in rows_out if r_["T"] == 65536]
+    print(json.dumps({"sweep": "k1 codes output", "points": len(rows_out), "peak_gbs": hbm,
+                      "peak_kind": pk_kind,
+                      "T65536_frac_min": min(r_["frac"] for r_ in big) if big else None,
+                      "T65536_frac_max": max(r_["frac"] for r_ in big) if big else None}),
+          flush=True)
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -511,6 +567,10 @@ def main():
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    if args.sweep:
+        if rank == 0:
+            run_sweep(args, dev)
+        return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=dev)
