@@ -9,7 +9,7 @@
 // B200 design (one HBM-bound pass: read 2d bytes per bf16 row, write d*b/8 + 4):
 //   * Persistent CTAs, each with `groups` thread groups of d/32 threads; a group owns one
 //     token PAIR per round.  The pair's two rows stream into shared memory with bulk copies
-//     (cp.async.bulk, mbarrier completion, no multicast) one round ahead of the compute.
+//     (bulk copies that complete on an mbarrier) one round ahead of the compute.
 //   * bf16 rows are interleaved into 32-bit words (x_t0[j], x_t1[j]), so one 4-byte gather
 //     load serves both tokens and the butterfly runs on packed fp32x2 (add/sub/fma .f32x2,
 //     new on sm_100).  Each half of an 8-element chunk goes to a 16-byte slot the host
@@ -125,7 +125,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
-// One-dimensional bulk copy global -> shared, completion counted on `bar` (no multicast).
+// One-dimensional bulk copy global -> this CTA's shared memory, completion counted on `bar`.
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes,
                                           uint32_t bar) {
     asm volatile(

@@ -364,7 +364,8 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
 // time, and the ring holds 6 stages.  Barriers: the leader's full barrier counts both CTAs'
 // TMA bytes (only the leader arms it); the leader's MMA commits release both CTAs' stages and
 // signal both CTAs' accumulator-full barriers (multicast commit); every epilogue warp of both
-// CTAs arrives on the leader's accumulator-empty barrier.  TMA loads carry no multicast.
+// CTAs arrives on the leader's accumulator-empty barrier.  Every TMA load fills only its own
+// CTA's shared memory.
 // ------------------------------------------------------------------------------------------
 constexpr int P_STAGES = 6;
 constexpr int P_BM = 256, P_BN = 256;                    // pair tile

@@ -1,7 +1,7 @@
 // sm100_common.cuh -- small sm_100a building blocks shared by liboq's GEMM kernels:
 // shared-memory addressing, bounded mbarrier waits, TMA tile loads and stores, tcgen05
 // descriptors, MMA issue/commit, TMEM loads and stores, the output epilogue chunk.  Inline PTX;
-// no multicast anywhere.
+// every tile load writes only the issuing CTA's shared memory.
 #pragma once
 
 #include <cuda.h>
@@ -305,7 +305,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
 }
 
 // Pair TMA load: this CTA's tile lands in its own shared memory; the transaction bytes count
-// on the mbarrier at `cluster_bar` (the leader CTA's).  No multicast.
+// on the mbarrier at `cluster_bar` (the leader CTA's); the data lands in this CTA only.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x,
                                                  int y, uint32_t cluster_bar) {
     asm volatile(
