@@ -269,7 +269,8 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     uint32_t *table = reinterpret_cast<uint32_t *>(smem);
     uint32_t *gent = table + p.tbl_words;
     uint32_t *dect = gent + p.ent_words;             // A16 only (dec_words = 0 otherwise)
-    float2 *red = reinterpret_cast<float2 *>(dect + p.dec_words);
+    uint32_t *wdect = dect + p.dec_words;            // fused 2-bit weight decode table
+    float2 *red = reinterpret_cast<float2 *>(wdect + p.wdec_words);
     unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + 2 * NG * kMaxSeg);
     // [0] next pair, [1 + grp] a group's next pair, [16] next decode chunk, [17 + grp] a
     // group's decode chunk
@@ -291,11 +292,14 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     __syncthreads();
     if (tid == 0) {
         // host-built table, entry and decode images: bulk copies
-        mbar_expect_tx(setup_bar, 4u * (p.tbl_words + p.ent_words + p.dec_words));
+        mbar_expect_tx(setup_bar,
+                       4u * (p.tbl_words + p.ent_words + p.dec_words + p.wdec_words));
         bulk_copy(smem_u32(table), p.tbl_img, 4u * p.tbl_words, setup_bar);
         bulk_copy(smem_u32(gent), p.ent_img, 4u * p.ent_words, setup_bar);
         if (p.dec_words > 0)
             bulk_copy(smem_u32(dect), p.dec_img, 4u * p.dec_words, setup_bar);
+        if (p.wdec_words > 0)
+            bulk_copy(smem_u32(wdect), p.wdec_img, 4u * p.wdec_words, setup_bar);
     }
 
     // this thread's 32 rotated positions: pos0 + e with pos0 = g * 32
@@ -564,7 +568,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             const long long dlo = (long long)blockIdx.x * p.wdec_groups / gridDim.x;
             const long long dcnt = ((long long)blockIdx.x + 1) * p.wdec_groups / gridDim.x - dlo;
             const uint32_t *wc = p.wdec_codes + dlo;
-            uint4 *wo = p.wdec_out + dlo;
+            uint4 *wo = p.wdec_out + (p.wdec_bits == 4 ? dlo : 2 * dlo);
             constexpr int kU = 8;                          // code words per thread and chunk
             for (;;) {
                 if (g == 0)
@@ -584,10 +588,18 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
                 for (int j = 0; j < kU; ++j) {
                     const long long i = c0 + g + (long long)j * GT;
                     if (i < dcnt) {
-                        uint32_t o[4];
-                        decode8(wv[j], p.wdec_src[0], p.wdec_src[1], p.wdec_src[2],
-                                p.wdec_src[3], o);
-                        wo[i] = make_uint4(o[0], o[1], o[2], o[3]);
+                        if (p.wdec_bits == 4) {
+                            uint32_t o[4];
+                            decode8(wv[j], p.wdec_src[0], p.wdec_src[1], p.wdec_src[2],
+                                    p.wdec_src[3], o);
+                            wo[i] = make_uint4(o[0], o[1], o[2], o[3]);
+                        } else {                           // 2-bit: a byte = 4 centroids
+                            const uint2 *t2 = reinterpret_cast<const uint2 *>(wdect);
+                            const uint2 q0 = t2[wv[j] & 0xffu], q1 = t2[(wv[j] >> 8) & 0xffu];
+                            const uint2 q2 = t2[(wv[j] >> 16) & 0xffu], q3 = t2[wv[j] >> 24];
+                            wo[2 * i] = make_uint4(q0.x, q0.y, q1.x, q1.y);
+                            wo[2 * i + 1] = make_uint4(q2.x, q2.y, q3.x, q3.y);
+                        }
                     }
                 }
             }
@@ -678,7 +690,7 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
 
 size_t k1_smem(const K1Params &p, int in_f32, int NG, int stages) {
     const size_t row_in = (size_t)p.d * (in_f32 ? 4 : 2);
-    size_t b = 4 * (size_t)(p.tbl_words + p.ent_words + p.dec_words);   // tables, entries
+    size_t b = 4 * (size_t)(p.tbl_words + p.ent_words + p.dec_words + p.wdec_words);
     b += sizeof(float2) * 2 * NG * kMaxSeg;                // norm partials, two buffers
     b += 8 * (size_t)(2 * NG + 2);                         // mbarriers
     b += 4 * 32;                                           // pair and decode scheduling words

@@ -576,12 +576,25 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
             p.dec_words = (int)cw->dec_img.size();
         }
         if (fd && fd->rows > 0) {
-            if (!oq::decode8_sources(fd->cb->lut, &p.wdec_src[0], &p.wdec_src[1],
-                                     &p.wdec_src[2], &p.wdec_src[3]))
-                return fail(OQ_EINVAL, "%s: 4-bit weight codebook is not odd-symmetric", who);
+            oq_codebook *fw = const_cast<oq_codebook *>(fd->cb);
+            if (fw->bits == 4) {
+                if (!oq::decode8_sources(fw->lut, &p.wdec_src[0], &p.wdec_src[1],
+                                         &p.wdec_src[2], &p.wdec_src[3]))
+                    return fail(OQ_EINVAL, "%s: 4-bit weight codebook is not odd-symmetric",
+                                who);
+            } else if (fw->bits == 2) {
+                if ((rc = upload(fw->mu, &fw->dev_dec[dev], fw->dec_img,
+                                 "upload weight decode table")) != OQ_OK)
+                    return rc;
+                p.wdec_img = fw->dev_dec[dev];
+                p.wdec_words = (int)fw->dec_img.size();
+            } else {
+                return fail(OQ_EINVAL, "%s: fused weight decode takes 2- or 4-bit codes", who);
+            }
+            p.wdec_bits = fw->bits;
             p.wdec_codes = reinterpret_cast<const uint32_t *>(fd->codes);
             p.wdec_out = reinterpret_cast<uint4 *>(fd->out);
-            p.wdec_groups = fd->rows * (long long)d / 8;
+            p.wdec_groups = fd->rows * (long long)d * fw->bits / 32;
         }
     }
     cudaError_t e = timed(OQ_KERNEL_QUANTIZE, st, [&] {
@@ -1121,13 +1134,17 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     float *sv = s ? s : reinterpret_cast<float *>(w8 + a_bytes + b_bytes);
     uint8_t *codes = direct ? nullptr : w8 + a_bytes + b_bytes + s_bytes;
     std::string why;
-    // 4-bit weights of an odd-symmetric codebook with the one-CTA-per-SM K1: the K1 groups
-    // that run out of token pairs decode the weights (no second kernel, no side stream)
+    // 2-bit weights, or 4-bit weights of an odd-symmetric codebook, with the one-CTA-per-SM
+    // K1: the K1 groups that run out of token pairs decode the weights (no second kernel, no
+    // side stream)
     uint32_t src_probe[4];
-    const bool fuse = direct && cw->bits == 4 && !tc_k1_requested() &&
-                      oq::k1_named(d, dtype == OQ_BF16) &&
-                      oq::decode8_sources(cw->lut, &src_probe[0], &src_probe[1], &src_probe[2],
-                                          &src_probe[3]);
+    // Only while the decode is no bigger than K1's own work (N <= T): a larger weight matrix
+    // decodes faster beside K1 than in its tail.
+    const bool fuse =
+        direct && out_features <= T && !tc_k1_requested() && oq::k1_named(d, dtype == OQ_BF16) &&
+        (cw->bits == 2 || (cw->bits == 4 && oq::decode8_sources(cw->lut, &src_probe[0],
+                                                                 &src_probe[1], &src_probe[2],
+                                                                 &src_probe[3])));
     if (fuse) {
         FusedDecode fd;
         fd.cb = cw;

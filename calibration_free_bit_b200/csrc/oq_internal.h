@@ -80,12 +80,17 @@ struct K1Params {
     int dec_words;             // its size in words (multiple of 4; 0 without a16)
     uint32_t dec_src[4];       // a16 with 4-bit codes: byte-permute decode sources
     // Fused weight decode (a16, groups of whole warps): once a group has no token pair left it
-    // decodes 4-bit weight codes of an odd-symmetric codebook into fp16 unit centroids, each
-    // CTA an equal share of the wdec_groups groups of 8 codes (one 32-bit code word -> 16 bytes).
-    const uint32_t *wdec_codes;   // [wdec_groups] code words (W_codes [N, d/2] as words)
-    uint4 *wdec_out;              // [wdec_groups] fp16 x 8 (B16 [N, d])
+    // decodes weight codes into fp16 unit centroids, each CTA an equal share of the
+    // wdec_groups 32-bit code words.  4-bit codes of an odd-symmetric codebook: byte-permute
+    // decode, one word -> 8 centroids (16 bytes).  2-bit codes: the codebook's byte table
+    // (wdec_img, bulk-copied beside the other images), one word -> 16 centroids (32 bytes).
+    const uint32_t *wdec_codes;   // [wdec_groups] code words (W_codes [N, d*bits/8] as words)
+    uint4 *wdec_out;              // B16 [N, d]: 1 (4-bit) or 2 (2-bit) uint4 per word
     long long wdec_groups;        // 0: no fused decode
-    uint32_t wdec_src[4];         // byte-permute decode sources of the weight codebook
+    int wdec_bits;                // 4 or 2
+    uint32_t wdec_src[4];         // 4-bit: byte-permute decode sources of the weight codebook
+    const uint32_t *wdec_img;     // 2-bit: byte -> four fp16 centroids (256 x 8 bytes)
+    int wdec_words;               // its size in words (0 for 4-bit)
 };
 // True when K1 can write fp16 centroids itself (launch_k1 with p.a16 set).
 inline bool k1_a16_supported(int bits, int h, bool bf16_in) {

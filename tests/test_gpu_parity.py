@@ -445,14 +445,17 @@ def test_k1_tensor_core_path(oq):
     (2560, 128, 6, 6, 50, 336, False, torch.float32),       # fallback: 6-bit
     (2048, 512, 4, 4, 40, 128, False, torch.float32),       # fallback: h = 512
     (3072, 128, 4, 2, 100, 384, True, torch.float32),       # GELU pre-activation
-    (1024, 64, 2, 4, 2, 48, False, torch.bfloat16),         # fused weight decode, one pair
-    (3072, 128, 4, 4, 1, 16, True, torch.float32),          # fused decode, T = 1, GELU
+    (1024, 64, 2, 4, 64, 48, False, torch.bfloat16),        # fused decode, 32 pairs < SMs
+    (2048, 128, 2, 2, 400, 400, False, torch.float32),      # fused 2-bit weight decode
+    (3072, 128, 4, 4, 17, 16, True, torch.float32),         # fused decode, odd T, GELU
+    (3072, 128, 4, 4, 1, 16, False, torch.float32),         # N > T: decode beside K1
 ])
 def test_quantized_linear_matches_the_two_calls(oq, d, h, ba, bw, T, N, gelu, out):
     """oq_quantized_linear (x -> y, codes never in memory) is bit-identical to
-    oq_quantize_act (or _gelu) followed by oq_linear: y and the norms s.  With 4-bit weights,
-    2/4/8-bit activations and d a multiple of 1024 the weight decode runs inside K1 (also when
-    there are fewer token pairs than SMs); the other rows take the side-stream decode."""
+    oq_quantize_act (or _gelu) followed by oq_linear: y and the norms s.  With 2- or 4-bit
+    weights, 2/4/8-bit activations, d a multiple of 1024 and N <= T the weight decode runs
+    inside K1 (also when there are fewer token pairs than SMs); the other rows take the
+    side-stream decode."""
     p = synth.sweep_projection(d, 128, 4, T) if d != 3072 or T != 4608 else \
         synth.get("flux_attn_w4a4")[0]
     x = synth.activations(p).cuda()
