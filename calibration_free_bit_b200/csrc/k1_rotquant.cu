@@ -7,9 +7,12 @@
 // the RPBH rotation of the summary's RPBH paragraph, applied as an O(d log h) butterfly.
 //
 // B200 design (one HBM-bound pass: read 2d bytes per bf16 row, write d*b/8 + 4):
-//   * Persistent CTAs, each with `groups` thread groups of d/32 threads; a group owns one
-//     token PAIR per round.  The pair's two rows stream into shared memory with bulk copies
-//     (bulk copies that complete on an mbarrier) one round ahead of the compute.
+//   * Thread groups of d/32 threads; a group works on one token PAIR at a time, whose two
+//     rows stream into shared memory with bulk copies (completing on an mbarrier) one pair
+//     ahead of the compute.  bf16 rows whose groups are whole warps: one CTA per SM, an
+//     equal contiguous share of the pairs per CTA, each group on its own named barrier
+//     taking its next pair from a shared counter.  Otherwise several smaller CTAs per SM
+//     step through the pairs in lockstep rounds.
 //   * bf16 rows are interleaved into 32-bit words (x_t0[j], x_t1[j]), so one 4-byte gather
 //     load serves both tokens and the butterfly runs on packed fp32x2 (add/sub/fma .f32x2,
 //     new on sm_100).  Each half of an 8-element chunk goes to a 16-byte slot the host
@@ -27,6 +30,9 @@
 //     round-down, word = table[q >> F], code = (word + q*G) >> 24.  The table words fold the
 //     cell's base code and its boundary, so the decision is exact in the fixed-point q grid
 //     (2^-23 of the grid span, < 1.2e-6 sigma).  Bit widths 2/3/4/6/8 pack LSB-first.
+//   * fp16 output (the one-call path): each code's fp16 unit centroid instead of the packed
+//     codes (the GEMM's A operand); with it, the groups that run out of pairs can decode the
+//     layer's 2- or 4-bit weight codes into the GEMM's B operand (each CTA an equal share).
 //   * Every mbarrier wait is bounded (about 2 s of SM clock); a wait that gives up sets a bit
 //     in the device error word (read by oq_check) and the round's outputs are not written.
 #include <cuda_bf16.h>
