@@ -152,7 +152,10 @@ int oq_quantize_act_gelu(const oq_rpbh *r, const oq_codebook *ca, const void *x,
  * are instead decoded inside the GEMM kernel, into its shared-memory operand tiles, and only
  * the weight codes get an fp16 buffer (less device memory, more decode work per call).
  * Either way the temporary device memory is stream-ordered, from a library-owned
- * pool.  Errors: as above, plus OQ_ECUDA if the pool allocation fails. */
+ * pool.  The fp16 operands meet in a tcgen05 GEMM on pairs of CTAs (256 x 256 output tiles);
+ * the environment variable OQ_GEMM_PAIR=0 (read once per process) selects the single-CTA
+ * GEMM (128 x 256 tiles) instead; both give the same y.
+ * Errors: as above, plus OQ_ECUDA if the pool allocation fails. */
 int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
               const float *s, const uint8_t *W_codes, const float *row_norms, int T, int d,
               int out_features, void *y, int out_dtype, void *stream);
@@ -164,8 +167,11 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * oq_quantize_act followed by oq_linear, without materialising x_codes: the rotate+quantize
  * kernel writes each code's fp16 unit centroid straight into the GEMM's A operand (bf16 x,
  * ba in {2, 4, 8}, h <= 256; otherwise codes and the decode prepass are used inside the
- * call), and the weight codes are decoded on a library-owned side stream of the device
- * while x is quantized.  y and s are bit-identical to oq_quantize_act + oq_linear.
+ * call).  With 2- or 4-bit weight codes, d a multiple of 1024, bf16 x and
+ * out_features <= T, that kernel also decodes the weight codes into the GEMM's B operand once
+ * it runs out of tokens; otherwise the weight codes are decoded on a library-owned side
+ * stream of the device while x is quantized.  y and s are bit-identical to
+ * oq_quantize_act + oq_linear.
  * x: device [T, d] of dtype; W_codes [out_features, d*bw/8]; row_norms fp32 [out_features];
  * y: device [T, out_features] of out_dtype (OQ_F32 or OQ_BF16); s: optional device fp32 [T]
  * receiving the norms (NULL: kept internal).  flags: OQ_FORWARD_GELU quantizes GELU(x)
