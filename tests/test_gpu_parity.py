@@ -476,3 +476,33 @@ def test_quantized_linear_matches_the_two_calls(oq, d, h, ba, bw, T, N, gelu, ou
     y2 = oq.oq_quantized_linear(r, ca, cw, x, wc, rn, out_dtype=out, gelu=gelu)
     oq.oq_check()
     assert torch.equal(y2, y)
+
+
+def test_quantized_linear_back_to_back_on_one_stream(oq):
+    """Kernels launched with programmatic stream serialisation start while their predecessor
+    finishes and wait for it before touching data.  Steps that follow each other on one
+    stream, with x rewritten in place by a torch kernel between them and the pooled workspace
+    reused, each equal the two-call result for the x they saw."""
+    p = synth.get("flux_attn_w4a4")[0]
+    x0 = synth.activations(p, rows=np.arange(0, 1024)).cuda()
+    x1 = synth.activations(p, rows=np.arange(1024, 2048)).cuda()
+    W = (torch.randn(3072, p.d, generator=torch.Generator().manual_seed(7)) /
+         math.sqrt(p.d)).cuda()
+    r = oq.oq_build_rpbh(p.d, p.h, 0)
+    ca, cw = oq.oq_lloyd_max(p.d, 4), oq.oq_lloyd_max(p.d, 4)
+    wc, rn = oq.oq_quantize_weight(r, cw, W)
+    refs = []
+    for xx in (x0, x1, 2 * x0):
+        xc, s = oq.oq_quantize_act(r, ca, xx)
+        refs.append(oq.oq_linear(ca, cw, xc, s, wc, rn))
+    x = x0.clone()
+    ys = []
+    for k in range(3):
+        if k == 1:
+            x.copy_(x1)                                   # a torch kernel between two steps
+        if k == 2:
+            x.copy_(x0).mul_(2)
+        ys.append(oq.oq_quantized_linear(r, ca, cw, x, wc, rn))
+    oq.oq_check()
+    for y, ref in zip(ys, refs):
+        assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
