@@ -354,7 +354,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     if (!mbar_wait(setup_bar, 0))
         atomicOr(&g_k1_err, K1_ERR_COPY_WAIT);
 
-    int my = grp;                                      // this round's pair: lo + my
+    int my = grp;                                      // the pair in hand: lo + my
     for (int round = 0;; ++round) {
         if (dyn ? my >= cnt : my - grp >= cnt)
             break;                                     // uniform across the group / the CTA
