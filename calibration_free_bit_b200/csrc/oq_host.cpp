@@ -1138,10 +1138,12 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     // K1: the K1 groups that run out of token pairs decode the weights (no second kernel, no
     // side stream)
     uint32_t src_probe[4];
-    // Only while the decode is no bigger than K1's own work (N <= T): a larger weight matrix
-    // decodes faster beside K1 than in its tail.
+    // Only while the decode is no bigger than K1's own work (N <= T) and K1 holds at least
+    // four groups per SM (d <= 5120): a larger weight matrix, or one decoded by a single group
+    // per SM, decodes faster beside K1 than in its tail.
     const bool fuse =
-        direct && out_features <= T && !tc_k1_requested() && oq::k1_named(d, dtype == OQ_BF16) &&
+        direct && out_features <= T && d <= 5120 && !tc_k1_requested() &&
+        oq::k1_named(d, dtype == OQ_BF16) &&
         (cw->bits == 2 || (cw->bits == 4 && oq::decode8_sources(cw->lut, &src_probe[0],
                                                                  &src_probe[1], &src_probe[2],
                                                                  &src_probe[3])));

@@ -167,7 +167,7 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * oq_quantize_act followed by oq_linear, without materialising x_codes: the rotate+quantize
  * kernel writes each code's fp16 unit centroid straight into the GEMM's A operand (bf16 x,
  * ba in {2, 4, 8}, h <= 256; otherwise codes and the decode prepass are used inside the
- * call).  With 2- or 4-bit weight codes, d a multiple of 1024, bf16 x and
+ * call).  With 2- or 4-bit weight codes, d a multiple of 1024 up to 5120, bf16 x and
  * out_features <= T, that kernel also decodes the weight codes into the GEMM's B operand once
  * it runs out of tokens; otherwise the weight codes are decoded on a library-owned side
  * stream of the device while x is quantized.  y and s are bit-identical to

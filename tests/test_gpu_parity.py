@@ -453,9 +453,9 @@ def test_k1_tensor_core_path(oq):
 def test_quantized_linear_matches_the_two_calls(oq, d, h, ba, bw, T, N, gelu, out):
     """oq_quantized_linear (x -> y, codes never in memory) is bit-identical to
     oq_quantize_act (or _gelu) followed by oq_linear: y and the norms s.  With 2- or 4-bit
-    weights, 2/4/8-bit activations, d a multiple of 1024 and N <= T the weight decode runs
-    inside K1 (also when there are fewer token pairs than SMs); the other rows take the
-    side-stream decode."""
+    weights, 2/4/8-bit activations, d a multiple of 1024 up to 5120 and N <= T the weight
+    decode runs inside K1 (also when there are fewer token pairs than SMs); the other rows take
+    the side-stream decode."""
     p = synth.sweep_projection(d, 128, 4, T) if d != 3072 or T != 4608 else \
         synth.get("flux_attn_w4a4")[0]
     x = synth.activations(p).cuda()
