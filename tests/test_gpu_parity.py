@@ -506,3 +506,26 @@ def test_quantized_linear_back_to_back_on_one_stream(oq):
     oq.oq_check()
     for y, ref in zip(ys, refs):
         assert torch.equal(y.view(torch.int32), ref.view(torch.int32))
+
+
+@pytest.mark.parametrize("d,h,ba,bw,T,N", [(256, 64, 4, 4, 64, 256), (3072, 128, 4, 4, 50, 48)])
+def test_quantized_linear_fp32_input(oq, d, h, ba, bw, T, N):
+    """fp32 x takes the in-call fallback (packed codes, then the decode prepass): y and s are
+    still bit-identical to oq_quantize_act + oq_linear, and y is within the linear bound of
+    the fp64 oracle on the same codes."""
+    g = torch.Generator().manual_seed(d + T)
+    x = torch.randn(T, d, generator=g).cuda()
+    W = (torch.randn(N, d, generator=g) / math.sqrt(d)).cuda()
+    r = oq.oq_build_rpbh(d, h, 0)
+    ca, cw = oq.oq_lloyd_max(d, ba), oq.oq_lloyd_max(d, bw)
+    wc, rn = oq.oq_quantize_weight(r, cw, W)
+    xc, s_ref = oq.oq_quantize_act(r, ca, x)
+    y_ref = oq.oq_linear(ca, cw, xc, s_ref, wc, rn)
+    s = torch.empty(T, device="cuda")
+    y = oq.oq_quantized_linear(r, ca, cw, x, wc, rn, s=s)
+    oq.oq_check()
+    assert torch.equal(s, s_ref)
+    assert torch.equal(y.view(torch.int32), y_ref.view(torch.int32))
+    ref = O.linear(xc.cpu().numpy(), s_ref.cpu().double().numpy(), wc.cpu().numpy(),
+                   rn.cpu().double().numpy(), d, ba, bw)
+    assert rel_l2(y.cpu().double().numpy(), ref) <= LINEAR_RTOL
