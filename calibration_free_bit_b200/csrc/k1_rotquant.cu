@@ -52,11 +52,15 @@ namespace {
 __device__ unsigned int g_k1_err;
 
 constexpr int kE = 32;                // rotated positions per thread (per token)
+constexpr int kSmallH = 16;           // template tag of the block sizes 2, 4, 8, 16
 constexpr int kMaxSeg = 18;           // segment slots per group for the norm reduction
 constexpr int kEntStride = kK1EntStride;   // padded entry rows (conflict-free 16 B loads)
 static_assert(kEntStride == kE + 4, "entry image layout");
 
-enum : unsigned { K1_ERR_COPY_WAIT = 1u };
+enum : unsigned {
+    K1_ERR_COPY_WAIT = 1u,        // a bulk copy of rows or tables did not complete in time
+    K1_ERR_ARMED_WAIT = 2u,       // the armed test wait (oq_debug_arm_wait_timeout) gave up
+};
 
 // Packed fp32x2 arithmetic (sm_100 FADD2/FFMA2 through the CUDA builtins).
 __device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
@@ -117,18 +121,23 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for the phase of the given parity; false after 4e9 SM cycles (about 2 s at the boost
-// clock; the caller records an error).  The first test reads no clock.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of the given parity; false after `limit` SM cycles (by default 4e9,
+// about 2 s at the boost clock; the caller records an error).  The first test reads no clock.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          long long limit = 4000000000ll) {
     if (mbar_try(bar, parity))
         return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try(bar, parity))
             return true;
-        if (clock64() - t0 > 4000000000ll)
+        if (clock64() - t0 > limit)
             return false;
     }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 // One-dimensional bulk copy global -> this CTA's shared memory, completion counted on `bar`.
@@ -239,12 +248,17 @@ __device__ __forceinline__ float gelu_erf(float x) {
 // and takes pairs from a shared counter; the kernel then reserves all 16 barriers of the SM's
 // CTA slot, so it is launched one CTA per SM.  Otherwise the CTA synchronises as a whole and
 // its groups step through the CTA's pairs in lockstep.
+// H = kSmallH stands for every block size below 32 (2, 4, 8, 16): a thread's 32 positions
+// then hold 32/h whole blocks, the butterfly stops after log2(h) in-register stages (h read
+// from p.h) and no shuffle stage runs.
 template <int BITS, bool IN_F32, int H, bool GELU = false, bool A16 = false, bool NAMED = false>
 __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     static_assert(!(GELU && IN_F32), "fused GELU is bf16-only");
     static_assert(!(NAMED && IN_F32), "named-barrier groups are bf16-only");
     static_assert(!A16 || (!IN_F32 && (BITS == 2 || BITS == 4 || BITS == 8)), "A16 output");
-    constexpr int Q = H / kE;                        // threads per h-block
+    static_assert(H >= kE || (H == kSmallH && !A16), "small blocks: one variant, codes out");
+    constexpr int Q = H >= kE ? H / kE : 1;          // threads per h-block
+    const int hrt = H >= kE ? H : p.h;               // the block size (run time below 32)
     constexpr bool REPL = (BITS <= 4);               // per-lane table copies (conflict-free)
     constexpr int TSH = REPL ? 7 : 2;                // table row stride: 32 lanes x 4 B, or 4 B
     constexpr int NW = kE * BITS / 32;               // packed code words per token per thread
@@ -291,6 +305,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     if (tid == 0) {
         for (int b = 0; b < 2 * NG + 1; ++b)
             mbar_init(smem_u32(&bars[b]), 1);
+        mbar_init(smem_u32(&bars[2 * NG + 1]), 2);   // the armed test wait's barrier
         sched[0] = NG;                               // pairs lo .. lo + NG - 1 start the groups
         sched[16] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -308,9 +323,10 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             bulk_copy(smem_u32(wdect), p.wdec_img, 4u * p.wdec_words, setup_bar);
     }
 
-    // this thread's 32 rotated positions: pos0 + e with pos0 = g * 32
-    const int blk = g / Q, r = g - blk * Q;
-    const int pos0 = blk * H + r * kE;
+    // this thread's 32 rotated positions: pos0 + e with pos0 = g * 32; r = its index inside
+    // the h-block (0 when a block fits inside one thread)
+    const int r = g % Q;
+    const int pos0 = g * kE;
     const uint4 *myent = reinterpret_cast<const uint4 *>(gent + g * kEntStride);
     const uint32_t tbl_lane =
         smem_u32(table) + (REPL ? lane * 4 : 0) - ((0x3F800000u >> p.F) << TSH);
@@ -443,6 +459,8 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
         // ---- block Walsh-Hadamard (natural order), unnormalised --------------------------
 #pragma unroll
         for (int s = 1; s < kE; s <<= 1) {
+            if (H < kE && s >= hrt)
+                break;                                 // blocks of h < 32 end here
 #pragma unroll
             for (int e = 0; e < kE; ++e) {
                 if ((e & s) == 0) {
@@ -498,8 +516,9 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             ss.x += o.x;
             ss.y += o.y;
         }
-        const float s0 = sqrtf(ss.x * (1.0f / H));
-        const float s1 = sqrtf(ss.y * (1.0f / H));
+        const float inv_h = H >= kE ? 1.0f / H : 1.0f / (float)hrt;   // exact: h = 2^k
+        const float s0 = sqrtf(ss.x * inv_h);
+        const float s1 = sqrtf(ss.y * inv_h);
         const float m0 = (s0 + p.eps > 0.f) ? p.K / (s0 + p.eps) : 0.f;
         const float m1 = (s1 + p.eps > 0.f) ? p.K / (s1 + p.eps) : 0.f;
 
@@ -611,6 +630,17 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
             }
         }
     }
+
+    // ---- armed test of the bounded waits (oq_debug_arm_wait_timeout): after all of its work,
+    // one thread waits on a barrier that expects two arrivals and gets one, gives up after
+    // p.test_wait_cycles and records it, exactly as a stalled copy's wait would.  No copy
+    // targets this barrier, so nothing is in flight when the CTA exits.
+    if (p.test_wait_cycles > 0 && blockIdx.x == 0 && tid == 0) {
+        const uint32_t tb = smem_u32(&bars[2 * NG + 1]);
+        mbar_arrive(tb);
+        if (!mbar_wait(tb, 0, p.test_wait_cycles))
+            atomicOr(&g_k1_err, K1_ERR_ARMED_WAIT);
+    }
 }
 
 // Shared-memory attributes are set once per kernel and device, and occupancy is cached per
@@ -683,6 +713,10 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
         }
     } else {
         switch (h) {
+            case 2:
+            case 4:
+            case 8:
+            case 16: return pick(k1_rotquant<BITS, F32, kSmallH, GELU, false, !F32>, k1_rotquant<BITS, F32, kSmallH, GELU>);
             case 32: return pick(k1_rotquant<BITS, F32, 32, GELU, false, !F32>, k1_rotquant<BITS, F32, 32, GELU>);
             case 64: return pick(k1_rotquant<BITS, F32, 64, GELU, false, !F32>, k1_rotquant<BITS, F32, 64, GELU>);
             case 128: return pick(k1_rotquant<BITS, F32, 128, GELU, false, !F32>, k1_rotquant<BITS, F32, 128, GELU>);

@@ -48,6 +48,7 @@ enum : unsigned {
     ERR_WAIT_FULL = 1u << 0,
     ERR_WAIT_EMPTY = 1u << 1,
     ERR_WAIT_ACCUM = 1u << 2,
+    ERR_ARMED_WAIT = 1u << 3,     // the armed test wait (oq_debug_arm_wait_timeout) gave up
 };
 
 // ------------------------------------------------------------------------------------------
@@ -65,7 +66,17 @@ struct GemmParams {
     uint32_t L0, L1, H0, H1;    // ACODES: decode8 sources of the activation codebook
     int M, N, K;
     float inv_d;
+    long long test_wait_cycles; // > 0: the armed test wait (oq_debug_arm_wait_timeout)
 };
+
+// The armed test of the bounded waits: after all of the kernel's work, one thread waits on a
+// barrier that expects two arrivals and gets one, gives up after `cycles` and records it in
+// the error word, exactly as a stalled pipeline wait would.  Nothing targets this barrier.
+__device__ __forceinline__ void armed_test_wait(uint32_t bar, long long cycles) {
+    mbar_arrive(bar);
+    if (!mbar_wait(bar, 0, cycles))
+        atomicOr(&g_k2_err, ERR_ARMED_WAIT);
+}
 
 constexpr int kEpiWarps = 4;         // warps 2..5
 constexpr int kDecWarps = 8;         // ACODES: warps 6..13, two per TMEM lane quarter
@@ -123,6 +134,7 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain_bar + 8u - base));
     float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][64]
     __shared__ int abort_flag;
+    __shared__ __align__(8) unsigned long long test_bar;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = (p.N + BN - 1) / BN;
@@ -141,6 +153,7 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
             mbar_init(tempty_bar(a), kEpiWarps);
         }
         mbar_init(drain_bar, 1);
+        mbar_init(smem_u32(&test_bar), 2);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         abort_flag = 0;
     }
@@ -346,6 +359,8 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
         }
     }
     __syncwarp();
+    if (p.test_wait_cycles > 0 && blockIdx.x == 0 && threadIdx.x == 0)
+        armed_test_wait(smem_u32(&test_bar), p.test_wait_cycles);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -404,6 +419,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain_bar + 8u - base));
     float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][64]
     __shared__ int abort_flag;
+    __shared__ __align__(8) unsigned long long test_bar;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();                      // 0: the leader
@@ -423,6 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             mbar_init(tempty_bar(a), 2 * kEpiWarps);
         }
         mbar_init(drain_bar, 1);
+        mbar_init(smem_u32(&test_bar), 2);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         abort_flag = 0;
     }
@@ -576,6 +593,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             bulk_wait_all();
     }
     __syncwarp();
+    if (p.test_wait_cycles > 0 && blockIdx.x == 0 && threadIdx.x == 0)
+        armed_test_wait(smem_u32(&test_bar), p.test_wait_cycles);
     tc_fence_before();
     cluster_sync_all();                 // no MMA, load or arrive of the pair is still pending
     if (warp == 1) {
@@ -751,9 +770,10 @@ bool gemm_pair_enabled() {
 cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
                         const uint16_t *B16, const float *s, const float *rn, void *y,
                         bool y_bf16, int T, int N, int d, cudaStream_t st, int num_sms,
-                        std::string *why) {
+                        std::string *why, long long test_wait_cycles) {
     const bool acodes = A16 == nullptr;
     GemmParams gp;
+    gp.test_wait_cycles = test_wait_cycles;
     gp.s = s;
     gp.rn = rn;
     gp.L0 = gp.L1 = gp.H0 = gp.H1 = 0;

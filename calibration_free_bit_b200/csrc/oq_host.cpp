@@ -80,6 +80,18 @@ cudaError_t timed(int kernel, cudaStream_t st, F &&launch) {
     return e;
 }
 
+// Armed test of the kernels' bounded waits (oq_debug_arm_wait_timeout): one-shot, per thread.
+thread_local int g_armed_kernel = 0;
+thread_local long long g_armed_cycles = 0;
+
+// The armed wait's limit for a launch of `kernel` (0 if not armed for it); disarms.
+long long take_armed(int kernel) {
+    if (g_armed_kernel != kernel)
+        return 0;
+    g_armed_kernel = 0;
+    return g_armed_cycles;
+}
+
 // ---------------------------------------------------------------------------------------
 // RPBH tables.  SplitMix64 (Steele, Lea & Flood 2014), Fisher-Yates (Durstenfeld) with
 // rejection-sampled bounded integers, then one sign per position from the draw's top bit.
@@ -451,6 +463,12 @@ int upload(std::mutex &mu, uint32_t **slot, const std::vector<T> &host, const ch
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// y rows are written by TMA tensor stores, whose global row stride must be a multiple of 16
+// bytes: out_features a multiple of 4 for fp32 y, of 8 for bf16 y.
+bool out_rows_aligned(int out_features, int out_dtype) {
+    return ((long long)out_features * (out_dtype == OQ_BF16 ? 2 : 4)) % 16 == 0;
+}
+
 int check_dims(int d, const char *who) {
     if (d < 128 || d > 16384 || d % 128 != 0)
         return fail(OQ_EINVAL, "%s: d = %d must be a multiple of 128 in [128, 16384]", who, d);
@@ -555,11 +573,13 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
     p.tbl_words = (int)cw->tbl_img.size();
     p.T = rows;
     p.d = d;
+    p.h = r->h;
     p.eps = eps;
     p.K = Kq;
     p.G = cb->G;
     p.F = cb->F;
     p.gelu = gelu ? 1 : 0;
+    p.test_wait_cycles = take_armed(OQ_KERNEL_QUANTIZE);
     if (a16) {
         if (!oq::k1_a16_supported(cb->bits, r->h, dtype == OQ_BF16))
             return fail(OQ_EINVAL, "%s: no fp16 centroid output for bits %d, h %d", who,
@@ -758,8 +778,8 @@ int build_rotation(int d, int h, uint64_t seed, bool permute, oq_rpbh **out, con
     *out = nullptr;
     if (check_dims(d, who) != OQ_OK)
         return OQ_EINVAL;
-    if (h < 32 || h > 1024 || (h & (h - 1)) != 0 || d % h != 0)
-        return fail(OQ_EINVAL, "%s: h = %d must be a power of two in [32, 1024] dividing "
+    if (h < 2 || h > 1024 || (h & (h - 1)) != 0 || d % h != 0)
+        return fail(OQ_EINVAL, "%s: h = %d must be a power of two in [2, 1024] dividing "
                                "d = %d", who, h, d);
     oq_rpbh *r = new (std::nothrow) oq_rpbh;
     if (!r)
@@ -959,9 +979,10 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
                     cw->d);
     if (out_dtype != OQ_F32 && out_dtype != OQ_BF16)
         return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32 or OQ_BF16", who);
-    if (T < 0 || out_features < 1 || out_features % 16 != 0)
-        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
-                               "multiple of 16", who, T, out_features);
+    if (T < 0 || out_features < 1 || !out_rows_aligned(out_features, out_dtype))
+        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d positive with "
+                               "16-byte rows of y (a multiple of 4 for fp32, 8 for bf16)", who,
+                    T, out_features);
     if (T == 0)
         return OQ_OK;
     if (!x_codes || !s || !W_codes || !row_norms || !y)
@@ -1007,7 +1028,8 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     if (e == cudaSuccess)
         e = timed(OQ_KERNEL_GEMM, st, [&] {
             return oq::launch_gemm(A16, x_codes, ca->lut, B16, s, row_norms, y,
-                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why);
+                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
+                                   take_armed(OQ_KERNEL_GEMM));
         });
     cudaError_t e2 = cudaFreeAsync(ws, st);
     if (e != cudaSuccess)
@@ -1030,9 +1052,10 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
                     cw->d);
     if (out_dtype != OQ_F32 && out_dtype != OQ_BF16)
         return fail(OQ_EINVAL, "%s: out_dtype must be OQ_F32 or OQ_BF16", who);
-    if (T < 0 || out_features < 1 || out_features % 16 != 0)
-        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
-                               "multiple of 16", who, T, out_features);
+    if (T < 0 || out_features < 1 || !out_rows_aligned(out_features, out_dtype))
+        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d positive with "
+                               "16-byte rows of y (a multiple of 4 for fp32, 8 for bf16)", who,
+                    T, out_features);
     const size_t need = oq::linear_workspace_bytes(T, d, out_features);
     const size_t have = oq::noalloc_workspace_bytes();
     if (need > have)
@@ -1062,13 +1085,20 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
     uint16_t *B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
                                                  oq::linear_workspace_b_offset(T, d));
     std::string why;
-    e = oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
+    e = timed(OQ_KERNEL_DECODE, st, [&] {
+        return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
+    });
     if (e == cudaSuccess)
-        e = oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st, di->sms,
-                              &why);
+        e = timed(OQ_KERNEL_DECODE, st, [&] {
+            return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
+                                     di->sms, &why);
+        });
     if (e == cudaSuccess)
-        e = oq::launch_gemm(A16, nullptr, nullptr, B16, s, row_norms, y, out_dtype == OQ_BF16, T,
-                            out_features, d, st, di->sms, &why);
+        e = timed(OQ_KERNEL_GEMM, st, [&] {
+            return oq::launch_gemm(A16, nullptr, nullptr, B16, s, row_norms, y,
+                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
+                                   take_armed(OQ_KERNEL_GEMM));
+        });
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());
     return OQ_OK;
@@ -1095,9 +1125,10 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     const bool gelu = (flags & OQ_FORWARD_GELU) != 0;
     if (gelu && dtype != OQ_BF16)
         return fail(OQ_EINVAL, "%s: OQ_FORWARD_GELU takes bf16 input", who);
-    if (T < 0 || out_features < 1 || out_features % 16 != 0)
-        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d a positive "
-                               "multiple of 16", who, T, out_features);
+    if (T < 0 || out_features < 1 || !out_rows_aligned(out_features, out_dtype))
+        return fail(OQ_EINVAL, "%s: T = %d must be >= 0 and out_features = %d positive with "
+                               "16-byte rows of y (a multiple of 4 for fp32, 8 for bf16)", who,
+                    T, out_features);
     if (T == 0)
         return OQ_OK;
     if (!x || !W_codes || !row_norms || !y)
@@ -1158,7 +1189,7 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
             e = timed(OQ_KERNEL_GEMM, st, [&] {
                 return oq::launch_gemm(A16, nullptr, nullptr, B16, sv, row_norms, y,
                                        out_dtype == OQ_BF16, T, out_features, d, st, di->sms,
-                                       &why);
+                                       &why, take_armed(OQ_KERNEL_GEMM));
             });
             if (e != cudaSuccess)
                 rc = fail_cuda(e, why.c_str());
@@ -1203,7 +1234,8 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     if (rc == OQ_OK && e == cudaSuccess) {
         e = timed(OQ_KERNEL_GEMM, st, [&] {
             return oq::launch_gemm(A16, nullptr, nullptr, B16, sv, row_norms, y,
-                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why);
+                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
+                                   take_armed(OQ_KERNEL_GEMM));
         });
         if (e != cudaSuccess)
             rc = fail_cuda(e, why.c_str());
@@ -1232,9 +1264,10 @@ int oq_check(void *stream) {
         return fail_cuda(e, "oq_check: read k2 error word");
     if (w1 || w2 || w3)
         return fail(OQ_EDEVICE, "device error word: quantize=0x%x quantize_tc=0x%x linear=0x%x "
-                                "(a bounded wait gave up; quantize bit 1 = row copy; quantize_tc "
-                                "bits 1/2/4/8/16 = staging/operand ring/accumulator/norm/code "
-                                "tile; linear bits 1/2/4 = operand stage/ring slot/accumulator)",
+                                "(a bounded wait gave up; quantize bits 1/2 = row copy/armed test "
+                                "wait; quantize_tc bits 1/2/4/8/16 = staging/operand "
+                                "ring/accumulator/norm/code tile; linear bits 1/2/4/8 = operand "
+                                "stage/ring slot/accumulator/armed test wait)",
                     w1, w3, w2);
     return OQ_OK;
 }
@@ -1278,6 +1311,22 @@ void oq_free_codebook(oq_codebook *cb) {
     if (cur >= 0)
         cudaSetDevice(cur);
     delete cb;
+}
+
+int oq_debug_arm_wait_timeout(int kernel, long long limit_cycles) {
+    if (kernel == 0) {
+        g_armed_kernel = 0;
+        return OQ_OK;
+    }
+    if (kernel != OQ_KERNEL_QUANTIZE && kernel != OQ_KERNEL_GEMM)
+        return fail(OQ_EINVAL, "oq_debug_arm_wait_timeout: kernel = %d (OQ_KERNEL_QUANTIZE or "
+                               "OQ_KERNEL_GEMM, or 0 to disarm)", kernel);
+    if (limit_cycles < 1000 || limit_cycles > 1000000000LL)
+        return fail(OQ_EINVAL, "oq_debug_arm_wait_timeout: limit_cycles = %lld not in "
+                               "[1e3, 1e9]", limit_cycles);
+    g_armed_kernel = kernel;
+    g_armed_cycles = limit_cycles;
+    return OQ_OK;
 }
 
 int oq_timing_enable(int on) {

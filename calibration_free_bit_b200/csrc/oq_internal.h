@@ -69,6 +69,7 @@ struct K1Params {
     const uint32_t *tbl_img;   // quantizer-table image (see above)
     int ent_words, tbl_words;  // image sizes in 32-bit words (multiples of 4)
     int T, d;
+    int h;                  // Hadamard block size (read by the kernel only when h < 32)
     float eps;              // added to the norm before division (0 for weights)
     float K;                // sqrt(d/h) / (G * delta): z_unnormalised * K / (s+eps) = u/(G delta)
     int G, F;               // grid cells (power of two), F = 23 - log2(G)
@@ -91,10 +92,11 @@ struct K1Params {
     uint32_t wdec_src[4];         // 4-bit: byte-permute decode sources of the weight codebook
     const uint32_t *wdec_img;     // 2-bit: byte -> four fp16 centroids (256 x 8 bytes)
     int wdec_words;               // its size in words (0 for 4-bit)
+    long long test_wait_cycles;   // > 0: the armed test wait (oq_debug_arm_wait_timeout)
 };
 // True when K1 can write fp16 centroids itself (launch_k1 with p.a16 set).
 inline bool k1_a16_supported(int bits, int h, bool bf16_in) {
-    return bf16_in && h <= 256 && (bits == 2 || bits == 4 || bits == 8);
+    return bf16_in && h >= 32 && h <= 256 && (bits == 2 || bits == 4 || bits == 8);
 }
 // True when K1 runs as one CTA per SM with named-barrier groups (bf16 rows, d/32 threads per
 // token pair a whole number of warps); the fused weight decode needs it.
@@ -136,10 +138,11 @@ cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long lo
 // A is A16 (fp16 centroids from the prepass) or, when A16 is null, x_codes4: 4-bit codes of
 // the codebook whose fp16 LUT is lut_a (must be odd-symmetric), decoded inside the kernel.
 // y is fp32, or bf16 (round to nearest even of the fp32 epilogue value) when y_bf16.
+// test_wait_cycles > 0 arms the kernel's test of its bounded waits (oq_debug_arm_wait_timeout).
 cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
                         const uint16_t *B16, const float *s, const float *rn, void *y,
                         bool y_bf16, int T, int N, int d, cudaStream_t st, int num_sms,
-                        std::string *why);
+                        std::string *why, long long test_wait_cycles = 0);
 
 // Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
 // its size, and its address on the current device (looked up once per device).

@@ -55,16 +55,18 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for the phase with the given parity to complete; false after kWaitLimitCycles.  The
-// first test costs no clock read (most waits in a running pipeline are already satisfied).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete; false after `limit` SM cycles
+// (kWaitLimitCycles by default).  The first test costs no clock read (most waits in a running
+// pipeline are already satisfied).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          long long limit = kWaitLimitCycles) {
     if (mbar_try(bar, parity))
         return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try(bar, parity))
             return true;
-        if (clock64() - t0 > kWaitLimitCycles)
+        if (clock64() - t0 > limit)
             return false;
     }
 }

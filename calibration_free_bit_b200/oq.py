@@ -63,6 +63,7 @@ def lib():
     L.oq_free_rpbh.restype = None
     L.oq_free_codebook.argtypes = [vp]
     L.oq_free_codebook.restype = None
+    L.oq_debug_arm_wait_timeout.argtypes = [i32, C.c_longlong]
     L.oq_timing_enable.argtypes = [i32]
     L.oq_timing_collect.argtypes = [vp, i32, C.POINTER(i32)]
     L.oq_last_error.restype = C.c_char_p
@@ -71,7 +72,8 @@ def lib():
                  "oq_codebook_values",
                  "oq_codebook_grid", "oq_quantize_weight", "oq_quantize_act",
                  "oq_quantize_act_gelu", "oq_linear", "oq_quantized_linear",
-                 "oq_linear_noalloc", "oq_check", "oq_timing_enable", "oq_timing_collect"):
+                 "oq_linear_noalloc", "oq_check", "oq_timing_enable", "oq_timing_collect",
+                 "oq_debug_arm_wait_timeout"):
         getattr(L, name).restype = i32
     _lib = L
     return L
@@ -274,6 +276,13 @@ def oq_check(stream=None):
 
 
 KERNEL_NAMES = {1: "quantize", 2: "decode", 3: "gemm"}
+OQ_KERNEL_QUANTIZE, OQ_KERNEL_DECODE, OQ_KERNEL_GEMM = 1, 2, 3
+
+
+def oq_debug_arm_wait_timeout(kernel: int, limit_cycles: int):
+    """Arm the one-shot test of the bounded waits for this thread's next launch of `kernel`
+    (OQ_KERNEL_QUANTIZE or OQ_KERNEL_GEMM; 0 disarms); see include/oq.h."""
+    _check(lib().oq_debug_arm_wait_timeout(kernel, limit_cycles))
 
 
 class _TimingRecord(C.Structure):

@@ -21,9 +21,19 @@
  *     streams and threads, and are freed with oq_free_*.  Their first use on a device copies
  *     small tables to that device synchronously; make that first use outside any CUDA graph
  *     capture.
+ *   - The library keeps per-device state (uploaded tables, its memory pool, side stream and
+ *     events, the device address of its fixed workspace).  cudaDeviceReset() on a device the
+ *     library has used invalidates that state: do not call the library on that device (or
+ *     free handles used there) after resetting it.
  *   - Sizes: d is a multiple of 128 and of h, 128 <= d <= 16384; h is a power of two,
- *     32 <= h <= 1024; bits in {2, 3, 4, 6, 8}; 0 <= T < 2^31 rows (T = 0 is a no-op returning
- *     OQ_OK); the linear layer also needs 1 <= out_features < 2^31.
+ *     2 <= h <= 1024; bits in {2, 3, 4, 6, 8}; 0 <= T < 2^31 rows (T = 0 is a no-op returning
+ *     OQ_OK); the linear layer also needs 1 <= out_features < 2^31 with rows of y a
+ *     multiple of 16 bytes (out_features a multiple of 4 for fp32 y, of 8 for bf16 y).
+ *     Why these limits: a row of 3-bit codes is d*3/8 bytes, a multiple of 16 (the alignment
+ *     of the 128-bit stores and TMA copies of code rows) only when d is a multiple of 128;
+ *     the quantizer stages a token pair in shared memory (8*d bytes for bf16 rows, 128 KB at
+ *     d = 16384); y is written by TMA tensor stores, whose row stride must be a multiple of
+ *     16 bytes.
  *   - Packed codes: row-major, one row per token (or weight row), row stride d*bits/8 bytes,
  *     element k of a row in bits [k*bits, k*bits + bits) of the row's byte stream, bit i of
  *     the stream being bit (i mod 8) of byte i/8 (LSB first).  Code 0 is the most negative
@@ -123,7 +133,7 @@ int oq_quantize_weight(const oq_rpbh *r, const oq_codebook *cw, const void *W, i
  * A code is the number of sigma-scaled boundaries <= x_rot/(s+eps) (ties go up), decided in
  * fp32.  An all-zero row gives codes 2^ba/2 and s = 0.  The rotation runs as register
  * butterflies on the CUDA cores; with the environment variable OQ_K1_PATH=tc (read once per
- * process) bf16 rows with h <= 256 and d up to about 3.9K use a kernel that runs the block
+ * process) bf16 rows with 32 <= h <= 256 and d up to about 3.9K use a kernel that runs the block
  * transform as tcgen05 MMAs instead (same results under the same parity rules).
  * Errors: as oq_quantize_weight. */
 int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype, int T,
@@ -166,7 +176,7 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * ([RCAP] pseudocode, online part, and rotation-cancellation paragraph), i.e. the result of
  * oq_quantize_act followed by oq_linear, without materialising x_codes: the rotate+quantize
  * kernel writes each code's fp16 unit centroid straight into the GEMM's A operand (bf16 x,
- * ba in {2, 4, 8}, h <= 256; otherwise codes and the decode prepass are used inside the
+ * ba in {2, 4, 8}, 32 <= h <= 256; otherwise codes and the decode prepass are used inside the
  * call).  With 2- or 4-bit weight codes, d a multiple of 1024 up to 5120, bf16 x and
  * out_features <= T, that kernel also decodes the weight codes into the GEMM's B operand once
  * it runs out of tokens; otherwise the weight codes are decoded on a library-owned side
@@ -186,8 +196,11 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
                         int flags, void *stream);
 
 /* oq_linear for callers that cannot allocate device memory.  The paper has no counterpart;
- * this is a deployment variant of the same computation, with the same arguments, result and
- * errors as oq_linear.
+ * this is a deployment variant of the same computation, with the same arguments and errors as
+ * oq_linear.  It always runs the decode prepass into fp16 operands followed by the GEMM (the
+ * default form of oq_linear, bit-identical to it); it ignores OQ_LINEAR_PATH, so in a process
+ * that set OQ_LINEAR_PATH=fused the two calls may differ in the last bits (both are within the
+ * linear layer's parity bound).  oq_timing_* records its kernels like oq_linear's.
  * Who needs it: code that runs inside a host framework which owns all device memory and gives
  * plug-ins no allocator (a side cudaMalloc would bypass its accounting or fail under its
  * memory cap), and latency-critical serving loops that forbid allocation on the request path
@@ -208,6 +221,20 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
 int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_codes,
                       const float *s, const uint8_t *W_codes, const float *row_norms, int T,
                       int d, int out_features, void *y, int out_dtype, void *stream);
+
+/* Test of failure detection (the pages have no counterpart; this checks the library's own
+ * error path).  Every wait inside liboq's kernels is bounded: a wait that runs out records a
+ * bit in a device error word and the kernel returns instead of hanging.  This call arms, for
+ * the calling thread, a one-shot test of that path: the next launch of `kernel` made by this
+ * thread (OQ_KERNEL_QUANTIZE: the CUDA-core rotate+quantize kernel; OQ_KERNEL_GEMM: either
+ * GEMM form) does all of its normal work, then one of its threads waits on a shared-memory
+ * barrier that nothing completes, gives up after `limit_cycles` SM clock cycles and records
+ * the timeout (quantize bit 2, linear bit 8) before returning normally.  oq_check() then
+ * returns OQ_EDEVICE and names the bit; the outputs are those of an unarmed call and the
+ * context stays usable.  No fault, trap or unbounded wait is involved.
+ * kernel = 0 disarms.  Errors: OQ_EINVAL for another kernel id or limit_cycles outside
+ * [1e3, 1e9]. */
+int oq_debug_arm_wait_timeout(int kernel, long long limit_cycles);
 
 /* Synchronise `stream`, then read and clear the library's device error word.
  * Returns OQ_OK, OQ_EDEVICE (a kernel gave up a bounded wait or saw an internal

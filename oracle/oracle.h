@@ -18,7 +18,7 @@
  *     norms and nearest-centroid codes per weight matrix; x_rot, s = norm(x_rot) and
  *     nearest-centroid codes of x_rot/(s+eps) per token.
  *
- * Readings where the page is silent (each listed in the design doc):
+ * Readings where the page is silent:
  *   RNG = SplitMix64; permutation = Fisher-Yates (Durstenfeld) with rejection-sampled
  *   bounded integers; sign[k] = top bit of the next draw, drawn after the permutation;
  *   gather semantics y[i] = x[perm[i]]; signs applied after the permutation and before the

@@ -102,7 +102,8 @@ def test_quantized_linear_validation_without_a_gpu():
     assert call(args(flags=4)) == oq.OQ_EINVAL                        # unknown flag
     assert call(args(flags=1, dtype=oq.OQ_F32)) == oq.OQ_EINVAL       # GELU needs bf16
     assert call(args(cw=c_other.handle)) == oq.OQ_EINVAL              # d mismatch
-    assert call(args(N=100)) == oq.OQ_EINVAL                          # N not a multiple of 16
+    assert call(args(N=102)) == oq.OQ_EINVAL                          # fp32 rows not 16 B
+    assert call(args(N=100, od=oq.OQ_BF16)) == oq.OQ_EINVAL           # bf16 rows not 16 B
     assert call(args(x=fake + 4)) == oq.OQ_EINVAL                     # misaligned x
     assert call(args(s=fake + 2)) == oq.OQ_EINVAL                     # misaligned s
     assert call(args(T=0, x=None, wc=None, rn=None, y=None)) == oq.OQ_OK
@@ -157,7 +158,6 @@ def test_validation_rejects_bad_arguments_without_a_gpu():
     assert L.oq_build_rpbh(100, 64, 0, C.byref(h)) == oq.OQ_EINVAL
     assert L.oq_build_rpbh(3072, 48, 0, C.byref(h)) == oq.OQ_EINVAL
     assert L.oq_build_rpbh(3072, 2048, 0, C.byref(h)) == oq.OQ_EINVAL
-    assert L.oq_build_rpbh(3072, 16, 0, C.byref(h)) == oq.OQ_EINVAL
     assert L.oq_build_rpbh(32768, 128, 0, C.byref(h)) == oq.OQ_EINVAL
     assert L.oq_lloyd_max(3072, 5, C.byref(h)) == oq.OQ_EINVAL
     assert b"bits" in L.oq_last_error()
@@ -180,8 +180,8 @@ def test_validation_rejects_bad_arguments_without_a_gpu():
     # T = 0 is a no-op that succeeds without touching a device
     assert L.oq_quantize_act(r.handle, ca.handle, None, oq.OQ_BF16, 0, 3072, None, None,
                              None) == oq.OQ_OK
-    # linear: out_features not a multiple of 16, unknown output type, d mismatch
-    assert L.oq_linear(ca.handle, ca.handle, fake, fake, fake, fake, 8, 3072, 100, fake,
+    # linear: rows of y not a multiple of 16 bytes, unknown output type, d mismatch
+    assert L.oq_linear(ca.handle, ca.handle, fake, fake, fake, fake, 8, 3072, 102, fake,
                        oq.OQ_F32, None) == oq.OQ_EINVAL
     assert L.oq_linear(ca.handle, ca.handle, fake, fake, fake, fake, 8, 3072, 128, fake,
                        2, None) == oq.OQ_EINVAL
@@ -192,3 +192,52 @@ def test_validation_rejects_bad_arguments_without_a_gpu():
                        oq.OQ_F32, None) == oq.OQ_EINVAL
     assert L.oq_linear(ca.handle, ca.handle, None, None, None, None, 0, 3072, 128, None,
                        oq.OQ_F32, None) == oq.OQ_OK
+
+
+@pytest.mark.parametrize("d,h,ok", [
+    (3072, 2, True), (3072, 4, True), (3072, 8, True), (3072, 16, True), (3072, 1024, True),
+    (128, 128, True), (16384, 1024, True),
+    (3072, 1, False),      # h below 2
+    (3072, 2048, False),   # h above 1024
+    (3072, 48, False),     # h not a power of two
+    (3072, 12, False),
+    (2048, 4096, False),   # h larger than d
+    (1536, 1024, False),   # h does not divide d
+    (100, 4, False),       # d not a multiple of 128 (3-bit code rows would not be 16-byte)
+    (3008, 64, False),
+    (64, 64, False),       # d below 128
+    (16512, 128, False),   # d above 16384 (a bf16 token pair no longer fits shared memory)
+])
+def test_size_limits_of_the_rotation(d, h, ok):
+    """Each size limit of oq_build_rpbh / oq_build_block_rht, accepted or refused with
+    OQ_EINVAL before anything touches a device."""
+    L = oq.lib()
+    for build in (L.oq_build_rpbh, L.oq_build_block_rht):
+        hd = C.c_void_p()
+        rc = build(d, h, 0, C.byref(hd))
+        assert rc == (oq.OQ_OK if ok else oq.OQ_EINVAL), (d, h, L.oq_last_error())
+        if ok:
+            L.oq_free_rpbh(hd)
+
+
+@pytest.mark.parametrize("N,out_dtype,ok", [
+    (4, oq.OQ_F32, True), (20, oq.OQ_F32, True), (3072, oq.OQ_F32, True),
+    (8, oq.OQ_BF16, True), (24, oq.OQ_BF16, True),
+    (2, oq.OQ_F32, False), (102, oq.OQ_F32, False),      # fp32 rows of y not 16-byte
+    (4, oq.OQ_BF16, False), (20, oq.OQ_BF16, False),     # bf16 rows of y not 16-byte
+    (0, oq.OQ_F32, False), (-16, oq.OQ_F32, False),
+])
+def test_output_row_rule_of_the_linear_calls(N, out_dtype, ok):
+    """out_features must give 16-byte rows of y (the TMA store's row-stride rule), checked by
+    oq_linear, oq_linear_noalloc and oq_quantized_linear alike.  Calls with T = 0 stop after
+    validation, so no device is needed."""
+    L = oq.lib()
+    r = oq.oq_build_rpbh(1024, 128)
+    ca = oq.oq_lloyd_max(1024, 4)
+    want = oq.OQ_OK if ok else oq.OQ_EINVAL
+    assert L.oq_linear(ca.handle, ca.handle, None, None, None, None, 0, 1024, N, None,
+                       out_dtype, None) == want
+    assert L.oq_linear_noalloc(ca.handle, ca.handle, None, None, None, None, 0, 1024, N, None,
+                               out_dtype, None) == want
+    assert L.oq_quantized_linear(r.handle, ca.handle, ca.handle, None, oq.OQ_BF16, None, None,
+                                 0, 1024, N, None, out_dtype, None, 0, None) == want
