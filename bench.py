@@ -15,6 +15,7 @@ is bracketed by a barrier + synchronize, and the max over ranks is reported.
 Rank 0 prints one JSON line on stdout; everything else goes to stderr.
 """
 import argparse
+import csv
 import datetime
 import hashlib
 import json
@@ -83,23 +84,48 @@ def source_sha(rels):
 
 
 GEMM_SOURCES = ("calibration_free_bit_b200/csrc/k2_linear.cu",
-                "calibration_free_bit_b200/csrc/sm100_common.cuh")
+                "calibration_free_bit_b200/csrc/sm100_common.cuh",
+                "calibration_free_bit_b200/csrc/decode4.cuh")
+K1_SOURCES = ("calibration_free_bit_b200/csrc/k1_rotquant.cu",
+              "calibration_free_bit_b200/csrc/decode4.cuh")
 
 
 def profile_traffic(profile_name, kernel_src):
-    """DRAM bytes per launch from a committed ncu summary, or None if absent or stale (the
-    summary records the hash of the kernel sources it was captured from)."""
+    """DRAM bytes per launch of a kernel from a committed ncu export, or None if absent or
+    stale.  The file is `ncu --csv --page raw` output (one row per captured launch, columns
+    dram__bytes_read.sum and dram__bytes_write.sum in bytes) after comment lines written by the
+    capture command, one of which records the SHA-256 (first 16 hex digits) of the kernel's
+    sources at capture time: a capture of other sources is not used."""
     path = os.path.join(ROOT, "profiles", profile_name)
     if not os.path.exists(path):
         return None, "no profile"
-    text = open(path).read()
-    m = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
-    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not h:
-        return None, "profile lacks traffic"
-    if h.group(1) != source_sha(kernel_src):
+    lines = open(path).read().splitlines()
+    sha = None
+    for ln in lines:
+        m = re.match(r"#\s*sources_sha256_16:\s*([0-9a-f]{16})", ln)
+        if m:
+            sha = m.group(1)
+    if sha is None:
+        return None, "profile lacks the sources hash"
+    if sha != source_sha(kernel_src):
         return None, "kernel changed since capture"
-    return float(m.group(1)), "ncu"
+    rows = list(csv.reader([ln for ln in lines if ln and not ln.startswith("#")]))
+    if len(rows) < 2:
+        return None, "profile has no launch rows"
+    head = rows[0]
+    try:
+        ir, iw = head.index("dram__bytes_read.sum"), head.index("dram__bytes_write.sum")
+    except ValueError:
+        return None, "profile lacks DRAM byte counters"
+    vals = []
+    for r_ in rows[1:]:
+        try:
+            vals.append(float(r_[ir]) + float(r_[iw]))
+        except (ValueError, IndexError):
+            continue                               # the units row of the raw page
+    if not vals:
+        return None, "profile has no numeric rows"
+    return statistics.mean(vals), "ncu (profiles/" + profile_name + ")"
 
 
 class ClockSampler:
@@ -178,19 +204,40 @@ class OracleStep:
         self.x = synth.activations(p, rows=np.arange(min(p.T, 2048))).double().numpy()
         self.cursor = 0
 
-    def run(self, S):
-        rows = (self.cursor + np.arange(S)) % len(self.x)
-        self.cursor = int(rows[-1] + 1)
-        t0 = time.perf_counter()
-        xc, s = self.O.quantize_act(self.x[rows], self.p.h, self.perm, self.sign, self.p.bits_a,
+    def _rows(self, xr):
+        xc, s = self.O.quantize_act(xr, self.p.h, self.perm, self.sign, self.p.bits_a,
                                     marginal=self.marginal, gelu_input=self.p.fused_gelu)
         self.O.linear(xc, s, self.wc, self.rn, self.p.d, self.p.bits_a, self.p.bits_w,
                       marginal=self.marginal)
+
+    def run(self, S, threads=1):
+        """Seconds for S tokens; threads > 1 splits the tokens into one chunk per host thread
+        (the oracle's C calls release the GIL, so the chunks run in parallel)."""
+        rows = (self.cursor + np.arange(S)) % len(self.x)
+        self.cursor = int(rows[-1] + 1)
+        xr = self.x[rows]
+        self.O.codebook(self.p.bits_a, self.marginal, self.p.d)   # cached before timing
+        self.O.codebook(self.p.bits_w, self.marginal, self.p.d)
+        t0 = time.perf_counter()
+        if threads <= 1:
+            self._rows(xr)
+        else:
+            import concurrent.futures as cf
+            parts = np.array_split(np.arange(S), threads)
+            with cf.ThreadPoolExecutor(threads) as ex:
+                list(ex.map(lambda ix: self._rows(xr[ix]), [q for q in parts if len(q)]))
         return time.perf_counter() - t0
 
 
 def cores_used():
     return 1   # the oracle is single-threaded C
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def run_reference(args, p):
@@ -224,9 +271,18 @@ def cpu_baseline(p):
     per_tok = step.run(8) / 8
     S = int(max(8, min(1024, 15.0 / max(per_tok, 1e-9))))
     t = step.run(S)
-    return {"value": S / t, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
-            "sample": f"{S} tokens of {p.name}: fp64 rotate+quantize then all {p.out} outputs "
-                      f"(naive loop), {t:.1f} s on one host core"}
+    out = {"value": S / t, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+           "sample": f"{S} tokens of {p.name}: fp64 rotate+quantize then all {p.out} outputs "
+                     f"(naive loop), {t:.1f} s on one host core"}
+    # the same oracle over token chunks on every host core, reported separately
+    n = host_cores()
+    if n > 1:
+        Sn = int(max(8 * n, min(8192, 10.0 * n / max(per_tok, 1e-9))))
+        tn = step.run(Sn, threads=n)
+        out["threads"] = {"value": Sn / tn, "unit": "tokens/s", "cores": n,
+                          "sample": f"{Sn} tokens in {n} chunks on {n} host threads, "
+                                    f"{tn:.1f} s"}
+    return out
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -370,8 +426,12 @@ def run_ours(args, p, rank, world, dev):
     ms_max = max_over_ranks(g0.elapsed_time(g1), world, dev)
     # the quantizer writes the fp16 operand itself on the forward path with 2/4/8-bit
     # activations, bf16 x and h <= 256 (and, for 4-bit weights, decodes the weights too)
-    direct = (args.api == "forward" and p.bits_a in (2, 4, 8) and p.dtype == torch.bfloat16
-              and p.h <= 256)
+    # with OQ_LINEAR_PATH=fused and 4-bit activations the quantizer writes packed codes and the
+    # GEMM decodes them in shared memory
+    acodes = (os.environ.get("OQ_LINEAR_PATH") == "fused" and p.bits_a == 4
+              and p.dtype == torch.bfloat16)
+    direct = (args.api == "forward" and not acodes and p.bits_a in (2, 4, 8)
+              and p.dtype == torch.bfloat16 and 32 <= p.h <= 256)
     launches = launches_per_step * args.steps
     del graphs
 
@@ -440,7 +500,8 @@ def run_ours(args, p, rank, world, dev):
     dec_ms = statistics.mean(per_kernel["decode"]) if "decode" in per_kernel else None
     flops = 2.0 * p.T * p.d * p.out
     gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
-    traffic, traffic_src = profile_traffic(f"k2_gemm_{p.name}.md", GEMM_SOURCES)
+    traffic, traffic_src = profile_traffic(
+        f"k2_gemm_{'acodes_' if acodes else ''}{p.name}.ncu.csv", GEMM_SOURCES)
     in_bytes = 2 if p.dtype == torch.bfloat16 else 4
     # K1's algorithmic bytes are the method's: x in, the packed codes and s out, T (in*d +
     # d*ba/8 + 4).  What this design moves besides (the fp16 centroids K1 writes for the GEMM
@@ -450,10 +511,12 @@ def run_ours(args, p, rank, world, dev):
     design_bytes = p.T * (in_bytes * p.d + (2 * p.d if direct else p.d * p.bits_a // 8) + 4)
     # with 2/4-bit weights the one-call path's K1 also decodes the weight codes (no decode
     # launch)
-    fused_dec = direct and dec_ms is None
+    fused_dec = args.api == "forward" and (direct or acodes) and dec_ms is None
     if fused_dec:
         design_bytes += p.out * p.d * (p.bits_w / 8 + 2)
     q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9
+    q_traffic, q_traffic_src = profile_traffic(
+        f"k1_rotquant_{'codes_' if acodes else ''}{p.name}.ncu.csv", K1_SOURCES)
     out = {
         "metric": METRIC,
         "value": whole_job_rate(world, p.T, args.steps, ms_max),
@@ -467,9 +530,13 @@ def run_ours(args, p, rank, world, dev):
         "api": ("oq_quantized_linear (one call; x_codes stay on chip)" if args.api == "forward"
                 else "oq_quantize_act + oq_linear"),
         "kernels_ms_mean": {"quantize": quant_ms, "decode": dec_ms, "gemm": gemm_ms},
+        "gemm_a_operand": ("4-bit codes, decoded in the GEMM's shared memory" if acodes else
+                           "fp16 centroids written by the quantizer" if direct else
+                           "fp16 centroids from the decode prepass"),
         "roofline": {
             "kernel": ("k2_gemm_pair (tcgen05 cta_group::2 kind::f16, 256x256x64 tiles per "
-                       "CTA pair)"),
+                       "CTA pair" + (", 4-bit A codes decoded in shared memory)" if acodes
+                                    else ")")),
             "bound": "tensor", "achieved": gemm_tf,
             "peak": pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
             "peak_note": f"{pk_kind} dense bf16 burst (fp16 kind::f16 runs at the bf16 rate)",
@@ -483,8 +550,8 @@ def run_ours(args, p, rank, world, dev):
             "algorithmic_per_launch": flops,
         },
         "roofline_quantize": {
-            "kernel": ("k1_rotquant (fp16-operand output + fused weight decode)" if fused_dec
-                       else "k1_rotquant (fp16-operand output)" if direct else "k1_rotquant"),
+            "kernel": "k1_rotquant (" + ("fp16-operand output" if direct else "codes output")
+                      + (" + fused weight decode)" if fused_dec else ")"),
             "bound": "hbm", "achieved": q_gbs,
             "peak": pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]), "unit": "GB/s",
             "frac": q_gbs / pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
@@ -493,6 +560,7 @@ def run_ours(args, p, rank, world, dev):
             "algorithmic_bytes_rule": "T * (in_bytes*d + d*bits_a/8 + 4): x in, codes and s out",
             "design_bytes_per_launch": design_bytes,
             "design_gbs": design_bytes / (quant_ms * 1e-3) / 1e9,
+            "traffic": q_traffic, "traffic_source": q_traffic_src,
         },
         "gpu_launches": launches,
         "timing": f"value/ms_per_step: {timing_mode} of the step; kernels_ms_mean and the "
@@ -540,17 +608,26 @@ def run_sweep(args, dev):
         for i in range(max(3, min(args.warmup, 5))):
             oq.oq_quantize_act(r, ca, xs[i % nb], codes, s)
         torch.cuda.synchronize()
+        # the n launches are captured once in a CUDA graph and replayed, so the time is the
+        # device's (back-to-back launches), not the host's call rate
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                oq.oq_quantize_act(r, ca, xs[i % nb], codes, s)
+        g.replay()
+        torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for i in range(n):
-            oq.oq_quantize_act(r, ca, xs[i % nb], codes, s)
+        g.replay()
         e1.record()
         torch.cuda.synchronize()
         oq.oq_check()
+        del g
         us = e0.elapsed_time(e1) / n * 1e3
         byts = T * (2 * d + d * bits // 8 + 4)
         gbs = byts / (us * 1e-6) / 1e9
         row = {"d": d, "h": h, "bits_a": bits, "T": T, "k1_us": round(us, 3),
+               "timing": f"CUDA-graph replay of {n} back-to-back launches",
                "gbs": round(gbs, 1), "frac": round(gbs / hbm, 4), "tokens_per_s": T / (us * 1e-6)}
         rows_out.append(row)
         print(json.dumps(row), flush=True)

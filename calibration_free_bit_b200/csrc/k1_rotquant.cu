@@ -235,9 +235,11 @@ __device__ __forceinline__ void decode_store(const uint32_t *dect, const uint32_
 // the NEXT round's two rows stream into a raw buffer while the current round computes from
 // the interleaved pair buffer.  fp32 input: rows are gathered straight from `stages` raw
 // buffers (2 when shared memory allows, else 1).
-// GELU in its erf form, x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2, in fp32 (CUDA's erff).
+// GELU in its exact (erf) form, x * Phi(x), in fp32, with Phi(x) = erfc(-x / sqrt 2) / 2
+// (CUDA's erfcf): no cancellation of 1 + erf(x / sqrt 2) for negative x, so the left tail
+// keeps its relative accuracy (the erf form loses it below about x = -4).
 __device__ __forceinline__ float gelu_erf(float x) {
-    return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+    return 0.5f * x * erfcf(x * -0.70710678118654752f);
 }
 
 // GELU (bf16 input only): the kernel quantizes R * GELU(x) instead of R * x; GELU is applied
@@ -587,7 +589,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
         my = nxt;
     }
 
-    if constexpr (NAMED && A16) {
+    if constexpr (NAMED) {
         // ---- fused weight decode: this CTA's share of the code words, in chunks of GT * 8 ---
         if (p.wdec_groups > 0) {
             const long long dlo = (long long)blockIdx.x * p.wdec_groups / gridDim.x;
@@ -753,8 +755,8 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     long long ctas_needed;
     int NG;
     const bool named = GT % 32 == 0 && !in_f32;
-    if (p.wdec_groups > 0 && !(named && p.a16)) {
-        *why = "fused weight decode needs fp16 output and whole-warp groups";
+    if (p.wdec_groups > 0 && !named) {
+        *why = "fused weight decode needs whole-warp groups (bf16 rows, d a multiple of 1024)";
         return cudaErrorInvalidValue;
     }
     if (named) {

@@ -382,40 +382,62 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
 // CTAs arrives on the leader's accumulator-empty barrier.  Every TMA load fills only its own
 // CTA's shared memory.
 // ------------------------------------------------------------------------------------------
-constexpr int P_STAGES = 6;
+// ACODES (4-bit activation codes of a symmetric codebook): each CTA's TMA brings the packed
+// codes of its own 128 rows (128 x 32 bytes per k-block) into a code stage and signals its own
+// barrier; eight decoder warps per CTA expand them into the fp16 A stage in the 128-byte
+// swizzled layout the MMA reads and arrive on the leader's A-ready barrier (16 arrivals: both
+// CTAs' decoders).  The ring then holds 5 stages.  The stage's A tile is free when its codes
+// land, because the producer issued the code load only after the MMAs that last read the
+// stage had completed.
+template <bool ACODES>
+__host__ __device__ constexpr int pair_stages() { return ACODES ? 5 : 6; }
 constexpr int P_BM = 256, P_BN = 256;                    // pair tile
 constexpr int P_A_BYTES = 128 * BK * 2;                  // 16 KB: this CTA's 128 rows of A
 constexpr int P_B_BYTES = 128 * BK * 2;                  // 16 KB: this CTA's 128 rows of B
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
-constexpr int kPairNumBars = 2 * P_STAGES + 5;
-constexpr int kPairThreads = 32 * (2 + kEpiWarps);
+constexpr int P_CODE_BYTES = 128 * BK / 2;               // ACODES: 128 rows x 32 bytes
+// barriers: full, empty, [ACODES: code-full, A-ready] per stage; 2 accumulator-full,
+// 2 accumulator-empty, drain
+template <bool ACODES>
+__host__ __device__ constexpr int pair_num_bars() { return (ACODES ? 4 : 2) * pair_stages<ACODES>() + 5; }
+template <bool ACODES>
+__host__ __device__ constexpr int pair_threads() { return 32 * (2 + kEpiWarps + (ACODES ? kDecWarps : 0)); }
 constexpr uint32_t kIdescPair = idesc_f16(P_BM, P_BN);
 
+template <bool ACODES>
 __host__ __device__ constexpr size_t gemm_pair_smem() {
-    return 1024 + (size_t)P_STAGES * P_STAGE_BYTES + (size_t)kEpiWarps * 2 * kStageOut +
-           8 * kPairNumBars + 8 + kEpiWarps * 64 * sizeof(float) + 64;
+    return 1024 + (size_t)pair_stages<ACODES>() * (P_STAGE_BYTES + (ACODES ? P_CODE_BYTES : 0)) +
+           (size_t)kEpiWarps * 2 * kStageOut + 8 * pair_num_bars<ACODES>() + 8 +
+           kEpiWarps * 64 * sizeof(float) + 64;
 }
-static_assert(gemm_pair_smem() <= 227 * 1024, "shared memory budget (pair)");
+static_assert(gemm_pair_smem<false>() <= 227 * 1024 && gemm_pair_smem<true>() <= 227 * 1024,
+              "shared memory budget (pair)");
 
 // Warp roles as in k2_gemm: warp 0 lane 0 loads (both CTAs), warp 1 owns tensor memory (both
 // CTAs allocate the same columns) and its lane 0 issues the MMAs (leader only), warps 2..5
-// are the epilogue (both CTAs, each its own 128 rows).  Pair p takes tiles p, p + #pairs, ...
-template <bool BF16>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+// are the epilogue (both CTAs, each its own 128 rows), ACODES: warps 6..13 decode (both CTAs,
+// each its own 128 rows).  Pair p takes tiles p, p + #pairs, ...
+template <bool BF16, bool ACODES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<ACODES>(), 1)
     k2_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+    constexpr int S = pair_stages<ACODES>();
+    constexpr int kBarSets = ACODES ? 4 : 2;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;                 // same offsets in both CTAs
     unsigned char *basep = smem_raw + (base - raw);
-    const uint32_t sA = base, sB = base + P_STAGES * P_A_BYTES;
-    const uint32_t sOut = sB + P_STAGES * P_B_BYTES;              // [4 warps][2][4 KB]
+    const uint32_t sA = base, sB = base + S * P_A_BYTES;
+    const uint32_t sC = sB + S * P_B_BYTES;                       // ACODES: code stages
+    const uint32_t sOut = sC + (ACODES ? S * P_CODE_BYTES : 0);   // [4 warps][2][4 KB]
     const uint32_t bars = sOut + kEpiWarps * 2 * kStageOut;
     auto full_bar = [&](int s) { return bars + 8u * s; };                   // leader's is used
-    auto empty_bar = [&](int s) { return bars + 8u * (P_STAGES + s); };
-    auto tfull_bar = [&](int a) { return bars + 8u * (2 * P_STAGES + a); };
-    auto tempty_bar = [&](int a) { return bars + 8u * (2 * P_STAGES + 2 + a); };   // leader's
-    const uint32_t drain_bar = bars + 8u * (2 * P_STAGES + 4);
+    auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
+    auto cfull_bar = [&](int s) { return bars + 8u * (2 * S + s); };        // ACODES, local
+    auto afull_bar = [&](int s) { return bars + 8u * (3 * S + s); };        // ACODES, leader's
+    auto tfull_bar = [&](int a) { return bars + 8u * (kBarSets * S + a); };
+    auto tempty_bar = [&](int a) { return bars + 8u * (kBarSets * S + 2 + a); };   // leader's
+    const uint32_t drain_bar = bars + 8u * (kBarSets * S + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(basep + (drain_bar + 8u - base));
     float *rn_s = reinterpret_cast<float *>(basep + (drain_bar + 16u - base));   // [4][64]
     __shared__ int abort_flag;
@@ -430,9 +452,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
     pdl_trigger();
     if (threadIdx.x == 0) {
-        for (int s = 0; s < P_STAGES; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
+            if constexpr (ACODES) {
+                mbar_init(cfull_bar(s), 1);
+                mbar_init(afull_bar(s), 2 * kDecWarps);
+            }
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar(a), 1);
@@ -467,26 +493,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 const int m0 = (tile / n_tiles) * P_BM + (int)rank * 128;
                 const int n0 = (tile % n_tiles) * P_BN + (int)rank * 128;
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int s = it % P_STAGES;
-                    if (it >= P_STAGES &&
-                        !mbar_wait(empty_bar(s), ((it / P_STAGES) & 1) ^ 1)) {
+                    const int s = it % S;
+                    if (it >= S && !mbar_wait(empty_bar(s), ((it / S) & 1) ^ 1)) {
                         give_up(ERR_WAIT_EMPTY);
                         break;
                     }
                     if (aborted())
                         break;
-                    if (rank == 0)
-                        mbar_expect_tx(full_bar(s), 2 * P_STAGE_BYTES);
                     const uint32_t fb = mapa_shared(full_bar(s), 0);
-                    tma_load_2d_pair(sA + s * P_A_BYTES, &tmA, kb * BK, m0, fb);
+                    if constexpr (ACODES) {
+                        if (rank == 0)
+                            mbar_expect_tx(full_bar(s), 2 * P_B_BYTES);
+                        mbar_expect_tx(cfull_bar(s), P_CODE_BYTES);
+                        tma_load_2d(sC + s * P_CODE_BYTES, &tmA, kb * (BK / 2), m0, cfull_bar(s));
+                    } else {
+                        if (rank == 0)
+                            mbar_expect_tx(full_bar(s), 2 * P_STAGE_BYTES);
+                        tma_load_2d_pair(sA + s * P_A_BYTES, &tmA, kb * BK, m0, fb);
+                    }
                     tma_load_2d_pair(sB + s * P_B_BYTES, &tmB, kb * BK, n0, fb);
                 }
             }
-            if (aborted() && rank == 0) {
+            if (aborted()) {
                 // let the loads already issued land before the pair can exit
-                const uint32_t from = it > (uint32_t)P_STAGES ? it - P_STAGES : 0;
-                for (uint32_t j = from; j < it; ++j)
-                    mbar_wait(full_bar(j % P_STAGES), (j / P_STAGES) & 1);
+                const uint32_t from = it > (uint32_t)S ? it - S : 0;
+                for (uint32_t j = from; j < it; ++j) {
+                    if (rank == 0)
+                        mbar_wait(full_bar(j % S), (j / S) & 1);
+                    if (ACODES)
+                        mbar_wait(cfull_bar(j % S), (j / S) & 1);
+                }
             }
         }
     } else if (warp == 1) {
@@ -504,8 +540,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * kAccCols);
                 bool ok = true;
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
-                    const int s = it % P_STAGES;
-                    if (!mbar_wait(full_bar(s), (it / P_STAGES) & 1)) {
+                    const int s = it % S;
+                    if (!mbar_wait(full_bar(s), (it / S) & 1) ||
+                        (ACODES && !mbar_wait(afull_bar(s), (it / S) & 1))) {
                         give_up(ERR_WAIT_FULL);
                         ok = false;
                         break;
@@ -526,7 +563,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             if (!mbar_wait(drain_bar, 0))
                 atomicOr(&g_k2_err, ERR_WAIT_ACCUM);
         }
-    } else {
+    } else if (warp < 2 + kEpiWarps) {
         // ---------------- epilogue (both CTAs): this CTA's 128 rows of the tile ----------
         const int q = warp & 3;                               // TMEM lane quarter
         float *rn_w = rn_s + (warp - 2) * 64;
@@ -591,6 +628,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         if (lane == 0)
             bulk_wait_all();
+    } else if constexpr (ACODES) {
+        // ---------------- decoders (both CTAs): 4-bit codes -> this CTA's fp16 A stages ----
+        // Thread = row r of this CTA's 128 rows and one half of its 64 codes per k-block: 16
+        // bytes of codes in, 64 bytes of the fp16 row out in the 128-byte swizzled layout
+        // (16-byte piece k of row r at piece k ^ (r % 8), 8-row atoms of 1024 bytes).
+        const int r = (warp & 3) * 32 + lane;
+        const int half = (warp - 2 - kEpiWarps) >> 2;
+        const uint32_t row_off = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+        unsigned char *sAp = basep + (sA - base);
+        const unsigned char *sCp = basep + (sC - base);
+        const uint32_t ready = rank == 0 ? 0u : 1u;
+        uint32_t it = 0;
+        bool stop = false;
+        for (int tile = pair0; tile < num_tiles && !stop; tile += npair) {
+            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                const int s = it % S;
+                const bool ok = mbar_wait(cfull_bar(s), (it / S) & 1);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0)
+                        give_up(ERR_WAIT_FULL);
+                    stop = true;
+                    break;
+                }
+                if (__shfl_sync(0xffffffffu, aborted() ? 1 : 0, 0)) {
+                    stop = true;
+                    break;
+                }
+                const uint4 c = *reinterpret_cast<const uint4 *>(
+                    sCp + s * P_CODE_BYTES + r * (BK / 2) + half * 16);
+                const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+                unsigned char *dst = sAp + s * P_A_BYTES + row_off;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int k = half * 4 + j;               // 16-byte piece of the row
+                    uint32_t o[4];
+                    decode8(words[j], p.L0, p.L1, p.H0, p.H1, o);
+                    *reinterpret_cast<uint4 *>(dst + ((k ^ (r & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                fence_async_smem();                           // visible to the tensor core
+                __syncwarp();
+                if (lane == 0) {
+                    if (ready == 0)
+                        mbar_arrive(afull_bar(s));
+                    else
+                        mbar_arrive_remote(mapa_shared(afull_bar(s), 0));
+                }
+            }
+        }
     }
     __syncwarp();
     if (p.test_wait_cycles > 0 && blockIdx.x == 0 && threadIdx.x == 0)
@@ -607,8 +693,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 // ------------------------------------------------------------------------------------------
 // Host side.
 // ------------------------------------------------------------------------------------------
+// Encoded tensor maps, kept per host thread: a map is a pure function of its arguments, so a
+// call with the same buffer and shape (the usual case for a layer called again and again)
+// reuses the encoding instead of paying for cuTensorMapEncodeTiled on every call.
+struct MapKey {
+    const void *ptr;
+    long long rows;
+    int cols, box, kind;
+    bool operator==(const MapKey &o) const {
+        return ptr == o.ptr && rows == o.rows && cols == o.cols && box == o.box && kind == o.kind;
+    }
+};
+constexpr int kMapCacheSize = 16;
+thread_local MapKey g_map_keys[kMapCacheSize];
+thread_local CUtensorMap g_maps[kMapCacheSize];
+thread_local int g_map_used = 0, g_map_next = 0;
+
+template <class Encode>
+bool cached_map(CUtensorMap *map, const MapKey &key, Encode &&encode) {
+    for (int i = 0; i < g_map_used; ++i)
+        if (g_map_keys[i] == key) {
+            *map = g_maps[i];
+            return true;
+        }
+    if (!encode(map))
+        return false;
+    const int slot = g_map_used < kMapCacheSize ? g_map_used++ : g_map_next;
+    g_map_next = (slot + 1) % kMapCacheSize;
+    g_map_keys[slot] = key;
+    g_maps[slot] = *map;
+    return true;
+}
+
 // fp16 [rows, K] row-major -> tiles of box_rows x 64 with 128-byte swizzle.
-bool make_map(CUtensorMap *map, const void *ptr, long long rows, int K, int box_rows) {
+bool make_map_uncached(CUtensorMap *map, const void *ptr, long long rows, int K, int box_rows) {
     auto fn = tensor_map_encoder();
     if (!fn)
         return false;
@@ -621,6 +739,11 @@ bool make_map(CUtensorMap *map, const void *ptr, long long rows, int K, int box_
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap *map, const void *ptr, long long rows, int K, int box_rows) {
+    return cached_map(map, MapKey{ptr, rows, K, box_rows, 0},
+                      [&](CUtensorMap *m) { return make_map_uncached(m, ptr, rows, K, box_rows); });
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -641,7 +764,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-bool make_out_map(CUtensorMap *map, void *y, int T, int N, bool bf16) {
+bool make_out_map_uncached(CUtensorMap *map, void *y, int T, int N, bool bf16) {
     auto fn = tensor_map_encoder();
     if (!fn)
         return false;
@@ -657,6 +780,11 @@ bool make_out_map(CUtensorMap *map, void *y, int T, int N, bool bf16) {
     return r == CUDA_SUCCESS;
 }
 
+bool make_out_map(CUtensorMap *map, void *y, int T, int N, bool bf16) {
+    return cached_map(map, MapKey{y, T, N, 0, bf16 ? 2 : 1},
+                      [&](CUtensorMap *m) { return make_out_map_uncached(m, y, T, N, bf16); });
+}
+
 size_t linear_workspace_bytes(int T, int d, int N) {
     return align_up((size_t)T * d * 2, 1024) + align_up((size_t)N * d * 2, 1024);
 }
@@ -667,7 +795,7 @@ namespace {
 
 // 4-bit codes, uint8 [rows, K/2] row-major -> 128-row x 32-byte boxes (one k-block), no
 // swizzle.
-bool make_code_map(CUtensorMap *map, const uint8_t *codes, long long rows, int K) {
+bool make_code_map_uncached(CUtensorMap *map, const uint8_t *codes, long long rows, int K) {
     auto fn = tensor_map_encoder();
     if (!fn)
         return false;
@@ -679,6 +807,11 @@ bool make_code_map(CUtensorMap *map, const uint8_t *codes, long long rows, int K
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool make_code_map(CUtensorMap *map, const uint8_t *codes, long long rows, int K) {
+    return cached_map(map, MapKey{codes, rows, K, 0, 3},
+                      [&](CUtensorMap *m) { return make_code_map_uncached(m, codes, rows, K); });
 }
 
 template <bool BF16, bool ACODES>
@@ -712,7 +845,7 @@ cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const CU
 
 // Pairs of the CTA-pair GEMM that fit on the device at once (0: the form is unavailable),
 // once per device and instantiation.
-template <bool BF16>
+template <bool BF16, bool ACODES>
 int gemm_pair_slots() {
     static std::mutex mu;
     static int slots[kMaxDevices];
@@ -724,16 +857,16 @@ int gemm_pair_slots() {
     if (!done[dev]) {
         done[dev] = true;
         slots[dev] = 0;
-        auto kern = k2_gemm_pair<BF16>;
+        auto kern = k2_gemm_pair<BF16, ACODES>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gemm_pair_smem()) != cudaSuccess) {
+                                 (int)gemm_pair_smem<ACODES>()) != cudaSuccess) {
             cudaGetLastError();
             return 0;
         }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2, 1, 1);
-        cfg.blockDim = dim3(kPairThreads, 1, 1);
-        cfg.dynamicSmemBytes = gemm_pair_smem();
+        cfg.blockDim = dim3(pair_threads<ACODES>(), 1, 1);
+        cfg.dynamicSmemBytes = gemm_pair_smem<ACODES>();
         int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
             cudaGetLastError();
@@ -744,12 +877,13 @@ int gemm_pair_slots() {
     return slots[dev];
 }
 
-template <bool BF16>
+template <bool BF16, bool ACODES>
 cudaError_t launch_gemm_pair_t(const CUtensorMap &ma, const CUtensorMap &mb,
                                const CUtensorMap &my, const GemmParams &gp, int pairs,
                                cudaStream_t st, std::string *why) {
-    const cudaError_t e = launch_pdl(k2_gemm_pair<BF16>, dim3(2 * pairs), dim3(kPairThreads),
-                                     gemm_pair_smem(), st, ma, mb, my, gp);
+    const cudaError_t e =
+        launch_pdl(k2_gemm_pair<BF16, ACODES>, dim3(2 * pairs), dim3(pair_threads<ACODES>()),
+                   gemm_pair_smem<ACODES>(), st, ma, mb, my, gp);
     if (e != cudaSuccess)
         *why = "k2_gemm_pair launch";
     return e;
@@ -787,18 +921,25 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
         return cudaErrorInvalidValue;
     }
     CUtensorMap ma, mb, my;
-    if (!acodes && gemm_pair_enabled()) {
-        const int slots = y_bf16 ? gemm_pair_slots<true>() : gemm_pair_slots<false>();
+    if (gemm_pair_enabled()) {
+        const int slots = acodes ? (y_bf16 ? gemm_pair_slots<true, true>()
+                                           : gemm_pair_slots<false, true>())
+                                 : (y_bf16 ? gemm_pair_slots<true, false>()
+                                           : gemm_pair_slots<false, false>());
         if (slots > 0) {
-            if (!make_map(&ma, A16, T, d, 128) || !make_map(&mb, B16, N, d, 128) ||
-                !make_out_map(&my, y, T, N, y_bf16)) {
+            const bool a_ok = acodes ? make_code_map(&ma, x_codes4, T, d)
+                                     : make_map(&ma, A16, T, d, 128);
+            if (!a_ok || !make_map(&mb, B16, N, d, 128) || !make_out_map(&my, y, T, N, y_bf16)) {
                 *why = "cuTensorMapEncodeTiled failed";
                 return cudaErrorInvalidValue;
             }
             const int tiles = ((N + P_BN - 1) / P_BN) * ((T + P_BM - 1) / P_BM);
             const int pairs = tiles < slots ? tiles : slots;
-            return y_bf16 ? launch_gemm_pair_t<true>(ma, mb, my, gp, pairs, st, why)
-                          : launch_gemm_pair_t<false>(ma, mb, my, gp, pairs, st, why);
+            if (acodes)
+                return y_bf16 ? launch_gemm_pair_t<true, true>(ma, mb, my, gp, pairs, st, why)
+                              : launch_gemm_pair_t<false, true>(ma, mb, my, gp, pairs, st, why);
+            return y_bf16 ? launch_gemm_pair_t<true, false>(ma, mb, my, gp, pairs, st, why)
+                          : launch_gemm_pair_t<false, false>(ma, mb, my, gp, pairs, st, why);
         }
     }
     const bool a_ok = acodes ? make_code_map(&ma, x_codes4, T, d) : make_map(&ma, A16, T, d, BM);

@@ -595,6 +595,8 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
             p.dec_img = cw->dev_dec[dev];
             p.dec_words = (int)cw->dec_img.size();
         }
+    }
+    {
         if (fd && fd->rows > 0) {
             oq_codebook *fw = const_cast<oq_codebook *>(fd->cb);
             if (fw->bits == 4) {
@@ -1148,9 +1150,20 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     cudaStream_t side = device_side(di, &rc);
     if (!side)
         return rc;
-    // workspace: A16 [T, d] fp16 | B16 [N, d] fp16 | s [T] (if not given) | codes (fallback)
-    const bool direct = oq::k1_a16_supported(ca->bits, r->h, dtype == OQ_BF16);
-    const size_t a_bytes = align_up((size_t)T * d * 2, 1024);
+    // The activation operand takes one of three forms:
+    //   direct: K1 writes each code's fp16 centroid straight into the GEMM's A operand (bf16 x,
+    //           2/4/8-bit codes, 32 <= h <= 256);
+    //   codes:  K1 writes the packed 4-bit codes and the GEMM decodes them into its shared-
+    //           memory A tiles (OQ_LINEAR_PATH=fused; bf16 x, odd-symmetric 4-bit codebook);
+    //   else:   K1 writes codes and the decode prepass expands them into the fp16 A operand.
+    // workspace: A16 [T, d] fp16 (direct / prepass) | B16 [N, d] fp16 | s [T] (if not given) |
+    // codes [T, d*ba/8] (codes / prepass)
+    uint32_t src_probe[4];
+    const bool acodes = fused_requested() && ca->bits == 4 && dtype == OQ_BF16 &&
+                        oq::decode8_sources(ca->lut, &src_probe[0], &src_probe[1],
+                                            &src_probe[2], &src_probe[3]);
+    const bool direct = !acodes && oq::k1_a16_supported(ca->bits, r->h, dtype == OQ_BF16);
+    const size_t a_bytes = acodes ? 0 : align_up((size_t)T * d * 2, 1024);
     const size_t b_bytes = align_up((size_t)out_features * d * 2, 1024);
     const size_t s_bytes = s ? 0 : align_up((size_t)T * 4, 1024);
     const size_t c_bytes = direct ? 0 : align_up((size_t)T * d * ca->bits / 8, 1024);
@@ -1160,37 +1173,39 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     if (e != cudaSuccess)
         return fail_cuda(e, "oq_quantized_linear: workspace allocation");
     unsigned char *w8 = static_cast<unsigned char *>(ws);
-    uint16_t *A16 = reinterpret_cast<uint16_t *>(w8);
+    uint16_t *A16 = acodes ? nullptr : reinterpret_cast<uint16_t *>(w8);
     uint16_t *B16 = reinterpret_cast<uint16_t *>(w8 + a_bytes);
     float *sv = s ? s : reinterpret_cast<float *>(w8 + a_bytes + b_bytes);
     uint8_t *codes = direct ? nullptr : w8 + a_bytes + b_bytes + s_bytes;
     std::string why;
     // 2-bit weights, or 4-bit weights of an odd-symmetric codebook, with the one-CTA-per-SM
-    // K1: the K1 groups that run out of token pairs decode the weights (no second kernel, no
-    // side stream)
-    uint32_t src_probe[4];
-    // Only while the decode is no bigger than K1's own work (N <= T) and K1 holds at least
-    // four groups per SM (d <= 5120): a larger weight matrix, or one decoded by a single group
-    // per SM, decodes faster beside K1 than in its tail.
+    // K1 (direct or codes form): the K1 groups that run out of token pairs decode the weights
+    // (no second kernel, no side stream).  Only while the decode is no bigger than K1's own
+    // work (N <= T) and K1 holds at least four groups per SM (d <= 5120): a larger weight
+    // matrix, or one decoded by a single group per SM, decodes faster beside K1 than in its
+    // tail.
     const bool fuse =
-        direct && out_features <= T && d <= 5120 && !tc_k1_requested() &&
+        (direct || acodes) && out_features <= T && d <= 5120 && !tc_k1_requested() &&
         oq::k1_named(d, dtype == OQ_BF16) &&
         (cw->bits == 2 || (cw->bits == 4 && oq::decode8_sources(cw->lut, &src_probe[0],
                                                                  &src_probe[1], &src_probe[2],
                                                                  &src_probe[3])));
+    auto gemm = [&]() {
+        return timed(OQ_KERNEL_GEMM, st, [&] {
+            return oq::launch_gemm(A16, codes, ca->lut, B16, sv, row_norms, y,
+                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
+                                   take_armed(OQ_KERNEL_GEMM));
+        });
+    };
     if (fuse) {
         FusedDecode fd;
         fd.cb = cw;
         fd.codes = W_codes;
         fd.out = B16;
         fd.rows = out_features;
-        rc = quantize_rows(r, ca, x, dtype, T, d, nullptr, sv, st, 1e-8f, who, gelu, A16, &fd);
+        rc = quantize_rows(r, ca, x, dtype, T, d, codes, sv, st, 1e-8f, who, gelu, A16, &fd);
         if (rc == OQ_OK) {
-            e = timed(OQ_KERNEL_GEMM, st, [&] {
-                return oq::launch_gemm(A16, nullptr, nullptr, B16, sv, row_norms, y,
-                                       out_dtype == OQ_BF16, T, out_features, d, st, di->sms,
-                                       &why, take_armed(OQ_KERNEL_GEMM));
-            });
+            e = gemm();
             if (e != cudaSuccess)
                 rc = fail_cuda(e, why.c_str());
         }
@@ -1221,7 +1236,7 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     }
     rc = quantize_rows(r, ca, x, dtype, T, d, codes, sv, st, 1e-8f, who, gelu,
                        direct ? A16 : nullptr);
-    if (rc == OQ_OK && !direct) {
+    if (rc == OQ_OK && !direct && !acodes) {
         e = timed(OQ_KERNEL_DECODE, st, [&] {
             return oq::launch_decode(ca->bits, codes, A16, T, d, ca->lut, st, di->sms, &why);
         });
@@ -1232,11 +1247,7 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     // workspace is released after every use of it
     e = cudaStreamWaitEvent(st, di->join, 0);
     if (rc == OQ_OK && e == cudaSuccess) {
-        e = timed(OQ_KERNEL_GEMM, st, [&] {
-            return oq::launch_gemm(A16, nullptr, nullptr, B16, sv, row_norms, y,
-                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
-                                   take_armed(OQ_KERNEL_GEMM));
-        });
+        e = gemm();
         if (e != cudaSuccess)
             rc = fail_cuda(e, why.c_str());
     } else if (rc == OQ_OK) {

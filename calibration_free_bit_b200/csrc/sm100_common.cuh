@@ -306,6 +306,13 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                  ::"r"(cluster_bar) : "memory");
 }
 
+// The same arrive with the instruction's default semantics (release at CTA scope): for a
+// producer whose data the peer's tensor core reads through the async proxy, after
+// fence.proxy.async has ordered the data writes before it.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
 // Pair TMA load: this CTA's tile lands in its own shared memory; the transaction bytes count
 // on the mbarrier at `cluster_bar` (the leader CTA's); the data lands in this CTA only.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x,

@@ -159,8 +159,10 @@ int oq_quantize_act_gelu(const oq_rpbh *r, const oq_codebook *ca, const void *x,
  * Centroids enter the tensor cores as fp16 unit-variance values; accumulation is fp32.
  * Both code operands are decoded into fp16 buffers first.  With 4-bit activation codes and
  * the environment variable OQ_LINEAR_PATH=fused (read once per process), the activation codes
- * are instead decoded inside the GEMM kernel, into its shared-memory operand tiles, and only
- * the weight codes get an fp16 buffer (less device memory, more decode work per call).
+ * are instead brought into the GEMM kernel by TMA as packed codes and decoded there, through
+ * the codebook's fp16 LUT held in registers, into its shared-memory operand tiles; only the
+ * weight codes get an fp16 buffer (less device memory and traffic, more decode work per call;
+ * the same y bit for bit, since both forms feed the MMA the same fp16 values).
  * Either way the temporary device memory is stream-ordered, from a library-owned
  * pool.  The fp16 operands meet in a tcgen05 GEMM on pairs of CTAs (256 x 256 output tiles);
  * the environment variable OQ_GEMM_PAIR=0 (read once per process) selects the single-CTA
@@ -177,11 +179,13 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * oq_quantize_act followed by oq_linear, without materialising x_codes: the rotate+quantize
  * kernel writes each code's fp16 unit centroid straight into the GEMM's A operand (bf16 x,
  * ba in {2, 4, 8}, 32 <= h <= 256; otherwise codes and the decode prepass are used inside the
- * call).  With 2- or 4-bit weight codes, d a multiple of 1024 up to 5120, bf16 x and
- * out_features <= T, that kernel also decodes the weight codes into the GEMM's B operand once
- * it runs out of tokens; otherwise the weight codes are decoded on a library-owned side
- * stream of the device while x is quantized.  y and s are bit-identical to
- * oq_quantize_act + oq_linear.
+ * call).  With OQ_LINEAR_PATH=fused (read once per process), bf16 x and 4-bit activation
+ * codes, the rotate+quantize kernel writes the packed codes instead and the GEMM decodes them
+ * in shared memory (as oq_linear does under that variable).  With 2- or 4-bit weight codes, d
+ * a multiple of 1024 up to 5120, bf16 x and out_features <= T, the rotate+quantize kernel
+ * also decodes the weight codes into the GEMM's B operand once it runs out of tokens;
+ * otherwise the weight codes are decoded on a library-owned side stream of the device while x
+ * is quantized.  y and s are bit-identical to oq_quantize_act + oq_linear.
  * x: device [T, d] of dtype; W_codes [out_features, d*bw/8]; row_norms fp32 [out_features];
  * y: device [T, out_features] of out_dtype (OQ_F32 or OQ_BF16); s: optional device fp32 [T]
  * receiving the norms (NULL: kept internal).  flags: OQ_FORWARD_GELU quantizes GELU(x)

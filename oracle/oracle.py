@@ -250,9 +250,11 @@ def quantize_rows(x, h: int, perm, sign, bits: int, eps: float, detail: bool = F
 
 
 def gelu(x) -> np.ndarray:
-    """GELU in its erf form, x Phi(x) = x (1 + erf(x / sqrt 2)) / 2, in fp64."""
+    """GELU in its exact (erf) form, x Phi(x), in fp64, with the normal CDF written as
+    Phi(x) = erfc(-x / sqrt 2) / 2: the same function as (1 + erf(x / sqrt 2)) / 2, evaluated
+    without the cancellation of 1 + erf for negative x (which loses the left tail)."""
     x = np.asarray(x, dtype=np.float64)
-    return 0.5 * x * (1.0 + special.erf(x / math.sqrt(2.0)))
+    return 0.5 * x * special.erfc(-x / math.sqrt(2.0))
 
 
 def quantize_act(x, h, perm, sign, bits, detail=False, marginal="gauss", gelu_input=False):

@@ -63,8 +63,10 @@ def handles(oq, d, h, ba, bw, seed=0):
     return _HANDLES[key]
 
 
-def check_codes(gpu_packed, orc_packed, orc_u, d, bits, what, marginal="gauss"):
-    """Code-parity rule on a block of rows; returns the number of mismatches."""
+def check_codes(gpu_packed, orc_packed, orc_u, d, bits, what, marginal="gauss",
+                count_rule=True):
+    """Code-parity rule on a block of rows; returns the number of mismatches.  count_rule:
+    apply the 99.99 % bound (off only for inputs built to sit on a boundary)."""
     gpu_packed = np.ascontiguousarray(gpu_packed)
     gcodes = O.unpack(gpu_packed, d, bits)
     # layout: the oracle's packer reproduces the GPU's bytes exactly
@@ -72,7 +74,8 @@ def check_codes(gpu_packed, orc_packed, orc_u, d, bits, what, marginal="gauss"):
     ocodes = O.unpack(orc_packed, d, bits)
     bad = np.argwhere(gcodes != ocodes)
     n = gcodes.size
-    assert len(bad) <= (1 - CODE_MATCH) * n + 1e-9, f"{what}: {len(bad)} of {n} codes differ"
+    if count_rule:
+        assert len(bad) <= (1 - CODE_MATCH) * n + 1e-9, f"{what}: {len(bad)} of {n} codes differ"
     _, t = O.codebook(bits, marginal, d)
     for r, k in bad:
         u = orc_u[r, k]
@@ -348,26 +351,33 @@ def test_linear_video_ffn_up_full_size(oq, variant):
     _sampled_linear(oq, p, rows, cols)
 
 
-@pytest.mark.parametrize("path", ["fused", "default", "single"])
-def test_linear_path_selection(oq, path):
-    """Every oq_linear GEMM form against the oracle: the fp16 prepass feeding the CTA-pair
-    GEMM (default), the same prepass feeding the single-CTA GEMM (OQ_GEMM_PAIR=0), and 4-bit
-    activation codes decoded inside the GEMM (OQ_LINEAR_PATH=fused); each runs in a child
-    process because the variables are read once per process."""
+def test_linear_path_selection(oq):
+    """Every GEMM form against the oracle, each in a child process (the variables are read
+    once per process): the fp16 prepass feeding the CTA-pair GEMM (default), the same prepass
+    feeding the single-CTA GEMM (OQ_GEMM_PAIR=0), and 4-bit activation codes decoded inside
+    the CTA-pair GEMM (OQ_LINEAR_PATH=fused) or the single-CTA one (both variables).  In each,
+    oq_quantized_linear takes the same form and equals the two calls bit for bit, and the
+    attention workload's y is identical across all forms (same fp16 operands, same MMA
+    order)."""
     import os
+    import re
     import subprocess
     import sys
-    env = dict(os.environ)
-    env.pop("OQ_LINEAR_PATH", None)
-    env.pop("OQ_GEMM_PAIR", None)
-    if path == "fused":
-        env["OQ_LINEAR_PATH"] = "fused"
-    if path == "single":
-        env["OQ_GEMM_PAIR"] = "0"
     child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_linear_path_child.py")
-    r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
-                       timeout=600)
-    assert r.returncode == 0, r.stdout + r.stderr
+    hashes = {}
+    for path in ("default", "fused", "single", "fused_single"):
+        env = dict(os.environ)
+        env.pop("OQ_LINEAR_PATH", None)
+        env.pop("OQ_GEMM_PAIR", None)
+        if path.startswith("fused"):
+            env["OQ_LINEAR_PATH"] = "fused"
+        if path.endswith("single"):
+            env["OQ_GEMM_PAIR"] = "0"
+        r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
+                           timeout=600)
+        assert r.returncode == 0, path + ": " + r.stdout + r.stderr
+        hashes[path] = re.search(r"yhash ([0-9a-f]+)", r.stdout).group(1)
+    assert len(set(hashes.values())) == 1, hashes
 
 
 @pytest.mark.parametrize("ba,bw", [(4, 4), (2, 8)])
@@ -569,7 +579,14 @@ def test_k1_blocks_below_32(oq, h, bits, dtype, d, gelu):
     perm, sign = O.build_rpbh(d, 0)
     o, os_, _, ou = O.quantize_act(x.double().numpy(), h, perm, sign, bits, detail=True,
                                    gelu_input=gelu)
-    check_codes(xc.cpu().numpy(), o, ou, d, bits, f"h={h} b={bits} d={d}")
+    # GELU sends every strongly negative input to almost zero, and a block of 2 or 4 such
+    # values rotates to almost zero, which is the middle boundary of every codebook here: on
+    # this input about 0.6 % (h = 2) and 0.1 % (h = 4) of the values lie within 2e-6 sigma of
+    # a boundary, far more than the 0.01 % the count rule allows for.  There every mismatch
+    # must still be a neighbour code within 1e-5 sigma of their boundary, without the count.
+    concentrated = gelu and h <= 4
+    check_codes(xc.cpu().numpy(), o, ou, d, bits, f"h={h} b={bits} d={d}",
+                count_rule=not concentrated)
     np.testing.assert_allclose(s.cpu().double().numpy(), os_, rtol=NORM_RTOL)
 
 

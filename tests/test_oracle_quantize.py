@@ -167,6 +167,10 @@ def test_gelu_pins():
     np.testing.assert_allclose(O.gelu(x) - O.gelu(-x), x, atol=1e-14)
     assert O.gelu(0.0) == 0.0
     assert O.gelu(40.0) == 40.0 and abs(O.gelu(-40.0)) < 1e-300
+    # the left tail keeps its relative accuracy: Phi(-5) = 2.866515718791939e-7 and
+    # Phi(-10) = 7.619853024160527e-24 from the normal tail tables (Q(5), Q(10))
+    assert O.gelu(-5.0) == pytest.approx(-5.0 * 2.866515718791939e-07, rel=1e-12)
+    assert O.gelu(-10.0) == pytest.approx(-10.0 * 7.619853024160527e-24, rel=1e-12)
 
 
 def test_quantize_gelu_input_is_quantize_of_gelu():
