@@ -3,7 +3,8 @@
 Sources: csrc/oq_host.cpp (handles, table builders, launches), csrc/k1_rotquant.cu (fused
 rotate + norm + quantize on the CUDA cores), csrc/k1_tc.cu (the same with the block transform
 on the tensor cores, bf16 rows), csrc/k2_decode.cu (code -> fp16 prepass), csrc/k2_linear.cu
-(tcgen05 GEMM; it decodes 4-bit activation codes itself).  Objects are compiled
+(tcgen05 GEMM; it decodes 4-bit activation codes itself), csrc/k3_fused.cu (the one-call step
+as one persistent kernel).  Objects are compiled
 in parallel into calibration_free_bit_b200/_build/ and linked into
 calibration_free_bit_b200/liboq.so; the CUDA runtime is linked statically, the driver API is
 reached through cudaGetDriverEntryPoint, so the library loads on a machine without a GPU.
@@ -19,7 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "liboq.so")
 INCLUDE = os.path.join(ROOT, "include")
-SOURCES = ["oq_host.cpp", "k1_rotquant.cu", "k1_tc.cu", "k2_decode.cu", "k2_linear.cu"]
+SOURCES = ["oq_host.cpp", "k1_rotquant.cu", "k1_tc.cu", "k2_decode.cu", "k2_linear.cu",
+           "k3_fused.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3",
                 "-I" + INCLUDE, "-I" + CSRC]

@@ -956,6 +956,10 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
                   : launch_gemm_t<false, false>(ma, mb, my, gp, grid, st, why);
 }
 
+bool make_operand_map(CUtensorMap *map, const void *ptr, long long rows, int K) {
+    return make_map(map, ptr, rows, K, 128);
+}
+
 size_t noalloc_workspace_bytes() { return kNoAllocWorkspaceBytes; }
 
 cudaError_t noalloc_workspace(void **out) {

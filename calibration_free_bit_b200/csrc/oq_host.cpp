@@ -684,6 +684,118 @@ bool fused_requested() {
     return v;
 }
 
+// OQ_FUSED_STEP=1 runs oq_quantized_linear as one persistent kernel (k3_fused.cu) where it
+// applies (read once per process).
+bool fused_step_requested() {
+    static const bool v = [] {
+        const char *e = std::getenv("OQ_FUSED_STEP");
+        return e != nullptr && std::strcmp(e, "1") == 0;
+    }();
+    return v;
+}
+
+// oq_quantized_linear as one persistent kernel: the decode prepass of the weights, then the
+// quantize stage and the CTA-pair GEMM side by side (k3_fused.cu).  Arguments validated by
+// the caller.
+int fused_step(const oq_rpbh *r, const oq_codebook *ca, const oq_codebook *cw, const void *x,
+               const uint8_t *W_codes, const float *row_norms, int T, int d, int out_features,
+               void *y, int out_dtype, float *s, cudaStream_t st, int dev, DeviceInfo *di,
+               cudaMemPool_t pool, const char *who) {
+    oq_rpbh *rw = const_cast<oq_rpbh *>(r);
+    oq_codebook *caw = const_cast<oq_codebook *>(ca);
+    int rc;
+    if ((rc = upload(caw->mu, &caw->dev_tbl[dev], caw->tbl_img, "upload quantizer table")) !=
+        OQ_OK)
+        return rc;
+    if ((rc = upload(rw->mu, &rw->dev_ent[0][dev], rw->ent_img[0], "upload rotation table")) !=
+        OQ_OK)
+        return rc;
+    oq::FusedStepParams p{};
+    if (ca->bits == 4) {
+        if (!oq::decode8_sources(ca->lut, &p.dec_src[0], &p.dec_src[1], &p.dec_src[2],
+                                 &p.dec_src[3]))
+            return fail(OQ_EINVAL, "%s: 4-bit codebook is not odd-symmetric", who);
+    } else {
+        if ((rc = upload(caw->mu, &caw->dev_dec[dev], caw->dec_img, "upload decode table")) !=
+            OQ_OK)
+            return rc;
+        p.dec_img = caw->dev_dec[dev];
+        p.dec_words = (int)caw->dec_img.size();
+    }
+    // workspace: A16 [T, d] | B16 [N, d] | s [T] (if not given) | progress counters
+    const size_t a_bytes = align_up((size_t)T * d * 2, 1024);
+    const size_t b_bytes = align_up((size_t)out_features * d * 2, 1024);
+    const size_t s_bytes = s ? 0 : align_up((size_t)T * 4, 1024);
+    const size_t c_bytes = align_up(4 * oq::fused_step_counter_words(T, out_features), 256);
+    void *ws = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(&ws, a_bytes + b_bytes + s_bytes + c_bytes, pool, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, "oq_quantized_linear: workspace allocation");
+    unsigned char *w8 = static_cast<unsigned char *>(ws);
+    uint16_t *A16 = reinterpret_cast<uint16_t *>(w8);
+    uint16_t *B16 = reinterpret_cast<uint16_t *>(w8 + a_bytes);
+    float *sv = s ? s : reinterpret_cast<float *>(w8 + a_bytes + b_bytes);
+    unsigned *ctr = reinterpret_cast<unsigned *>(w8 + a_bytes + b_bytes + s_bytes);
+    std::string why;
+    // 2-bit weights, or 4-bit weights of an odd-symmetric codebook: decoded inside the kernel
+    oq_codebook *cww = const_cast<oq_codebook *>(cw);
+    bool wdec_in = false;
+    if (cw->bits == 4 && oq::decode8_sources(cw->lut, &p.wdec_src[0], &p.wdec_src[1],
+                                             &p.wdec_src[2], &p.wdec_src[3])) {
+        wdec_in = true;
+    } else if (cw->bits == 2) {
+        if ((rc = upload(cww->mu, &cww->dev_dec[dev], cww->dec_img,
+                         "upload weight decode table")) != OQ_OK) {
+            cudaFreeAsync(ws, st);
+            return rc;
+        }
+        p.wdec_tab = reinterpret_cast<const uint2 *>(cww->dev_dec[dev]);
+        wdec_in = true;
+    }
+    if (wdec_in) {
+        p.wcodes = reinterpret_cast<const uint32_t *>(W_codes);
+        p.b16 = reinterpret_cast<uint4 *>(B16);
+        p.wdec_words = (long long)out_features * d * cw->bits / 32;
+        p.wdec_bits = cw->bits;
+    }
+    e = cudaMemsetAsync(ctr, 0, c_bytes, st);
+    if (e == cudaSuccess && !wdec_in)
+        e = timed(OQ_KERNEL_DECODE, st, [&] {
+            return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
+                                     di->sms, &why);
+        });
+    if (e == cudaSuccess) {
+        p.x = static_cast<const unsigned char *>(x);
+        p.a16 = A16;
+        p.s = sv;
+        p.ent_img = rw->dev_ent[0][dev];
+        p.tbl_img = caw->dev_tbl[dev];
+        p.ent_words = (int)rw->ent_img[0].size();
+        p.tbl_words = (int)caw->tbl_img.size();
+        p.eps = 1e-8f;
+        p.K = (float)(std::sqrt((double)d / r->h) / (ca->G * ca->delta));
+        p.G = ca->G;
+        p.F = ca->F;
+        p.rn = row_norms;
+        p.T = T;
+        p.N = out_features;
+        p.d = d;
+        p.inv_d = 1.0f / (float)d;
+        p.ctr = ctr;
+        p.test_wait_cycles = take_armed(OQ_KERNEL_GEMM);
+        e = timed(OQ_KERNEL_FUSED, st, [&] {
+            return oq::launch_fused_step(p, ca->bits, r->h, out_dtype == OQ_BF16, B16, y, st,
+                                         &why);
+        });
+    }
+    cudaError_t e2 = cudaFreeAsync(ws, st);
+    if (e != cudaSuccess)
+        return fail_cuda(e, why.empty() ? "oq_quantized_linear: fused step" : why.c_str());
+    if (e2 != cudaSuccess)
+        return fail_cuda(e2, "oq_quantized_linear: workspace release");
+    return OQ_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------------------
@@ -1150,6 +1262,11 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     cudaStream_t side = device_side(di, &rc);
     if (!side)
         return rc;
+    // The whole step as one persistent kernel where it applies (OQ_FUSED_STEP=1)
+    if (fused_step_requested() && !gelu && !tc_k1_requested() &&
+        oq::fused_step_supported(d, r->h, ca->bits, dtype == OQ_BF16))
+        return fused_step(r, ca, cw, x, W_codes, row_norms, T, d, out_features, y, out_dtype, s,
+                          (cudaStream_t)stream, dev, di, pool, who);
     // The activation operand takes one of three forms:
     //   direct: K1 writes each code's fp16 centroid straight into the GEMM's A operand (bf16 x,
     //           2/4/8-bit codes, 32 <= h <= 256);
@@ -1266,20 +1383,24 @@ int oq_check(void *stream) {
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess)
         return fail_cuda(e, "oq_check: stream synchronize");
-    unsigned w1 = 0, w2 = 0, w3 = 0;
+    unsigned w1 = 0, w2 = 0, w3 = 0, w4 = 0;
     if ((e = oq::read_and_clear_k1_error(&w1, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k1 error word");
+    if ((e = oq::read_and_clear_k3_error(&w4, st)) != cudaSuccess)
+        return fail_cuda(e, "oq_check: read fused-step error word");
     if ((e = oq::read_and_clear_k1tc_error(&w3, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k1 (tensor-core) error word");
     if ((e = oq::read_and_clear_k2_error(&w2, st)) != cudaSuccess)
         return fail_cuda(e, "oq_check: read k2 error word");
-    if (w1 || w2 || w3)
+    if (w1 || w2 || w3 || w4)
         return fail(OQ_EDEVICE, "device error word: quantize=0x%x quantize_tc=0x%x linear=0x%x "
-                                "(a bounded wait gave up; quantize bits 1/2 = row copy/armed test "
-                                "wait; quantize_tc bits 1/2/4/8/16 = staging/operand "
-                                "ring/accumulator/norm/code tile; linear bits 1/2/4/8 = operand "
-                                "stage/ring slot/accumulator/armed test wait)",
-                    w1, w3, w2);
+                                "fused=0x%x (a bounded wait gave up; quantize bits 1/2 = row "
+                                "copy/armed test wait; quantize_tc bits 1/2/4/8/16 = "
+                                "staging/operand ring/accumulator/norm/code tile; linear bits "
+                                "1/2/4/8 = operand stage/ring slot/accumulator/armed test wait; "
+                                "fused bits 1/2/4/8/16 = GEMM stage/quantized rows/tile id/row "
+                                "copy/armed test wait)",
+                    w1, w3, w2, w4);
     return OQ_OK;
 }
 

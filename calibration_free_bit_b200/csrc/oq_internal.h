@@ -7,6 +7,7 @@
 #include <string>
 #include <vector>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "oq.h"
@@ -143,6 +144,44 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
                         const uint16_t *B16, const float *s, const float *rn, void *y,
                         bool y_bf16, int T, int N, int d, cudaStream_t st, int num_sms,
                         std::string *why, long long test_wait_cycles = 0);
+
+// The online step in one persistent kernel (k3_fused.cu): the quantize stage and the CTA-pair
+// GEMM side by side on every SM, rows handed over through per-block counters.
+struct FusedStepParams {
+    // quantize stage (as K1 with fp16 output)
+    const unsigned char *x;             // bf16 [T, d]
+    uint16_t *a16;                      // fp16 [T, d]: the GEMM's A operand
+    float *s;                           // [T]
+    const uint32_t *ent_img, *tbl_img, *dec_img;   // K1's bf16 entry image and tables
+    int ent_words, tbl_words, dec_words;
+    uint32_t dec_src[4];
+    float eps, K;
+    int G, F;
+    // GEMM
+    const float *rn;
+    int T, N, d;
+    float inv_d;
+    // weight decode inside the kernel (2- or 4-bit weight codes; wdec_words = 0: B16 was
+    // decoded before the launch): W_codes as 32-bit words -> fp16 B16 [N, d]
+    const uint32_t *wcodes;
+    uint4 *b16;
+    long long wdec_words;
+    int wdec_bits;
+    uint32_t wdec_src[4];               // 4-bit: byte-permute sources of the weight codebook
+    const uint2 *wdec_tab;              // 2-bit: byte -> four fp16 centroids
+    // progress counters, zeroed before the launch: [0] next token pair, [1] next tile,
+    // [2] next weight-decode chunk, [3] weight-decode chunks done, [4 + b] rows of 256-row
+    // block b of x done (fused_step_counter_words(T, N) words)
+    unsigned *ctr;
+    long long test_wait_cycles;
+};
+bool fused_step_supported(int d, int h, int bits, bool bf16_in);
+size_t fused_step_counter_words(int T, int N);
+cudaError_t launch_fused_step(const FusedStepParams &p, int bits, int h, bool y_bf16,
+                              const uint16_t *B16, void *y, cudaStream_t st, std::string *why);
+cudaError_t read_and_clear_k3_error(unsigned *out, cudaStream_t st);
+// fp16 [rows, K] row-major operand -> TMA map of 128-row x 64 boxes, 128-byte swizzle
+bool make_operand_map(CUtensorMap *map, const void *ptr, long long rows, int K);
 
 // Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
 // its size, and its address on the current device (looked up once per device).

@@ -185,7 +185,12 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * a multiple of 1024 up to 5120, bf16 x and out_features <= T, the rotate+quantize kernel
  * also decodes the weight codes into the GEMM's B operand once it runs out of tokens;
  * otherwise the weight codes are decoded on a library-owned side stream of the device while x
- * is quantized.  y and s are bit-identical to oq_quantize_act + oq_linear.
+ * is quantized.  With OQ_FUSED_STEP=1 (read once per process), bf16 x without GELU, 2/4/8-bit
+ * activation codes, h in {64, 128, 256} and d in {1024, 2048, 3072, 4096}, one persistent
+ * kernel decodes 2- or 4-bit weight codes (others: a decode launch before it), then runs the
+ * rotate+quantize stage and the GEMM side by side on every SM, the GEMM taking each 256-row
+ * block as soon as its rows are quantized (opt-in: measured slower than the default form on
+ * a 4608 x 3072 x 3072 W4A4 projection).  y and s are bit-identical to oq_quantize_act + oq_linear in every form.
  * x: device [T, d] of dtype; W_codes [out_features, d*bw/8]; row_norms fp32 [out_features];
  * y: device [T, out_features] of out_dtype (OQ_F32 or OQ_BF16); s: optional device fp32 [T]
  * receiving the norms (NULL: kept internal).  flags: OQ_FORWARD_GELU quantizes GELU(x)
@@ -257,6 +262,7 @@ void oq_free_codebook(oq_codebook *cb);
 #define OQ_KERNEL_QUANTIZE 1   /* fused rotate + norm + quantize */
 #define OQ_KERNEL_DECODE 2     /* codes -> fp16 centroid prepass of oq_linear */
 #define OQ_KERNEL_GEMM 3       /* tcgen05 codebook GEMM of oq_linear */
+#define OQ_KERNEL_FUSED 4      /* quantize stage and GEMM in one kernel (OQ_FUSED_STEP=1) */
 typedef struct {
     int kernel;
     float ms;

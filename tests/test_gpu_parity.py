@@ -380,6 +380,23 @@ def test_linear_path_selection(oq):
     assert len(set(hashes.values())) == 1, hashes
 
 
+def test_fused_step_matches_the_two_calls(oq):
+    """OQ_FUSED_STEP=1: oq_quantized_linear as one persistent kernel (the rotate+quantize stage
+    and the CTA-pair GEMM side by side, rows handed over per 256-row block) equals
+    oq_quantize_act + oq_linear bit for bit on every supported shape tried, ragged T and N, one
+    token, bf16 y and two calls in a row; a shape outside its range takes the other forms.
+    Runs in a child process (the variable is read once per process)."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, OQ_FUSED_STEP="1")
+    env.pop("OQ_LINEAR_PATH", None)
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_fused_step_child.py")
+    r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 @pytest.mark.parametrize("ba,bw", [(4, 4), (2, 8)])
 @pytest.mark.parametrize("T,N,d", [(200, 272, 384), (129, 784, 1024)])
 def test_linear_bf16_output(oq, ba, bw, T, N, d):
