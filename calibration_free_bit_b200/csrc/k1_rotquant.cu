@@ -146,21 +146,26 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
 
     extern __shared__ __align__(16) unsigned char smem[];
     const int d = p.d;
-    const int GT = d / kE;                           // threads per token pair
+    const int GT = d / kE;                           // position-owning threads per token pair
+    // threads per group: NAMED groups are padded to whole warps, and their padding lanes own
+    // no positions (they run the group's steps on a duplicate entry row, take no part in the
+    // norm and store nothing)
+    const int GTP = NAMED ? ((GT + 31) & ~31) : GT;
     const int NG = p.groups;
     const int nstage = IN_F32 ? p.stages : 1;        // raw row buffers per group
     const int tid = threadIdx.x;
-    const int grp = tid / GT;
-    const int g = tid - grp * GT;
+    const int grp = tid / GTP;
+    const int g = tid - grp * GTP;
+    const bool owns = g < GT;
     const int lane = tid & 31;
     const int warp_start = tid - lane;
     const int active = min(32, (int)blockDim.x - warp_start);
     const unsigned wmask = active == 32 ? 0xffffffffu : ((1u << active) - 1u);
     const uint32_t row_in = (uint32_t)d * IN_BYTES;  // bytes of one input row
-    // NAMED: a group waits only for its own threads (named barrier 1 + grp, GT threads)
+    // NAMED: a group waits only for its own threads (named barrier 1 + grp, GTP threads)
     auto group_sync = [&]() {
         if constexpr (NAMED)
-            asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(GT) : "memory");
+            asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(GTP) : "memory");
         else
             __syncthreads();
     };
@@ -207,7 +212,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     // the h-block (0 when a block fits inside one thread)
     const int r = g % Q;
     const int pos0 = g * kE;
-    const uint4 *myent = reinterpret_cast<const uint4 *>(gent + g * kEntStride);
+    const uint4 *myent = reinterpret_cast<const uint4 *>(gent + min(g, GT - 1) * kEntStride);
     const uint32_t tbl_lane =
         smem_u32(table) + (REPL ? lane * 4 : 0) - ((0x3F800000u >> p.F) << TSH);
     const uint32_t G = (uint32_t)p.G;
@@ -216,7 +221,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     const int seg_end = min(active, lane + (GT - g));
     const bool seg_head = (lane == 0) || (g == 0);
     const int seg_slot = (g == 0) ? 0 : (g + 31) / 32;
-    const int nslots = 1 + ((grp * GT + GT - 1) / 32 - (grp * GT) / 32);
+    const int nslots = NAMED ? (GT + 31) / 32 : 1 + ((grp * GT + GT - 1) / 32 - (grp * GT) / 32);
     const int row_bytes = d * BITS / 8;
     const long long npairs = ((long long)p.T + 1) / 2;
     // The group's pairs are lo + my for my < cnt.  NAMED: the CTA owns an equal contiguous
@@ -269,7 +274,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
 
         if constexpr (!IN_F32) {
             // ---- interleave the staged rows into the pair buffer ---------------------------
-            if (valid) {
+            if (valid && owns) {
                 const uint4 *r0 = reinterpret_cast<const uint4 *>(cur);
                 const uint4 *r1 = reinterpret_cast<const uint4 *>(cur + row_in);
                 uint4 *slots = reinterpret_cast<uint4 *>(mypairs);
@@ -446,7 +451,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
                 w1[wi] = pack_codes<BITS>(d1);
             }
         }
-        if (valid) {
+        if (valid && owns) {
             if constexpr (A16) {
                 uint4 *a0 = reinterpret_cast<uint4 *>(p.a16 + t0 * d + pos0);
                 const uint32_t src[4] = {p.dec_src[0], p.dec_src[1], p.dec_src[2], p.dec_src[3]};
@@ -468,7 +473,7 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     }
 
     if constexpr (NAMED) {
-        // ---- fused weight decode: this CTA's share of the code words, in chunks of GT * 8 ---
+        // ---- fused weight decode: this CTA's share of the code words, in chunks of GTP * 8 --
         if (p.wdec_groups > 0) {
             const long long dlo = (long long)blockIdx.x * p.wdec_groups / gridDim.x;
             const long long dcnt = ((long long)blockIdx.x + 1) * p.wdec_groups / gridDim.x - dlo;
@@ -479,19 +484,19 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
                 if (g == 0)
                     sched[17 + grp] = atomicAdd(&sched[16], 1);
                 group_sync();
-                const long long c0 = (long long)sched[17 + grp] * GT * kU;
+                const long long c0 = (long long)sched[17 + grp] * GTP * kU;
                 group_sync();                              // read before the next claim
                 if (c0 >= dcnt)
                     break;
                 uint32_t wv[kU];
 #pragma unroll
                 for (int j = 0; j < kU; ++j) {
-                    const long long i = c0 + g + (long long)j * GT;
+                    const long long i = c0 + g + (long long)j * GTP;
                     wv[j] = i < dcnt ? __ldg(wc + i) : 0u;
                 }
 #pragma unroll
                 for (int j = 0; j < kU; ++j) {
-                    const long long i = c0 + g + (long long)j * GT;
+                    const long long i = c0 + g + (long long)j * GTP;
                     if (i < dcnt) {
                         if (p.wdec_bits == 4) {
                             uint32_t o[4];
@@ -632,9 +637,10 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
         stages = 1;
     long long ctas_needed;
     int NG;
-    const bool named = GT % 32 == 0 && !in_f32;
+    const bool named = k1_named(p.d, !in_f32);
+    const int GTP = named ? k1_group_threads(p.d) : GT;   // threads per group
     if (p.wdec_groups > 0 && !named) {
-        *why = "fused weight decode needs whole-warp groups (bf16 rows, d a multiple of 1024)";
+        *why = "fused weight decode needs the named-barrier K1 (bf16 rows, whole-warp groups)";
         return cudaErrorInvalidValue;
     }
     if (named) {
@@ -649,7 +655,7 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
         const long long share = (npairs + ctas_needed - 1) / ctas_needed;
         // registers: each of the SM's four 16K-register partitions holds 5 warps of 96
         constexpr int kWarpsPerSm = 4 * ((65536 / 4) / (96 * 32));
-        int ng_max = std::min(std::min(15, 1024 / GT), kWarpsPerSm * 32 / GT);
+        int ng_max = std::min(std::min(15, 1024 / GTP), kWarpsPerSm * 32 / GTP);
         while (ng_max > 1 && k1_smem(p, in_f32, ng_max, stages) > 220 * 1024)
             --ng_max;
         if (wdec) {
@@ -677,7 +683,7 @@ cudaError_t launch_k1(const K1Params &p_in, int bits, int h, int in_f32, cudaStr
     }
     p.groups = NG;
     p.stages = stages;
-    const int threads = NG * GT;
+    const int threads = NG * GTP;
     if (p.a16) {
         if (in_f32) {
             *why = "fp16 centroid output takes bf16 input";

@@ -814,8 +814,9 @@ namespace {
 // 32 lanes of a warp at the same step e reading positions perm[32g + e]; its bank is
 // 4 * colour + (j & 3).  A local search over colour swaps inside each octet lowers the sum
 // over (warp, step) of the largest number of lanes on one bank (for a random permutation
-// from about 3.6 to about 2.1 per load; for the identity, from 16 to 4).  Groups whose
-// threads do not fill whole warps keep colour = g & 7.
+// from about 3.6 to about 2.1 per load; for the identity, from 16 to 4).  The search runs
+// for the named-barrier K1, whose groups start at a warp (padded to whole warps); groups
+// that share warps (the lockstep K1) keep colour = g & 7.
 std::vector<uint8_t> pair_slot_colours(const std::vector<int32_t> &perm, int d) {
     const int GT = d / 32, NH = d / 4;
     std::vector<uint8_t> col(NH);
@@ -823,7 +824,7 @@ std::vector<uint8_t> pair_slot_colours(const std::vector<int32_t> &perm, int d) 
         const int c = h >> 1, g = c % GT;
         col[h] = (uint8_t)(((g & ~7) + 8 <= GT) ? ((g + (c / GT) * 3) & 7) : (g & 7));
     }
-    if (GT % 32 != 0)
+    if (!oq::k1_named(d, true))
         return col;
     // reads of each half-chunk: (event = warp * 32 + step, j & 3)
     std::vector<std::array<std::pair<int, int>, 4>> reads(NH);
@@ -832,7 +833,7 @@ std::vector<uint8_t> pair_slot_colours(const std::vector<int32_t> &perm, int d) 
         const int j = perm[i], g = i >> 5, e = i & 31;
         reads[j >> 2][nread[j >> 2]++] = {(g >> 5) * 32 + e, j & 3};
     }
-    const int NE = (GT / 32) * 32;
+    const int NE = ((GT + 31) / 32) * 32;
     std::vector<int> cnt((size_t)NE * 32, 0);
     for (int h = 0; h < NH; ++h)
         for (int t = 0; t < 4; ++t)

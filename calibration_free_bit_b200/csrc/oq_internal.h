@@ -99,9 +99,16 @@ struct K1Params {
 inline bool k1_a16_supported(int bits, int h, bool bf16_in) {
     return bf16_in && h >= 32 && h <= 256 && (bits == 2 || bits == 4 || bits == 8);
 }
-// True when K1 runs as one CTA per SM with named-barrier groups (bf16 rows, d/32 threads per
-// token pair a whole number of warps); the fused weight decode needs it.
-inline bool k1_named(int d, bool bf16_in) { return bf16_in && (d / 32) % 32 == 0; }
+// Threads of a named-barrier K1 group: the d/32 position-owning threads of a token pair,
+// padded to whole warps.
+inline int k1_group_threads(int d) { return (d / 32 + 31) & ~31; }
+// True when K1 runs as one CTA per SM with named-barrier groups: bf16 rows, and the padding
+// to whole warps leaves at most one lane in eight idle (d/32 a multiple of 32, or large
+// enough: d = 9728 and 13824 qualify, 2560 does not); the fused weight decode needs it.
+inline bool k1_named(int d, bool bf16_in) {
+    const int gt = d / 32, gtp = k1_group_threads(d);
+    return bf16_in && 8 * (gtp - gt) <= gtp;
+}
 // (4-bit additionally needs an odd-symmetric codebook, which every Lloyd-Max codebook here is;
 // the host checks it when it builds dec_src.)
 

@@ -134,6 +134,28 @@ def test_k1_every_block_size_and_bit_width(oq, h, bits):
     np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
 
 
+@pytest.mark.parametrize("d,h,bits,T", [
+    (896, 128, 4, 301),      # 28 position threads a pair: one warp, 4 padding lanes
+    (3968, 128, 2, 257),     # 124 threads: four warps, the last with 28
+    (3968, 64, 8, 64),       # fewer pairs than SMs
+    (9728, 256, 6, 101),     # the text encoder's down input: 304 threads in 10 warps
+    (13824, 128, 4, 67),     # the video FFN's down input: 432 threads in 14 warps
+])
+def test_k1_groups_padded_to_whole_warps(oq, d, h, bits, T):
+    """bf16 widths whose d/32 position threads a token pair are not a whole number of warps
+    but waste at most one lane in eight run the named-barrier K1 with each group padded to
+    whole warps (the padding lanes own no positions): codes and norms against the oracle,
+    bf16 input with outlier channels, odd T."""
+    p = synth.sweep_projection(d, 128, 4, T)
+    x = synth.activations(p)
+    r = oq.oq_build_rpbh(d, h, 0)
+    cb = oq.oq_lloyd_max(d, bits)
+    g, gs = k1_gpu(oq, r, cb, x)
+    o, os_, _, ou = k1_oracle(x, h, bits)
+    check_codes(g, o, ou, d, bits, f"d={d} h={h} b={bits}")
+    np.testing.assert_allclose(gs, os_, rtol=NORM_RTOL)
+
+
 @pytest.mark.parametrize("d,h,bits", [(128, 64, 2), (128, 128, 4), (256, 64, 8), (384, 128, 3)])
 def test_exact_marginal_codebook_k1_and_linear(oq, d, h, bits):
     """The f_d codebook (oq_lloyd_max_marginal, OQ_MARGINAL_EXACT) through K1 and the linear
@@ -490,13 +512,16 @@ def test_k1_tensor_core_path(oq):
     (2048, 128, 2, 2, 400, 400, False, torch.float32),      # fused 2-bit weight decode
     (3072, 128, 4, 4, 17, 16, True, torch.float32),         # fused decode, odd T, GELU
     (3072, 128, 4, 4, 1, 16, False, torch.float32),         # N > T: decode beside K1
+    (3968, 128, 4, 4, 300, 256, False, torch.float32),      # fused decode, padded groups
+    (896, 64, 8, 2, 77, 48, False, torch.bfloat16),         # the same, one warp a group
 ])
 def test_quantized_linear_matches_the_two_calls(oq, d, h, ba, bw, T, N, gelu, out):
     """oq_quantized_linear (x -> y, codes never in memory) is bit-identical to
     oq_quantize_act (or _gelu) followed by oq_linear: y and the norms s.  With 2- or 4-bit
-    weights, 2/4/8-bit activations, d a multiple of 1024 up to 5120 and N <= T the weight
-    decode runs inside K1 (also when there are fewer token pairs than SMs); the other rows take
-    the side-stream decode."""
+    weights, 2/4/8-bit activations, the named-barrier K1 (d/32 threads a pair in whole warps,
+    or padded to them), d <= 5120 and N <= T the weight
+    decode runs inside K1 (also when there are fewer token pairs than SMs, and with groups
+    padded to whole warps); the other rows take the side-stream decode."""
     p = synth.sweep_projection(d, 128, 4, T) if d != 3072 or T != 4608 else \
         synth.get("flux_attn_w4a4")[0]
     x = synth.activations(p).cuda()

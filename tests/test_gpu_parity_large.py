@@ -1,5 +1,6 @@
 """GPU parity at the large workloads: the video-DiT FFN (both projections, both bit settings),
-the activation sweep's (d, h, bits) grid, the widths whose K1 runs the lockstep schedule, and
+the activation sweep's (d, h, bits) grid, the widths whose token-pair groups do not fill whole
+warps (padded named groups, or the lockstep schedule), and
 the one-call path (oq_quantized_linear) against the fp64 oracle directly.
 
 Same bars as test_gpu_parity (rcap.io OrbitQuant summary, pseudocode block): codes >= 99.99 %
@@ -75,7 +76,7 @@ def count_checked(gpu_packed, orc_packed, orc_u, d, bits, what):
 
 
 # ----------------------------------------------------------------------------------------
-# K1 on the video FFN and at the lockstep-schedule widths
+# K1 on the video FFN and at the widths whose groups do not fill whole warps
 # ----------------------------------------------------------------------------------------
 
 def _spread_rows(T, n, seed):
@@ -89,9 +90,11 @@ def _spread_rows(T, n, seed):
 @pytest.mark.parametrize("variant,proj,n_rows", [
     ("video_ffn_w3a4", 1, 4096),     # 13824 -> 5120 input at A4: 432 threads a token pair
     ("video_ffn_w4a8", 1, 4096),     # the same rows at A8
+    ("text_encoder_w6a6", 1, 4096),  # 9728 -> 2560 input at A6: 304 threads a token pair
 ])
-def test_k1_lockstep_widths_against_oracle(oq, variant, proj, n_rows):
-    """Widths whose d/32 threads a token pair do not fill whole warps run K1's lockstep
+def test_k1_partial_warp_widths_against_oracle(oq, variant, proj, n_rows):
+    """Widths whose d/32 threads a token pair do not fill whole warps: d = 13824 and 9728
+    run the named-barrier K1 with groups padded to whole warps, d = 2560 (below) the lockstep
     schedule.  All rows are quantized on the GPU in one launch (the benchmark's
     configuration); n_rows of them, spread over the batch, are compared with the oracle, and
     every norm with ||x|| (R is orthogonal)."""
@@ -128,8 +131,9 @@ def test_linear_video_ffn_down_full_size(oq, variant):
     ("text_encoder_w6a6", 0, 4096),  # d = 2560: 80 threads a token pair
 ])
 def test_k1_lockstep_width_2560_against_oracle(oq, variant, proj, n_rows):
-    """As test_k1_lockstep_widths_against_oracle, at d = 2560 (6-bit codes)."""
-    test_k1_lockstep_widths_against_oracle(oq, variant, proj, n_rows)
+    """As test_k1_partial_warp_widths_against_oracle, at d = 2560 (6-bit codes), which runs
+    the lockstep schedule (80 threads a pair: padding to 96 would idle one lane in six)."""
+    test_k1_partial_warp_widths_against_oracle(oq, variant, proj, n_rows)
 
 
 def test_k1_video_ffn_up_w4a8_every_row(oq):
