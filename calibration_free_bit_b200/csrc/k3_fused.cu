@@ -17,9 +17,10 @@
 //     token pairs taken from a global counter, writing each code's fp16 unit centroid into
 //     the GEMM's A operand and the norms s, and publishing, per block of 256 rows, how many
 //     rows are done (release add at GPU scope after a proxy fence);
-//   * first of all, every quantize and epilogue warp takes chunks of the 2- or 4-bit weight
-//     codes from a global counter and decodes them into the fp16 B operand (one proxy fence
-//     and one count per warp); the GEMM producers wait for the count once.
+//   * first of all, the GEMM warps decode the 2- or 4-bit weight codes into the fp16 B operand
+//     (a static share a warp, one proxy fence and one count a warp; the producers wait for the
+//     count once), and then, as ramp groups of d/32 threads with their buffers in the stage
+//     ring, quantize a few token pairs each before they take up their GEMM roles.
 // A GEMM producer loads a tile's A rows only once their block's count is complete (acquire
 // load, then a proxy fence before the TMA); the epilogue acquires the same count before it
 // reads s.  The quantize groups never wait on the GEMM, and any CTA's group can take any
@@ -82,36 +83,28 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-constexpr int kDecWordsPerLane = 8;      // weight-decode chunk: 32 lanes x 8 code words
-constexpr long long kDecChunk = 32 * kDecWordsPerLane;
+constexpr int kDecBatch = 16;            // weight-code words a lane holds at once
 
-__device__ __forceinline__ unsigned wdec_chunks(const FusedStepParams &p) {
-    return (unsigned)((p.wdec_words + kDecChunk - 1) / kDecChunk);
-}
-
-// The kernel's first task for every quantize and epilogue warp: decode weight-code chunks taken
-// from a global counter into the fp16 B operand, then one proxy fence and one release add of
-// the warp's chunk count (for the TMA reads of B).
-__device__ __forceinline__ void decode_weight_chunks(const FusedStepParams &p, int lane) {
-    const unsigned nchunks = wdec_chunks(p);
-    unsigned done = 0;
-    for (;;) {
-        unsigned c = 0;
-        if (lane == 0)
-            c = atomicAdd(p.ctr + 2, 1u);
-        c = __shfl_sync(0xffffffffu, c, 0);
-        if (c >= nchunks)
-            break;
-        uint32_t wv[kDecWordsPerLane];
+// The GEMM warps' first task: warp wi of nw decodes its static share of the 2- or 4-bit weight
+// codes into the fp16 B operand, kDecBatch words a lane per batch with all of a batch's loads
+// issued before its stores, then one proxy fence and one release count (for the TMA reads of
+// B).
+__device__ __forceinline__ void decode_weight_share(const FusedStepParams &p, int lane,
+                                                    long long wi, long long nw) {
+    const long long per = (p.wdec_words + nw - 1) / nw;
+    const long long lo = wi * per;
+    const long long hi = min(p.wdec_words, lo + per);
+    for (long long b = lo; b < hi; b += 32 * kDecBatch) {
+        uint32_t wv[kDecBatch];
 #pragma unroll
-        for (int j = 0; j < kDecWordsPerLane; ++j) {
-            const long long i = (long long)c * kDecChunk + j * 32 + lane;
-            wv[j] = i < p.wdec_words ? __ldg(p.wcodes + i) : 0u;
+        for (int j = 0; j < kDecBatch; ++j) {
+            const long long i = b + j * 32 + lane;
+            wv[j] = i < hi ? __ldg(p.wcodes + i) : 0u;
         }
 #pragma unroll
-        for (int j = 0; j < kDecWordsPerLane; ++j) {
-            const long long i = (long long)c * kDecChunk + j * 32 + lane;
-            if (i >= p.wdec_words)
+        for (int j = 0; j < kDecBatch; ++j) {
+            const long long i = b + j * 32 + lane;
+            if (i >= hi)
                 continue;
             if (p.wdec_bits == 4) {
                 uint32_t o[4];
@@ -126,24 +119,22 @@ __device__ __forceinline__ void decode_weight_chunks(const FusedStepParams &p, i
                 p.b16[2 * i + 1] = make_uint4(q2.x, q2.y, q3.x, q3.y);
             }
         }
-        ++done;
     }
     fence_proxy_async_global();
     __syncwarp();
-    if (lane == 0 && done > 0)
-        red_release_add(p.ctr + 3, done);
+    if (lane == 0)
+        red_release_add(p.ctr + 3, 1u);
 }
 
-// Wait until every weight-decode chunk is written (no wait when the weights were decoded before
-// the launch); false after the wait limit.
-__device__ __forceinline__ bool wait_weights(const FusedStepParams &p) {
-    const unsigned need = wdec_chunks(p);
-    if (need == 0 || ld_acquire(p.ctr + 3) >= need)
+// Wait until all nw decoding warps have counted themselves (no wait when the weights were
+// decoded before the launch); false after the wait limit.
+__device__ __forceinline__ bool wait_weights(const FusedStepParams &p, unsigned nw) {
+    if (p.wdec_words == 0 || ld_acquire(p.ctr + 3) >= nw)
         return true;
     const long long t0 = clock64();
     for (;;) {
         __nanosleep(256);
-        if (ld_acquire(p.ctr + 3) >= need)
+        if (ld_acquire(p.ctr + 3) >= nw)
             return true;
         if (clock64() - t0 > kWaitCycles)
             return false;
@@ -166,6 +157,236 @@ __device__ __forceinline__ bool wait_rows(const FusedStepParams &p, int b) {
     }
 }
 
+// One quantize group's working memory: norm partials (two rounds), barriers ([0] the row
+// stage, [1] the table images (the first permanent group's), [2] the armed test wait), pair
+// scheduling words, the raw rows of a pair and the interleaved pair.
+struct QGroup {
+    float2 *red;
+    unsigned long long *bars;
+    int *sched;
+    unsigned char *raw;
+    unsigned char *pairs;
+};
+constexpr size_t kQSmallBytes = sizeof(float2) * 2 * kMaxSeg + 8 * 4 + 4 * 8;
+
+// The quantize stage of one group of GT = d/32 threads (g = 0 .. GT-1, named barrier bar_id):
+// token pairs from the global counter -> fp16 A rows and s, each finished pair's rows counted
+// in its 256-row block (proxy fence, then release add).  At most max_rounds pairs; on its last
+// round the group takes no further pair, so no copy is in flight when it returns.
+template <int BITS, int H>
+__device__ __forceinline__ void quantize_rounds(const FusedStepParams &p, const QGroup &q, int g,
+                                                int GT, int bar_id, const uint32_t *table,
+                                                const uint32_t *gent, const uint32_t *dect,
+                                                uint32_t setup_bar, int max_rounds) {
+    constexpr int Q = H / kE;                        // threads per h-block
+    constexpr int TSH = BITS <= 4 ? 7 : 2;           // per-lane table copies for <= 4 bits
+    constexpr int NW = kE * BITS / 32;
+    const int lane = (int)threadIdx.x & 31;
+    const int d = p.d;
+    const uint32_t row_in = (uint32_t)d * 2;
+    const long long npairs = ((long long)p.T + 1) / 2;
+    auto group_sync = [&]() {
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(GT) : "memory");
+    };
+    const uint32_t row_bar = smem_u32(&q.bars[0]);
+    const int r = g % Q;
+    const int pos0 = g * kE;
+    const uint4 *myent = reinterpret_cast<const uint4 *>(gent + g * kK1EntStride);
+    const uint32_t tbl_lane = smem_u32(table) + (BITS <= 4 ? lane * 4 : 0) -
+                              ((0x3F800000u >> p.F) << TSH);
+    const uint32_t G = (uint32_t)p.G;
+    const int F = p.F;
+    const int seg_end = min(32, lane + (GT - g));
+    const bool seg_head = lane == 0;
+    const int seg_slot = g >> 5;
+    const int nslots = (GT + 31) >> 5;
+    // the two rows of pair pr into the raw stage (the group's first thread issues)
+    auto issue = [&](long long pr) {
+        if (g != 0 || pr >= npairs)
+            return;
+        const long long t0 = 2 * pr;
+        const bool two = t0 + 1 < p.T;
+        mbar_expect_tx(row_bar, two ? 2 * row_in : row_in);
+        bulk_copy(smem_u32(q.raw), p.x + t0 * row_in, row_in, row_bar);
+        if (two)
+            bulk_copy(smem_u32(q.raw) + row_in, p.x + (t0 + 1) * row_in, row_in, row_bar);
+    };
+    if (g == 0) {
+        const int first = max_rounds > 0 ? (int)atomicAdd(p.ctr + 0, 1u) : (int)npairs;
+        q.sched[0] = first;
+        issue(first);
+    }
+    if (!mbar_wait(setup_bar, 0))
+        atomicOr(&g_k3_err, K3_ERR_COPY);
+    group_sync();
+    long long pr = q.sched[0];
+    // Rows of a round are published one round later: the proxy fence that must precede
+    // the count then finds the stores long done instead of waiting for them.
+    int pend_block = -1;
+    unsigned pend_rows = 0;
+    for (int round = 0; pr < npairs; ++round) {
+        bool valid = true;
+        if (!mbar_wait(row_bar, (uint32_t)round & 1u)) {
+            atomicOr(&g_k3_err, K3_ERR_COPY);
+            valid = false;
+        }
+        const long long t0 = 2 * pr, t1 = t0 + 1;
+        const bool has1 = valid && t1 < p.T;
+        // ---- interleave the staged rows into the pair buffer ----
+        if (valid) {
+            const uint4 *r0 = reinterpret_cast<const uint4 *>(q.raw);
+            const uint4 *r1 = reinterpret_cast<const uint4 *>(q.raw + row_in);
+            uint4 *slots = reinterpret_cast<uint4 *>(q.pairs);
+            const uint4 sl = myent[kE / 4];
+            const uint32_t slw[4] = {sl.x, sl.y, sl.z, sl.w};
+#pragma unroll
+            for (int k = 0; k < kE / 8; ++k) {
+                const int c = g + k * GT;
+                const uint4 a = r0[c], b = r1[c];
+                slots[slw[k] & 0xffffu] =
+                    make_uint4(prmt_b32(a.x, b.x, 0x5410), prmt_b32(a.x, b.x, 0x7632),
+                               prmt_b32(a.y, b.y, 0x5410), prmt_b32(a.y, b.y, 0x7632));
+                slots[slw[k] >> 16] =
+                    make_uint4(prmt_b32(a.z, b.z, 0x5410), prmt_b32(a.z, b.z, 0x7632),
+                               prmt_b32(a.w, b.w, 0x5410), prmt_b32(a.w, b.w, 0x7632));
+            }
+        }
+        group_sync();
+        if (pend_rows)
+            fence_proxy_async_global();            // the previous round's rows
+        // the raw stage is free: take the next pair (none after the last allowed round) and
+        // start its copy
+        if (g == 0) {
+            const int nx = round + 1 < max_rounds ? (int)atomicAdd(p.ctr + 0, 1u) : (int)npairs;
+            q.sched[1 + (round & 1)] = nx;
+            issue(nx);
+        }
+        // ---- gather y[i] = sign[i] x[perm[i]] for both tokens ----
+        float2 v[kE];
+        {
+            const uint32_t base0 = smem_u32(q.pairs);
+#pragma unroll
+            for (int e4 = 0; e4 < kE / 4; ++e4) {
+                const uint4 q4 = myent[e4];
+                const uint32_t en4[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t en = en4[i];
+                    const uint32_t sg = en & 0x80000000u;
+                    const uint32_t w = lds32(base0 + (en & 0x7fffffffu));
+                    v[4 * e4 + i].x = __uint_as_float((w << 16) + sg);
+                    v[4 * e4 + i].y = __uint_as_float((w ^ en) & 0xffff0000u);
+                }
+            }
+        }
+        // ---- block Walsh-Hadamard (natural order), unnormalised ----
+#pragma unroll
+        for (int s = 1; s < kE; s <<= 1) {
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                if ((e & s) == 0) {
+                    const float2 a = v[e], b = v[e + s];
+                    v[e] = f2add(a, b);
+                    v[e + s] = f2sub(a, b);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 1; m < Q; m <<= 1) {
+            const float sgn = (r & m) ? -1.0f : 1.0f;
+            const float2 sg2 = make_float2(sgn, sgn);
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                float2 o;
+                o.x = __shfl_xor_sync(0xffffffffu, v[e].x, m);
+                o.y = __shfl_xor_sync(0xffffffffu, v[e].y, m);
+                v[e] = f2fma(sg2, v[e], o);
+            }
+        }
+        // ---- per-token sum of squares over the group ----
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < kE; ++e)
+            acc = f2fma(v[e], v[e], acc);
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            float2 o;
+            o.x = __shfl_down_sync(0xffffffffu, acc.x, off);
+            o.y = __shfl_down_sync(0xffffffffu, acc.y, off);
+            if (lane + off < seg_end) {
+                acc.x += o.x;
+                acc.y += o.y;
+            }
+        }
+        if (seg_head)
+            q.red[(round & 1) * kMaxSeg + seg_slot] = acc;
+        group_sync();
+        if (g == 0 && pend_rows)
+            red_release_add(p.ctr + 4 + pend_block, pend_rows);
+        const float2 *myred = q.red + (round & 1) * kMaxSeg;
+        const long long nxt = q.sched[1 + (round & 1)];
+        float2 ss = myred[0];
+        for (int i = 1; i < nslots; ++i) {
+            const float2 o = myred[i];
+            ss.x += o.x;
+            ss.y += o.y;
+        }
+        const float s0 = sqrtf(ss.x * (1.0f / H));
+        const float s1 = sqrtf(ss.y * (1.0f / H));
+        const float m0 = (s0 + p.eps > 0.f) ? p.K / (s0 + p.eps) : 0.f;
+        const float m1 = (s1 + p.eps > 0.f) ? p.K / (s1 + p.eps) : 0.f;
+        // ---- nearest centroid, packed codes in registers ----
+        uint32_t w0[NW], w1[NW];
+        {
+            constexpr int PER = 32 / BITS;
+#pragma unroll
+            for (int wi = 0; wi < NW; ++wi) {
+                uint32_t d0[PER], d1[PER];
+#pragma unroll
+                for (int k = 0; k < PER; ++k) {
+                    const float2 vv = v[wi * PER + k];
+                    const float a0 = fma_sat(vv.x, m0, 0.5f);
+                    const float a1 = fma_sat(vv.y, m1, 0.5f);
+                    const uint2 qb = f2_add_one_rm_bits(a0, a1);
+                    d0[k] = qb.x * G + lds32(tbl_lane + ((qb.x >> F) << TSH));
+                    d1[k] = qb.y * G + lds32(tbl_lane + ((qb.y >> F) << TSH));
+                }
+                w0[wi] = pack_codes<BITS>(d0);
+                w1[wi] = pack_codes<BITS>(d1);
+            }
+        }
+        // ---- fp16 centroids into the A operand, norms, then publish the rows ----
+        if (valid) {
+            uint4 *a0 = reinterpret_cast<uint4 *>(p.a16 + t0 * d + pos0);
+            decode_store<BITS>(dect, w0, a0, p.dec_src);
+            if (has1)
+                decode_store<BITS>(dect, w1, a0 + d / 8, p.dec_src);
+            if (g == 0) {
+                p.s[t0] = s0;
+                if (has1)
+                    p.s[t1] = s1;
+            }
+        }
+        pend_block = (int)(t0 / 256);
+        pend_rows = valid ? (has1 ? 2u : 1u) : 0u;
+        if (round == 0 && pend_rows) {
+            // the first rows open the GEMM's first tiles: publish them at once
+            fence_proxy_async_global();
+            group_sync();
+            if (g == 0)
+                red_release_add(p.ctr + 4 + pend_block, pend_rows);
+            pend_rows = 0;
+        }
+        pr = nxt;
+    }
+    if (pend_rows) {                             // the last round's rows
+        fence_proxy_async_global();
+        group_sync();
+        if (g == 0)
+            red_release_add(p.ctr + 4 + pend_block, pend_rows);
+    }
+}
+
 // one epilogue staging chunk per warp (the stores of a tile overlap the next tile's mainloop
 // through the second TMEM accumulator, so a second staging buffer buys little here and its
 // 16 KB go to a second quantize group)
@@ -175,14 +396,29 @@ __host__ __device__ constexpr size_t gemm_bytes() {
 
 // shared memory: [GEMM stages + staging: 1 KB aligned][GEMM barriers][scalars, ring, norms]
 // [quantize: table | entries | decode table | partials | barriers | sched | raw rows | pairs]
-constexpr int kGemmBars = 2 * kS + 5 + 2 * kTileRing;
+constexpr int kGemmBars = 2 * kS + 5 + 2 * kTileRing + 1;   // + the ramp barrier
 constexpr size_t kBarsBytes = (8 * kGemmBars + 15) & ~(size_t)15;
 // scalars: TMEM base and abort flag (16 bytes), the tile-id ring, then the epilogue's
-// row-norm chunks (read as float4: 16-byte aligned)
+// row-norm chunks (read as float4: 16-byte aligned), then the small regions of the ramp
+// groups (their rows and pairs live in the GEMM's stage ring until the ramp ends)
+constexpr int kMaxRamp = kGemmThreads / 32;
 constexpr size_t kRnOffset = 16 + ((4 * kTileRing + 15) & ~(size_t)15);
-constexpr size_t kMiscBytes = kRnOffset + kEpi * 64 * 4;
-static_assert(kBarsBytes % 16 == 0 && kRnOffset % 16 == 0 && kMiscBytes % 16 == 0,
-              "16-byte aligned regions");
+constexpr size_t kRampOffset = kRnOffset + kEpi * 64 * 4;
+constexpr size_t kMiscBytes = kRampOffset + kMaxRamp * kQSmallBytes;
+static_assert(kBarsBytes % 16 == 0 && kRnOffset % 16 == 0 && kRampOffset % 16 == 0 &&
+              kQSmallBytes % 16 == 0 && kMiscBytes % 16 == 0, "16-byte aligned regions");
+
+// Ramp groups: before their GEMM roles, the GEMM warps form groups of d/32 threads that
+// quantize a few token pairs each (the GEMM's first wave needs many row blocks at once), with
+// their rows and pairs in the stage ring (8d bytes a group).
+__host__ __device__ inline int ramp_groups(int d, int ramp_rounds) {
+    const int gt = d / kE;
+    if (ramp_rounds <= 0 || gt > kGemmThreads)
+        return 0;
+    const int by_threads = kGemmThreads / gt;
+    const int by_ring = (int)(((size_t)kS * 2 * kAB) / ((size_t)8 * d));
+    return by_threads < by_ring ? by_threads : by_ring;
+}
 
 // per group: norm partials (two rounds), 4 barriers, 8 scheduling words, raw rows, pairs
 size_t quant_group_bytes(int d) {
@@ -218,12 +454,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     const uint32_t drain_bar = bars + 8u * (2 * kS + 4);
     auto idfull_bar = [&](int r) { return bars + 8u * (2 * kS + 5 + r); };
     auto idempty_bar = [&](int r) { return bars + 8u * (2 * kS + 5 + kTileRing + r); };
+    const uint32_t ramp_bar = bars + 8u * (2 * kS + 5 + 2 * kTileRing);
     unsigned char *miscp = basep + (bars + (uint32_t)kBarsBytes - base);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(miscp);
     int *abort_flag = reinterpret_cast<int *>(miscp + 4);
     int *ring = reinterpret_cast<int *>(miscp + 16);
     const uint32_t ring_addr = smem_u32(ring);
     float *rn_s = reinterpret_cast<float *>(miscp + kRnOffset);
+    unsigned char *rampsmall = miscp + kRampOffset;
     unsigned char *qbase = miscp + kMiscBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -234,6 +472,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     const int GT = p.d / kE;
     const int NQ = ((int)blockDim.x - kGemmThreads) / GT;     // quantize groups
     const int qgrp = threadIdx.x >= kGemmThreads ? ((int)threadIdx.x - kGemmThreads) / GT : 0;
+    const int NR = ramp_groups(p.d, p.ramp_rounds);           // ramp groups
+    auto ramp_group = [&](int rg) {
+        unsigned char *sm = rampsmall + (size_t)rg * kQSmallBytes;
+        float2 *rred = reinterpret_cast<float2 *>(sm);
+        unsigned long long *rbars = reinterpret_cast<unsigned long long *>(rred + 2 * kMaxSeg);
+        int *rsched = reinterpret_cast<int *>(rbars + 4);
+        unsigned char *rraw = basep + (sA - base) + (size_t)rg * 8 * p.d;
+        return QGroup{rred, rbars, rsched, rraw, rraw + (size_t)4 * p.d};
+    };
 
     // quantize-stage shared memory: shared tables, then one region per group
     uint32_t *table = reinterpret_cast<uint32_t *>(qbase);
@@ -250,6 +497,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     // the table images land once per CTA, on group 0's setup barrier
     unsigned long long *qbars0 = reinterpret_cast<unsigned long long *>(
         reinterpret_cast<unsigned char *>(dect + p.dec_words) + sizeof(float2) * 2 * kMaxSeg);
+    const uint32_t setup_bar = smem_u32(&qbars0[1]);
 
     pdl_trigger();
     if (threadIdx.x == 0) {
@@ -278,6 +526,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
             mbar_init(smem_u32(&b[1]), 1);         // table images (group 0's)
             mbar_init(smem_u32(&b[2]), 2);         // armed test wait (group 0's)
         }
+        for (int q = 0; q < NR; ++q)
+            mbar_init(smem_u32(&ramp_group(q).bars[0]), 1);   // a ramp group's row stage
+        mbar_init(ramp_bar, NR > 0 ? NR : 1);               // every ramp group is done
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         *abort_flag = 0;
     }
@@ -297,10 +548,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         atomicExch(abort_flag, 1);
     };
 
+    // ---------------- ramp (the GEMM warps, before their roles) ----------------
+    // Every GEMM warp decodes a share of the 2/4-bit weight codes.  The warps of the ramp
+    // groups then quantize up to ramp_rounds token pairs a group with their rows and pairs in
+    // the stage ring, order their shared-memory accesses before the async proxy's, and count
+    // their group on ramp_bar; the producers wait for it before their first TMA load.
+    if (warp < 2 + kEpi) {
+        if (p.wdec_words > 0)
+            decode_weight_share(p, lane, (long long)blockIdx.x * (2 + kEpi) + warp,
+                                (long long)gridDim.x * (2 + kEpi));
+        if ((int)threadIdx.x < NR * GT) {
+            const int rg = (int)threadIdx.x / GT, g = (int)threadIdx.x - rg * GT;
+            const int bar_id = 1 + kMaxGroups + rg;
+            quantize_rounds<BITS, H>(p, ramp_group(rg), g, GT, bar_id, table, gent, dect,
+                                     setup_bar, p.ramp_rounds);
+            fence_async_smem();
+            asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(GT) : "memory");
+            if (g == 0)
+                mbar_arrive(ramp_bar);
+        }
+    }
+
     if (warp == 0) {
         // ---------------- tile scheduler (leader) and TMA producer (both CTAs) -------------
         if (lane == 0) {
             uint32_t it = 0;
+            if (NR > 0 && !mbar_wait(ramp_bar, 0))
+                give_up(K3_ERR_STAGE);             // the ring may still be in use: load nothing
             for (int i = 0;; ++i) {
                 const int r = i % kTileRing;
                 const uint32_t par = (uint32_t)(i / kTileRing) & 1u;
@@ -333,7 +607,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
                 const int mb = tile / n_tiles;
                 const int m0 = mb * 256 + (int)rank * 128;
                 const int n0 = (tile % n_tiles) * 256 + (int)rank * 128;
-                if ((i == 0 && !wait_weights(p)) || !wait_rows(p, mb)) {
+                if ((i == 0 && !wait_weights(p, gridDim.x * (2 + kEpi))) || !wait_rows(p, mb)) {
                     give_up(K3_ERR_ROWS);
                     break;
                 }
@@ -413,9 +687,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     } else if (warp < 2 + kEpi) {
         // ---------------- epilogue (both CTAs) ----------------
         const int q = warp & 3;
-        // until the first accumulator is ready: a share of the weight decode
-        if (p.wdec_words > 0)
-            decode_weight_chunks(p, lane);
         float *rn_w = rn_s + (warp - 2) * 64;
         const uint32_t out0 = sOut + (uint32_t)((warp - 2) * kOut);
         unsigned char *out0p = basep + (out0 - base);
@@ -501,18 +772,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         if (lane == 0)
             bulk_wait_all();
     } else {
-        // ---------------- quantize group: token pairs -> fp16 A rows and s ----------------
-        constexpr int Q = H / kE;                        // threads per h-block
-        constexpr int TSH = BITS <= 4 ? 7 : 2;           // per-lane table copies for <= 4 bits
-        constexpr int NW = kE * BITS / 32;
+        // ---------------- permanent quantize group ----------------
         const int g = (int)threadIdx.x - kGemmThreads - qgrp * GT;   // 0 .. GT-1
-        const int d = p.d;
-        const uint32_t row_in = (uint32_t)d * 2;
-        const long long npairs = ((long long)p.T + 1) / 2;
-        auto group_sync = [&]() {
-            asm volatile("bar.sync %0, %1;" ::"r"(1 + qgrp), "r"(GT) : "memory");
-        };
-        const uint32_t row_bar = smem_u32(&qbars[0]), setup_bar = smem_u32(&qbars0[1]);
         if (g == 0 && qgrp == 0) {
             mbar_expect_tx(setup_bar, 4u * (p.tbl_words + p.ent_words + p.dec_words));
             bulk_copy(smem_u32(table), p.tbl_img, 4u * p.tbl_words, setup_bar);
@@ -520,204 +781,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
             if (p.dec_words > 0)
                 bulk_copy(smem_u32(dect), p.dec_img, 4u * p.dec_words, setup_bar);
         }
-        const int r = g % Q;
-        const int pos0 = g * kE;
-        const uint4 *myent = reinterpret_cast<const uint4 *>(gent + g * kK1EntStride);
-        const uint32_t tbl_lane = smem_u32(table) + (BITS <= 4 ? lane * 4 : 0) -
-                                  ((0x3F800000u >> p.F) << TSH);
-        const uint32_t G = (uint32_t)p.G;
-        const int F = p.F;
-        const int seg_end = min(32, lane + (GT - g));
-        const bool seg_head = lane == 0;
-        const int seg_slot = g >> 5;
-        const int nslots = (GT + 31) >> 5;
-        // the two rows of pair pr into the raw stage (the group's first thread issues)
-        auto issue = [&](long long pr) {
-            if (g != 0 || pr >= npairs)
-                return;
-            const long long t0 = 2 * pr;
-            const bool two = t0 + 1 < p.T;
-            mbar_expect_tx(row_bar, two ? 2 * row_in : row_in);
-            bulk_copy(smem_u32(qraw), p.x + t0 * row_in, row_in, row_bar);
-            if (two)
-                bulk_copy(smem_u32(qraw) + row_in, p.x + (t0 + 1) * row_in, row_in, row_bar);
-        };
-        if (g == 0) {
-            const int first = (int)atomicAdd(p.ctr + 0, 1u);
-            qsched[0] = first;
-            issue(first);
-        }
-        // the first pair's rows stream in while this group takes a share of the weight decode
-        if (p.wdec_words > 0)
-            decode_weight_chunks(p, lane);
-        if (!mbar_wait(setup_bar, 0))
-            atomicOr(&g_k3_err, K3_ERR_COPY);
-        group_sync();
-        long long pr = qsched[0];
-        // Rows of a round are published one round later: the proxy fence that must precede
-        // the count then finds the stores long done instead of waiting for them.
-        int pend_block = -1;
-        unsigned pend_rows = 0;
-        for (int round = 0; pr < npairs; ++round) {
-            bool valid = true;
-            if (!mbar_wait(row_bar, (uint32_t)round & 1u)) {
-                atomicOr(&g_k3_err, K3_ERR_COPY);
-                valid = false;
-            }
-            const long long t0 = 2 * pr, t1 = t0 + 1;
-            const bool has1 = valid && t1 < p.T;
-            // ---- interleave the staged rows into the pair buffer ----
-            if (valid) {
-                const uint4 *r0 = reinterpret_cast<const uint4 *>(qraw);
-                const uint4 *r1 = reinterpret_cast<const uint4 *>(qraw + row_in);
-                uint4 *slots = reinterpret_cast<uint4 *>(qpairs);
-                const uint4 sl = myent[kE / 4];
-                const uint32_t slw[4] = {sl.x, sl.y, sl.z, sl.w};
-#pragma unroll
-                for (int k = 0; k < kE / 8; ++k) {
-                    const int c = g + k * GT;
-                    const uint4 a = r0[c], b = r1[c];
-                    slots[slw[k] & 0xffffu] =
-                        make_uint4(prmt_b32(a.x, b.x, 0x5410), prmt_b32(a.x, b.x, 0x7632),
-                                   prmt_b32(a.y, b.y, 0x5410), prmt_b32(a.y, b.y, 0x7632));
-                    slots[slw[k] >> 16] =
-                        make_uint4(prmt_b32(a.z, b.z, 0x5410), prmt_b32(a.z, b.z, 0x7632),
-                                   prmt_b32(a.w, b.w, 0x5410), prmt_b32(a.w, b.w, 0x7632));
-                }
-            }
-            group_sync();
-            if (pend_rows)
-                fence_proxy_async_global();            // the previous round's rows
-            // the raw stage is free: take the next pair and start its copy
-            if (g == 0) {
-                const int nx = (int)atomicAdd(p.ctr + 0, 1u);
-                qsched[1 + (round & 1)] = nx;
-                issue(nx);
-            }
-            // ---- gather y[i] = sign[i] x[perm[i]] for both tokens ----
-            float2 v[kE];
-            {
-                const uint32_t base0 = smem_u32(qpairs);
-#pragma unroll
-                for (int e4 = 0; e4 < kE / 4; ++e4) {
-                    const uint4 q4 = myent[e4];
-                    const uint32_t en4[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t en = en4[i];
-                        const uint32_t sg = en & 0x80000000u;
-                        const uint32_t w = lds32(base0 + (en & 0x7fffffffu));
-                        v[4 * e4 + i].x = __uint_as_float((w << 16) + sg);
-                        v[4 * e4 + i].y = __uint_as_float((w ^ en) & 0xffff0000u);
-                    }
-                }
-            }
-            // ---- block Walsh-Hadamard (natural order), unnormalised ----
-#pragma unroll
-            for (int s = 1; s < kE; s <<= 1) {
-#pragma unroll
-                for (int e = 0; e < kE; ++e) {
-                    if ((e & s) == 0) {
-                        const float2 a = v[e], b = v[e + s];
-                        v[e] = f2add(a, b);
-                        v[e + s] = f2sub(a, b);
-                    }
-                }
-            }
-#pragma unroll
-            for (int m = 1; m < Q; m <<= 1) {
-                const float sgn = (r & m) ? -1.0f : 1.0f;
-                const float2 sg2 = make_float2(sgn, sgn);
-#pragma unroll
-                for (int e = 0; e < kE; ++e) {
-                    float2 o;
-                    o.x = __shfl_xor_sync(0xffffffffu, v[e].x, m);
-                    o.y = __shfl_xor_sync(0xffffffffu, v[e].y, m);
-                    v[e] = f2fma(sg2, v[e], o);
-                }
-            }
-            // ---- per-token sum of squares over the group ----
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int e = 0; e < kE; ++e)
-                acc = f2fma(v[e], v[e], acc);
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                float2 o;
-                o.x = __shfl_down_sync(0xffffffffu, acc.x, off);
-                o.y = __shfl_down_sync(0xffffffffu, acc.y, off);
-                if (lane + off < seg_end) {
-                    acc.x += o.x;
-                    acc.y += o.y;
-                }
-            }
-            if (seg_head)
-                red[(round & 1) * kMaxSeg + seg_slot] = acc;
-            group_sync();
-            if (g == 0 && pend_rows)
-                red_release_add(p.ctr + 4 + pend_block, pend_rows);
-            const float2 *myred = red + (round & 1) * kMaxSeg;
-            const long long nxt = qsched[1 + (round & 1)];
-            float2 ss = myred[0];
-            for (int i = 1; i < nslots; ++i) {
-                const float2 o = myred[i];
-                ss.x += o.x;
-                ss.y += o.y;
-            }
-            const float s0 = sqrtf(ss.x * (1.0f / H));
-            const float s1 = sqrtf(ss.y * (1.0f / H));
-            const float m0 = (s0 + p.eps > 0.f) ? p.K / (s0 + p.eps) : 0.f;
-            const float m1 = (s1 + p.eps > 0.f) ? p.K / (s1 + p.eps) : 0.f;
-            // ---- nearest centroid, packed codes in registers ----
-            uint32_t w0[NW], w1[NW];
-            {
-                constexpr int PER = 32 / BITS;
-#pragma unroll
-                for (int wi = 0; wi < NW; ++wi) {
-                    uint32_t d0[PER], d1[PER];
-#pragma unroll
-                    for (int k = 0; k < PER; ++k) {
-                        const float2 vv = v[wi * PER + k];
-                        const float a0 = fma_sat(vv.x, m0, 0.5f);
-                        const float a1 = fma_sat(vv.y, m1, 0.5f);
-                        const uint2 qb = f2_add_one_rm_bits(a0, a1);
-                        d0[k] = qb.x * G + lds32(tbl_lane + ((qb.x >> F) << TSH));
-                        d1[k] = qb.y * G + lds32(tbl_lane + ((qb.y >> F) << TSH));
-                    }
-                    w0[wi] = pack_codes<BITS>(d0);
-                    w1[wi] = pack_codes<BITS>(d1);
-                }
-            }
-            // ---- fp16 centroids into the A operand, norms, then publish the rows ----
-            if (valid) {
-                uint4 *a0 = reinterpret_cast<uint4 *>(p.a16 + t0 * d + pos0);
-                decode_store<BITS>(dect, w0, a0, p.dec_src);
-                if (has1)
-                    decode_store<BITS>(dect, w1, a0 + d / 8, p.dec_src);
-                if (g == 0) {
-                    p.s[t0] = s0;
-                    if (has1)
-                        p.s[t1] = s1;
-                }
-            }
-            pend_block = (int)(t0 / 256);
-            pend_rows = valid ? (has1 ? 2u : 1u) : 0u;
-            if (round == 0 && pend_rows) {
-                // the first rows open the GEMM's first tiles: publish them at once
-                fence_proxy_async_global();
-                group_sync();
-                if (g == 0)
-                    red_release_add(p.ctr + 4 + pend_block, pend_rows);
-                pend_rows = 0;
-            }
-            pr = nxt;
-        }
-        if (pend_rows) {                         // the last round's rows
-            fence_proxy_async_global();
-            group_sync();
-            if (g == 0)
-                red_release_add(p.ctr + 4 + pend_block, pend_rows);
-        }
+        const QGroup qgp{red, qbars, qsched, qraw, qpairs};
+        quantize_rounds<BITS, H>(p, qgp, g, GT, 1 + qgrp, table, gent, dect, setup_bar,
+                                 0x7fffffff);
         if (p.test_wait_cycles > 0 && blockIdx.x == 0 && g == 0 && qgrp == 0) {
             const uint32_t tb = smem_u32(&qbars[2]);
             mbar_arrive(tb);

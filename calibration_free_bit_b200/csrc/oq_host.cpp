@@ -694,6 +694,18 @@ bool fused_step_requested() {
     return v;
 }
 
+// Token pairs each ramp group of the fused step quantizes before its GEMM roles
+// (OQ_FUSED_RAMP = 0..8, read once per process; 0, no ramp groups, unless set).
+int fused_ramp_rounds() {
+    static const int v = [] {
+        const char *e = std::getenv("OQ_FUSED_RAMP");
+        if (e == nullptr || e[0] < '0' || e[0] > '8' || e[1] != '\0')
+            return 0;
+        return e[0] - '0';
+    }();
+    return v;
+}
+
 // oq_quantized_linear as one persistent kernel: the decode prepass of the weights, then the
 // quantize stage and the CTA-pair GEMM side by side (k3_fused.cu).  Arguments validated by
 // the caller.
@@ -783,6 +795,7 @@ int fused_step(const oq_rpbh *r, const oq_codebook *ca, const oq_codebook *cw, c
         p.inv_d = 1.0f / (float)d;
         p.ctr = ctr;
         p.test_wait_cycles = take_armed(OQ_KERNEL_GEMM);
+        p.ramp_rounds = fused_ramp_rounds();
         e = timed(OQ_KERNEL_FUSED, st, [&] {
             return oq::launch_fused_step(p, ca->bits, r->h, out_dtype == OQ_BF16, B16, y, st,
                                          &why);

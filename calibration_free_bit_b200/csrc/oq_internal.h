@@ -177,10 +177,11 @@ struct FusedStepParams {
     uint32_t wdec_src[4];               // 4-bit: byte-permute sources of the weight codebook
     const uint2 *wdec_tab;              // 2-bit: byte -> four fp16 centroids
     // progress counters, zeroed before the launch: [0] next token pair, [1] next tile,
-    // [2] next weight-decode chunk, [3] weight-decode chunks done, [4 + b] rows of 256-row
-    // block b of x done (fused_step_counter_words(T, N) words)
+    // [2] unused, [3] weight-decoding warps done, [4 + b] rows of 256-row block b of x done
+    // (fused_step_counter_words(T, N) words)
     unsigned *ctr;
     long long test_wait_cycles;
+    int ramp_rounds;                    // token pairs a ramp group quantizes (0: no ramp groups)
 };
 bool fused_step_supported(int d, int h, int bits, bool bf16_in);
 size_t fused_step_counter_words(int T, int N);

@@ -407,16 +407,19 @@ def test_fused_step_matches_the_two_calls(oq):
     and the CTA-pair GEMM side by side, rows handed over per 256-row block) equals
     oq_quantize_act + oq_linear bit for bit on every supported shape tried, ragged T and N, one
     token, bf16 y and two calls in a row; a shape outside its range takes the other forms.
-    Runs in a child process (the variable is read once per process)."""
+    Without ramp groups (the default) and with them (OQ_FUSED_RAMP=2: the GEMM warps first
+    quantize two token pairs a group in the stage ring).  Runs in child processes (the
+    variables are read once per process)."""
     import os
     import subprocess
     import sys
-    env = dict(os.environ, OQ_FUSED_STEP="1")
-    env.pop("OQ_LINEAR_PATH", None)
     child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_fused_step_child.py")
-    r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
-                       timeout=600)
-    assert r.returncode == 0, r.stdout + r.stderr
+    for ramp in ("0", "2"):                  # without and with ramp groups
+        env = dict(os.environ, OQ_FUSED_STEP="1", OQ_FUSED_RAMP=ramp)
+        env.pop("OQ_LINEAR_PATH", None)
+        r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
+                           timeout=600)
+        assert r.returncode == 0, f"OQ_FUSED_RAMP={ramp}: " + r.stdout + r.stderr
 
 
 @pytest.mark.parametrize("ba,bw", [(4, 4), (2, 8)])
