@@ -91,7 +91,8 @@ __device__ __forceinline__ void store_words(uint8_t *dst, const uint32_t (&w)[NW
 
 // 32 codes of one token (NW packed words, LSB-first) -> 32 fp16 unit centroids (16 words)
 // through the shared byte table `dect` (entry e of a byte: the centroids of the 8/BITS codes
-// it holds), stored as four 16-byte pieces.  BITS = 2, 4, 8.
+// it holds), stored as two 32-byte pieces (dst 32-byte aligned: rows of d fp16 with d a
+// multiple of 16, a thread's 32 positions at a multiple of 32).  BITS = 2, 4, 8.
 // 4-bit codes of the (odd-symmetric) codebook use the byte-permute decode instead (no table
 // loads): p.dec_src holds its four sources.
 template <int BITS>
@@ -126,9 +127,13 @@ __device__ __forceinline__ void decode_store(const uint32_t *dect, const uint32_
                 (uint32_t)d16[(w[i] >> 16) & 0xffu] | ((uint32_t)d16[w[i] >> 24] << 16);
         }
     }
+    // two 32-byte stores (256-bit, sm_100): every lane writes whole 32-byte sectors
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-        dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+    for (int k = 0; k < 2; ++k)
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                     ::"l"(dst + 2 * k), "r"(o[8 * k]), "r"(o[8 * k + 1]), "r"(o[8 * k + 2]),
+                     "r"(o[8 * k + 3]), "r"(o[8 * k + 4]), "r"(o[8 * k + 5]), "r"(o[8 * k + 6]),
+                     "r"(o[8 * k + 7]) : "memory");
 }
 
 // GELU in its exact (erf) form, x * Phi(x), in fp32, with Phi(x) = erfc(-x / sqrt 2) / 2
