@@ -431,6 +431,9 @@ def run_ours(args, p, rank, world, dev):
     # GEMM decodes them in shared memory
     acodes = (os.environ.get("OQ_LINEAR_PATH") == "fused" and p.bits_a == 4
               and p.dtype == torch.bfloat16)
+    # with OQ_LINEAR_PATH=wcodes and 4-bit weights the GEMM decodes the weight codes itself
+    wcodes = (os.environ.get("OQ_LINEAR_PATH") == "wcodes" and p.bits_w == 4
+              and os.environ.get("OQ_GEMM_PAIR") != "0")
     direct = (args.api == "forward" and not acodes and p.bits_a in (2, 4, 8)
               and p.dtype == torch.bfloat16 and 32 <= p.h <= 256)
     launches = launches_per_step * args.steps
@@ -508,7 +511,8 @@ def run_ours(args, p, rank, world, dev):
     flops = 2.0 * p.T * p.d * p.out
     gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
     traffic, traffic_src = profile_traffic(
-        f"k2_gemm_{'acodes_' if acodes else ''}{p.name}.ncu.csv", GEMM_SOURCES)
+        f"k2_gemm_{'acodes_' if acodes else 'wcodes_' if wcodes else ''}{p.name}.ncu.csv",
+        GEMM_SOURCES)
     in_bytes = 2 if p.dtype == torch.bfloat16 else 4
     # K1's algorithmic bytes are the method's: x in, the packed codes and s out, T (in*d +
     # d*ba/8 + 4).  What this design moves besides (the fp16 centroids K1 writes for the GEMM
@@ -518,7 +522,7 @@ def run_ours(args, p, rank, world, dev):
     design_bytes = p.T * (in_bytes * p.d + (2 * p.d if direct else p.d * p.bits_a // 8) + 4)
     # with 2/4-bit weights the one-call path's K1 also decodes the weight codes (no decode
     # launch)
-    fused_dec = args.api == "forward" and (direct or acodes) and dec_ms is None
+    fused_dec = args.api == "forward" and (direct or acodes) and dec_ms is None and not wcodes
     if fused_dec:
         design_bytes += p.out * p.d * (p.bits_w / 8 + 2)
     q_gbs = q_bytes / (quant_ms * 1e-3) / 1e9
@@ -541,11 +545,14 @@ def run_ours(args, p, rank, world, dev):
         "gemm_a_operand": ("4-bit codes, decoded in the GEMM's shared memory" if acodes else
                            "fp16 centroids written by the quantizer" if direct else
                            "fp16 centroids from the decode prepass"),
+        "gemm_b_operand": ("4-bit codes, decoded in the GEMM's shared memory" if wcodes else
+                           "fp16 centroids from the weight decode"),
         "roofline": {
             "kernel": ("k3_fused (rotate+quantize stage and tcgen05 cta_group::2 GEMM in one "
                        "persistent kernel; its time covers both)" if fused_step else
                        "k2_gemm_pair (tcgen05 cta_group::2 kind::f16, 256x256x64 tiles per "
                        "CTA pair" + (", 4-bit A codes decoded in shared memory)" if acodes
+                                    else ", 4-bit B codes decoded in shared memory)" if wcodes
                                     else ")")),
             "bound": "tensor", "achieved": gemm_tf,
             "peak": pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),

@@ -382,13 +382,17 @@ __global__ void __launch_bounds__(gemm_threads<ACODES>(), 1)
 // CTAs arrives on the leader's accumulator-empty barrier.  Every TMA load fills only its own
 // CTA's shared memory.
 // ------------------------------------------------------------------------------------------
-// ACODES (4-bit activation codes of a symmetric codebook): each CTA's TMA brings the packed
-// codes of its own 128 rows (128 x 32 bytes per k-block) into a code stage and signals its own
-// barrier; eight decoder warps per CTA expand them into the fp16 A stage in the 128-byte
-// swizzled layout the MMA reads and arrive on the leader's A-ready barrier (16 arrivals: both
-// CTAs' decoders).  The ring then holds 5 stages.  The stage's A tile is free when its codes
-// land, because the producer issued the code load only after the MMAs that last read the
-// stage had completed.
+// Codes (4-bit codes of a symmetric codebook, for the activations (kCodesA) or the weights
+// (kCodesB)): each CTA's TMA brings the packed codes of its own 128 rows of that operand
+// (128 x 32 bytes per k-block) into a code stage and signals its own barrier; eight decoder
+// warps per CTA expand them into the operand's fp16 stage in the 128-byte swizzled layout the
+// MMA reads and arrive on the leader's operand-ready barrier (16 arrivals: both CTAs'
+// decoders).  The ring then holds 5 stages.  The stage's tile is free when its codes land,
+// because the producer issued the code load only after the MMAs that last read the stage had
+// completed.  A row of codes is decoded once per tile it takes part in: an activation row
+// once per 256-column tile, a weight row once per 256-row tile.
+// CODES of k2_gemm_pair: which operand arrives as 4-bit codes decoded in the kernel
+constexpr int kCodesNone = 0, kCodesA = 1, kCodesB = 2;
 template <bool ACODES>
 __host__ __device__ constexpr int pair_stages() { return ACODES ? 5 : 6; }
 constexpr int P_BM = 256, P_BN = 256;                    // pair tile
@@ -417,10 +421,11 @@ static_assert(gemm_pair_smem<false>() <= 227 * 1024 && gemm_pair_smem<true>() <=
 // CTAs allocate the same columns) and its lane 0 issues the MMAs (leader only), warps 2..5
 // are the epilogue (both CTAs, each its own 128 rows), ACODES: warps 6..13 decode (both CTAs,
 // each its own 128 rows).  Pair p takes tiles p, p + #pairs, ...
-template <bool BF16, bool ACODES>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<ACODES>(), 1)
+template <bool BF16, int CODES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES != 0>(), 1)
     k2_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+    constexpr bool ACODES = CODES != 0;             // one operand arrives as codes
     constexpr int S = pair_stages<ACODES>();
     constexpr int kBarSets = ACODES ? 4 : 2;
     extern __shared__ unsigned char smem_raw[];
@@ -501,17 +506,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<ACODES>
                     if (aborted())
                         break;
                     const uint32_t fb = mapa_shared(full_bar(s), 0);
-                    if constexpr (ACODES) {
+                    if constexpr (CODES == kCodesA) {
                         if (rank == 0)
                             mbar_expect_tx(full_bar(s), 2 * P_B_BYTES);
                         mbar_expect_tx(cfull_bar(s), P_CODE_BYTES);
                         tma_load_2d(sC + s * P_CODE_BYTES, &tmA, kb * (BK / 2), m0, cfull_bar(s));
+                        tma_load_2d_pair(sB + s * P_B_BYTES, &tmB, kb * BK, n0, fb);
+                    } else if constexpr (CODES == kCodesB) {
+                        if (rank == 0)
+                            mbar_expect_tx(full_bar(s), 2 * P_A_BYTES);
+                        mbar_expect_tx(cfull_bar(s), P_CODE_BYTES);
+                        tma_load_2d_pair(sA + s * P_A_BYTES, &tmA, kb * BK, m0, fb);
+                        tma_load_2d(sC + s * P_CODE_BYTES, &tmB, kb * (BK / 2), n0, cfull_bar(s));
                     } else {
                         if (rank == 0)
                             mbar_expect_tx(full_bar(s), 2 * P_STAGE_BYTES);
                         tma_load_2d_pair(sA + s * P_A_BYTES, &tmA, kb * BK, m0, fb);
+                        tma_load_2d_pair(sB + s * P_B_BYTES, &tmB, kb * BK, n0, fb);
                     }
-                    tma_load_2d_pair(sB + s * P_B_BYTES, &tmB, kb * BK, n0, fb);
                 }
             }
             if (aborted()) {
@@ -629,14 +641,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<ACODES>
         if (lane == 0)
             bulk_wait_all();
     } else if constexpr (ACODES) {
-        // ---------------- decoders (both CTAs): 4-bit codes -> this CTA's fp16 A stages ----
+        // ---------------- decoders (both CTAs): 4-bit codes -> this CTA's fp16 stages of the
+        // coded operand (A rows or B rows) ----
         // Thread = row r of this CTA's 128 rows and one half of its 64 codes per k-block: 16
         // bytes of codes in, 64 bytes of the fp16 row out in the 128-byte swizzled layout
         // (16-byte piece k of row r at piece k ^ (r % 8), 8-row atoms of 1024 bytes).
         const int r = (warp & 3) * 32 + lane;
         const int half = (warp - 2 - kEpiWarps) >> 2;
         const uint32_t row_off = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
-        unsigned char *sAp = basep + (sA - base);
+        unsigned char *sAp = basep + ((CODES == kCodesA ? sA : sB) - base);
         const unsigned char *sCp = basep + (sC - base);
         const uint32_t ready = rank == 0 ? 0u : 1u;
         uint32_t it = 0;
@@ -845,8 +858,9 @@ cudaError_t launch_gemm_t(const CUtensorMap &ma, const CUtensorMap &mb, const CU
 
 // Pairs of the CTA-pair GEMM that fit on the device at once (0: the form is unavailable),
 // once per device and instantiation.
-template <bool BF16, bool ACODES>
+template <bool BF16, int CODES>
 int gemm_pair_slots() {
+    constexpr bool ACODES = CODES != kCodesNone;
     static std::mutex mu;
     static int slots[kMaxDevices];
     static bool done[kMaxDevices] = {};
@@ -857,7 +871,7 @@ int gemm_pair_slots() {
     if (!done[dev]) {
         done[dev] = true;
         slots[dev] = 0;
-        auto kern = k2_gemm_pair<BF16, ACODES>;
+        auto kern = k2_gemm_pair<BF16, CODES>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gemm_pair_smem<ACODES>()) != cudaSuccess) {
             cudaGetLastError();
@@ -877,17 +891,20 @@ int gemm_pair_slots() {
     return slots[dev];
 }
 
-template <bool BF16, bool ACODES>
+template <bool BF16, int CODES>
 cudaError_t launch_gemm_pair_t(const CUtensorMap &ma, const CUtensorMap &mb,
                                const CUtensorMap &my, const GemmParams &gp, int pairs,
                                cudaStream_t st, std::string *why) {
+    constexpr bool ACODES = CODES != kCodesNone;
     const cudaError_t e =
-        launch_pdl(k2_gemm_pair<BF16, ACODES>, dim3(2 * pairs), dim3(pair_threads<ACODES>()),
+        launch_pdl(k2_gemm_pair<BF16, CODES>, dim3(2 * pairs), dim3(pair_threads<ACODES>()),
                    gemm_pair_smem<ACODES>(), st, ma, mb, my, gp);
     if (e != cudaSuccess)
         *why = "k2_gemm_pair launch";
     return e;
 }
+
+}  // namespace
 
 // The CTA-pair GEMM is used when the device can hold it; OQ_GEMM_PAIR=0 selects the
 // single-CTA kernel (read once per process).
@@ -899,13 +916,12 @@ bool gemm_pair_enabled() {
     return on;
 }
 
-}  // namespace
-
 cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
-                        const uint16_t *B16, const float *s, const float *rn, void *y,
-                        bool y_bf16, int T, int N, int d, cudaStream_t st, int num_sms,
-                        std::string *why, long long test_wait_cycles) {
-    const bool acodes = A16 == nullptr;
+                        const uint16_t *B16, const uint8_t *w_codes4, const uint16_t *lut_w,
+                        const float *s, const float *rn, void *y, bool y_bf16, int T, int N,
+                        int d, cudaStream_t st, int num_sms, std::string *why,
+                        long long test_wait_cycles) {
+    const bool acodes = A16 == nullptr, wcodes = B16 == nullptr;
     GemmParams gp;
     gp.test_wait_cycles = test_wait_cycles;
     gp.s = s;
@@ -915,32 +931,53 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
     gp.N = N;
     gp.K = d;
     gp.inv_d = 1.0f / (float)d;
+    if (acodes && wcodes) {
+        *why = "k2_gemm: at most one operand can arrive as codes";
+        return cudaErrorInvalidValue;
+    }
     if (acodes && (!x_codes4 || !lut_a ||
                    !decode8_sources(lut_a, &gp.L0, &gp.L1, &gp.H0, &gp.H1))) {
         *why = "k2_gemm: activation codes need a 4-bit odd-symmetric codebook";
         return cudaErrorInvalidValue;
     }
+    if (wcodes && (!w_codes4 || !lut_w ||
+                   !decode8_sources(lut_w, &gp.L0, &gp.L1, &gp.H0, &gp.H1))) {
+        *why = "k2_gemm: weight codes need a 4-bit odd-symmetric codebook";
+        return cudaErrorInvalidValue;
+    }
     CUtensorMap ma, mb, my;
     if (gemm_pair_enabled()) {
-        const int slots = acodes ? (y_bf16 ? gemm_pair_slots<true, true>()
-                                           : gemm_pair_slots<false, true>())
-                                 : (y_bf16 ? gemm_pair_slots<true, false>()
-                                           : gemm_pair_slots<false, false>());
+        const int slots =
+            acodes ? (y_bf16 ? gemm_pair_slots<true, kCodesA>() : gemm_pair_slots<false, kCodesA>())
+            : wcodes ? (y_bf16 ? gemm_pair_slots<true, kCodesB>()
+                               : gemm_pair_slots<false, kCodesB>())
+                     : (y_bf16 ? gemm_pair_slots<true, kCodesNone>()
+                               : gemm_pair_slots<false, kCodesNone>());
         if (slots > 0) {
             const bool a_ok = acodes ? make_code_map(&ma, x_codes4, T, d)
                                      : make_map(&ma, A16, T, d, 128);
-            if (!a_ok || !make_map(&mb, B16, N, d, 128) || !make_out_map(&my, y, T, N, y_bf16)) {
+            const bool b_ok = wcodes ? make_code_map(&mb, w_codes4, N, d)
+                                     : make_map(&mb, B16, N, d, 128);
+            if (!a_ok || !b_ok || !make_out_map(&my, y, T, N, y_bf16)) {
                 *why = "cuTensorMapEncodeTiled failed";
                 return cudaErrorInvalidValue;
             }
             const int tiles = ((N + P_BN - 1) / P_BN) * ((T + P_BM - 1) / P_BM);
             const int pairs = tiles < slots ? tiles : slots;
             if (acodes)
-                return y_bf16 ? launch_gemm_pair_t<true, true>(ma, mb, my, gp, pairs, st, why)
-                              : launch_gemm_pair_t<false, true>(ma, mb, my, gp, pairs, st, why);
-            return y_bf16 ? launch_gemm_pair_t<true, false>(ma, mb, my, gp, pairs, st, why)
-                          : launch_gemm_pair_t<false, false>(ma, mb, my, gp, pairs, st, why);
+                return y_bf16 ? launch_gemm_pair_t<true, kCodesA>(ma, mb, my, gp, pairs, st, why)
+                              : launch_gemm_pair_t<false, kCodesA>(ma, mb, my, gp, pairs, st, why);
+            if (wcodes)
+                return y_bf16 ? launch_gemm_pair_t<true, kCodesB>(ma, mb, my, gp, pairs, st, why)
+                              : launch_gemm_pair_t<false, kCodesB>(ma, mb, my, gp, pairs, st, why);
+            return y_bf16
+                       ? launch_gemm_pair_t<true, kCodesNone>(ma, mb, my, gp, pairs, st, why)
+                       : launch_gemm_pair_t<false, kCodesNone>(ma, mb, my, gp, pairs, st, why);
         }
+    }
+    if (wcodes) {
+        *why = "k2_gemm: weight codes are decoded by the CTA-pair GEMM only";
+        return cudaErrorInvalidValue;
     }
     const bool a_ok = acodes ? make_code_map(&ma, x_codes4, T, d) : make_map(&ma, A16, T, d, BM);
     if (!a_ok || !make_map(&mb, B16, N, d, BN) || !make_out_map(&my, y, T, N, y_bf16)) {

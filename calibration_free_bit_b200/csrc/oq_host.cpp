@@ -673,15 +673,30 @@ cudaStream_t device_side(DeviceInfo *di, int *rc) {
     return st;
 }
 
-// OQ_LINEAR_PATH=fused decodes 4-bit activation codes inside the GEMM kernel instead of in
-// the prepass (read once per process): no [T, d] fp16 workspace, but each 128-row tile of
-// codes is decoded once per 256-column tile of the output.
-bool fused_requested() {
-    static const bool v = [] {
+// OQ_LINEAR_PATH (read once per process): "fused" decodes 4-bit activation codes inside the
+// GEMM kernel instead of in the prepass (no [T, d] fp16 workspace, but each 128-row tile of
+// codes is decoded once per 256-column tile of the output); "wcodes" decodes 4-bit weight
+// codes inside the CTA-pair GEMM (no [N, d] fp16 workspace and no weight decode launch, but
+// each weight row is decoded once per 256-row tile of the output).
+int linear_path() {
+    static const int v = [] {
         const char *e = std::getenv("OQ_LINEAR_PATH");
-        return e != nullptr && std::strcmp(e, "fused") == 0;
+        if (e != nullptr && std::strcmp(e, "fused") == 0)
+            return 1;
+        if (e != nullptr && std::strcmp(e, "wcodes") == 0)
+            return 2;
+        return 0;
     }();
     return v;
+}
+bool fused_requested() { return linear_path() == 1; }
+
+// The weight operand of this codebook decoded inside the GEMM (OQ_LINEAR_PATH=wcodes, 4-bit
+// odd-symmetric codebook, CTA-pair GEMM).
+bool wcodes_applies(const oq_codebook *cw) {
+    uint32_t src[4];
+    return linear_path() == 2 && cw->bits == 4 && oq::gemm_pair_enabled() &&
+           oq::decode8_sources(cw->lut, &src[0], &src[1], &src[2], &src[3]);
 }
 
 // OQ_FUSED_STEP=1 runs oq_quantized_linear as one persistent kernel (k3_fused.cu) where it
@@ -1131,8 +1146,10 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     // OQ_LINEAR_PATH=fused, 4-bit activation codes are decoded inside the GEMM kernel and only
     // the weight codes get the prepass.
     const bool fused = ca->bits == 4 && fused_requested();
-    const size_t ws_bytes = fused ? (size_t)out_features * d * 2
-                                  : oq::linear_workspace_bytes(T, d, out_features);
+    const bool wcodes = wcodes_applies(cw);
+    const size_t ws_bytes = fused    ? (size_t)out_features * d * 2
+                            : wcodes ? (size_t)T * d * 2
+                                     : oq::linear_workspace_bytes(T, d, out_features);
     void *ws = nullptr;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaMallocFromPoolAsync(&ws, ws_bytes, pool, st);
@@ -1140,24 +1157,27 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
         return fail_cuda(e, "oq_linear: workspace allocation");
     std::string why;
     uint16_t *A16 = nullptr, *B16 = static_cast<uint16_t *>(ws);
+    if (wcodes)
+        B16 = nullptr;
     if (!fused) {
         A16 = static_cast<uint16_t *>(ws);
-        B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
-                                           oq::linear_workspace_b_offset(T, d));
+        if (!wcodes)
+            B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
+                                               oq::linear_workspace_b_offset(T, d));
         e = timed(OQ_KERNEL_DECODE, st, [&] {
             return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
         });
     }
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !wcodes)
         e = timed(OQ_KERNEL_DECODE, st, [&] {
             return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
                                      di->sms, &why);
         });
     if (e == cudaSuccess)
         e = timed(OQ_KERNEL_GEMM, st, [&] {
-            return oq::launch_gemm(A16, x_codes, ca->lut, B16, s, row_norms, y,
-                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
-                                   take_armed(OQ_KERNEL_GEMM));
+            return oq::launch_gemm(A16, x_codes, ca->lut, B16, W_codes, cw->lut, s, row_norms,
+                                   y, out_dtype == OQ_BF16, T, out_features, d, st, di->sms,
+                                   &why, take_armed(OQ_KERNEL_GEMM));
         });
     cudaError_t e2 = cudaFreeAsync(ws, st);
     if (e != cudaSuccess)
@@ -1223,9 +1243,9 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
         });
     if (e == cudaSuccess)
         e = timed(OQ_KERNEL_GEMM, st, [&] {
-            return oq::launch_gemm(A16, nullptr, nullptr, B16, s, row_norms, y,
-                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
-                                   take_armed(OQ_KERNEL_GEMM));
+            return oq::launch_gemm(A16, nullptr, nullptr, B16, nullptr, nullptr, s, row_norms,
+                                   y, out_dtype == OQ_BF16, T, out_features, d, st, di->sms,
+                                   &why, take_armed(OQ_KERNEL_GEMM));
         });
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());
@@ -1287,15 +1307,18 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     //   codes:  K1 writes the packed 4-bit codes and the GEMM decodes them into its shared-
     //           memory A tiles (OQ_LINEAR_PATH=fused; bf16 x, odd-symmetric 4-bit codebook);
     //   else:   K1 writes codes and the decode prepass expands them into the fp16 A operand.
-    // workspace: A16 [T, d] fp16 (direct / prepass) | B16 [N, d] fp16 | s [T] (if not given) |
-    // codes [T, d*ba/8] (codes / prepass)
+    // The weight operand: decoded into B16 (in K1's tail or on the side stream), or, with
+    // OQ_LINEAR_PATH=wcodes, decoded from its codes inside the GEMM.
+    // workspace: A16 [T, d] fp16 (direct / prepass) | B16 [N, d] fp16 (not wcodes) | s [T] (if
+    // not given) | codes [T, d*ba/8] (codes / prepass)
     uint32_t src_probe[4];
     const bool acodes = fused_requested() && ca->bits == 4 && dtype == OQ_BF16 &&
                         oq::decode8_sources(ca->lut, &src_probe[0], &src_probe[1],
                                             &src_probe[2], &src_probe[3]);
     const bool direct = !acodes && oq::k1_a16_supported(ca->bits, r->h, dtype == OQ_BF16);
+    const bool wcodes = wcodes_applies(cw);
     const size_t a_bytes = acodes ? 0 : align_up((size_t)T * d * 2, 1024);
-    const size_t b_bytes = align_up((size_t)out_features * d * 2, 1024);
+    const size_t b_bytes = wcodes ? 0 : align_up((size_t)out_features * d * 2, 1024);
     const size_t s_bytes = s ? 0 : align_up((size_t)T * 4, 1024);
     const size_t c_bytes = direct ? 0 : align_up((size_t)T * d * ca->bits / 8, 1024);
     void *ws = nullptr;
@@ -1305,7 +1328,7 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
         return fail_cuda(e, "oq_quantized_linear: workspace allocation");
     unsigned char *w8 = static_cast<unsigned char *>(ws);
     uint16_t *A16 = acodes ? nullptr : reinterpret_cast<uint16_t *>(w8);
-    uint16_t *B16 = reinterpret_cast<uint16_t *>(w8 + a_bytes);
+    uint16_t *B16 = wcodes ? nullptr : reinterpret_cast<uint16_t *>(w8 + a_bytes);
     float *sv = s ? s : reinterpret_cast<float *>(w8 + a_bytes + b_bytes);
     uint8_t *codes = direct ? nullptr : w8 + a_bytes + b_bytes + s_bytes;
     std::string why;
@@ -1316,16 +1339,16 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     // matrix, or one decoded by a single group per SM, decodes faster beside K1 than in its
     // tail.
     const bool fuse =
-        (direct || acodes) && out_features <= T && d <= 5120 && !tc_k1_requested() &&
+        !wcodes && (direct || acodes) && out_features <= T && d <= 5120 && !tc_k1_requested() &&
         oq::k1_named(d, dtype == OQ_BF16) &&
         (cw->bits == 2 || (cw->bits == 4 && oq::decode8_sources(cw->lut, &src_probe[0],
                                                                  &src_probe[1], &src_probe[2],
                                                                  &src_probe[3])));
     auto gemm = [&]() {
         return timed(OQ_KERNEL_GEMM, st, [&] {
-            return oq::launch_gemm(A16, codes, ca->lut, B16, sv, row_norms, y,
-                                   out_dtype == OQ_BF16, T, out_features, d, st, di->sms, &why,
-                                   take_armed(OQ_KERNEL_GEMM));
+            return oq::launch_gemm(A16, codes, ca->lut, B16, W_codes, cw->lut, sv, row_norms,
+                                   y, out_dtype == OQ_BF16, T, out_features, d, st, di->sms,
+                                   &why, take_armed(OQ_KERNEL_GEMM));
         });
     };
     if (fuse) {
@@ -1347,7 +1370,7 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
             return fail_cuda(e2, "oq_quantized_linear: workspace release");
         return OQ_OK;
     }
-    {
+    if (!wcodes) {
         // the weight decode needs nothing from x: it runs on the side stream beside K1
         std::lock_guard<std::mutex> lk(g_side_mu);
         e = cudaEventRecord(di->fork, st);
@@ -1376,7 +1399,7 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     }
     // the GEMM waits for the weight operand (join) whether or not K1 succeeded, so the
     // workspace is released after every use of it
-    e = cudaStreamWaitEvent(st, di->join, 0);
+    e = wcodes ? cudaSuccess : cudaStreamWaitEvent(st, di->join, 0);
     if (rc == OQ_OK && e == cudaSuccess) {
         e = gemm();
         if (e != cudaSuccess)

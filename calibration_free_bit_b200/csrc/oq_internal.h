@@ -142,15 +142,18 @@ size_t linear_workspace_b_offset(int T, int d);
 cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long long rows, int d,
                           const uint16_t *lut, cudaStream_t st, int num_sms, std::string *why);
 
-// y[T, N] = (s_t rn_o / d) * A[T, d] . B16[N, d]^T   (fp16 x fp16 -> fp32 in TMEM)
+// y[T, N] = (s_t rn_o / d) * A[T, d] . B[N, d]^T   (fp16 x fp16 -> fp32 in TMEM)
 // A is A16 (fp16 centroids from the prepass) or, when A16 is null, x_codes4: 4-bit codes of
 // the codebook whose fp16 LUT is lut_a (must be odd-symmetric), decoded inside the kernel.
-// y is fp32, or bf16 (round to nearest even of the fp32 epilogue value) when y_bf16.
-// test_wait_cycles > 0 arms the kernel's test of its bounded waits (oq_debug_arm_wait_timeout).
+// B likewise: B16, or (B16 null; CTA-pair kernel only) w_codes4 with lut_w.  At most one
+// operand as codes.  y is fp32, or bf16 (round to nearest even of the fp32 epilogue value)
+// when y_bf16.  test_wait_cycles > 0 arms the kernel's test of its bounded waits
+// (oq_debug_arm_wait_timeout).
 cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
-                        const uint16_t *B16, const float *s, const float *rn, void *y,
-                        bool y_bf16, int T, int N, int d, cudaStream_t st, int num_sms,
-                        std::string *why, long long test_wait_cycles = 0);
+                        const uint16_t *B16, const uint8_t *w_codes4, const uint16_t *lut_w,
+                        const float *s, const float *rn, void *y, bool y_bf16, int T, int N,
+                        int d, cudaStream_t st, int num_sms, std::string *why,
+                        long long test_wait_cycles = 0);
 
 // The online step in one persistent kernel (k3_fused.cu): the quantize stage and the CTA-pair
 // GEMM side by side on every SM, rows handed over through per-block counters.
@@ -190,6 +193,9 @@ cudaError_t launch_fused_step(const FusedStepParams &p, int bits, int h, bool y_
 cudaError_t read_and_clear_k3_error(unsigned *out, cudaStream_t st);
 // fp16 [rows, K] row-major operand -> TMA map of 128-row x 64 boxes, 128-byte swizzle
 bool make_operand_map(CUtensorMap *map, const void *ptr, long long rows, int K);
+
+// False when OQ_GEMM_PAIR=0 asks for the single-CTA GEMM (read once per process).
+bool gemm_pair_enabled();
 
 // Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
 // its size, and its address on the current device (looked up once per device).

@@ -162,7 +162,10 @@ int oq_quantize_act_gelu(const oq_rpbh *r, const oq_codebook *ca, const void *x,
  * are instead brought into the GEMM kernel by TMA as packed codes and decoded there, through
  * the codebook's fp16 LUT held in registers, into its shared-memory operand tiles; only the
  * weight codes get an fp16 buffer (less device memory and traffic, more decode work per call;
- * the same y bit for bit, since both forms feed the MMA the same fp16 values).
+ * the same y bit for bit, since both forms feed the MMA the same fp16 values).  With 4-bit
+ * weight codes and OQ_LINEAR_PATH=wcodes, the weight codes are the ones decoded inside the
+ * (CTA-pair) GEMM, each weight row once per 256-row tile of y, and only the activation codes
+ * get an fp16 buffer (again the same y; with OQ_GEMM_PAIR=0 the variable has no effect).
  * Either way the temporary device memory is stream-ordered, from a library-owned
  * pool.  The fp16 operands meet in a tcgen05 GEMM on pairs of CTAs (256 x 256 output tiles);
  * the environment variable OQ_GEMM_PAIR=0 (read once per process) selects the single-CTA
@@ -181,7 +184,9 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * ba in {2, 4, 8}, 32 <= h <= 256; otherwise codes and the decode prepass are used inside the
  * call).  With OQ_LINEAR_PATH=fused (read once per process), bf16 x and 4-bit activation
  * codes, the rotate+quantize kernel writes the packed codes instead and the GEMM decodes them
- * in shared memory (as oq_linear does under that variable).  With 2- or 4-bit weight codes, d
+ * in shared memory (as oq_linear does under that variable); with OQ_LINEAR_PATH=wcodes and
+ * 4-bit weight codes the GEMM decodes the weight codes itself (no weight decode launch and no
+ * [out_features, d] fp16 buffer).  Otherwise, with 2- or 4-bit weight codes, d
  * a multiple of 1024 up to 5120, bf16 x and out_features <= T, the rotate+quantize kernel
  * also decodes the weight codes into the GEMM's B operand once it runs out of tokens;
  * otherwise the weight codes are decoded on a library-owned side stream of the device while x

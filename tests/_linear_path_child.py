@@ -1,6 +1,6 @@
 """Child process for the oq_linear path test: OQ_LINEAR_PATH and OQ_GEMM_PAIR are read once per
-process, so each GEMM form (in-GEMM decode of 4-bit activation codes; fp16 prepass into the
-CTA-pair or the single-CTA GEMM) is exercised in a process of its own.  Checks oq_linear on uniform
+process, so each GEMM form (in-GEMM decode of 4-bit activation or weight codes; fp16 prepass
+into the CTA-pair or the single-CTA GEMM) is exercised in a process of its own.  Checks oq_linear on uniform
 random codes (every centroid used, ragged M and N tails) against the fp64 oracle, and the bf16
 output against the fp32 output rounded to nearest even, and oq_quantized_linear (which takes the
 same form) against oq_quantize_act + oq_linear bit for bit; prints the SHA-256 of the attention

@@ -376,8 +376,10 @@ def test_linear_video_ffn_up_full_size(oq, variant):
 def test_linear_path_selection(oq):
     """Every GEMM form against the oracle, each in a child process (the variables are read
     once per process): the fp16 prepass feeding the CTA-pair GEMM (default), the same prepass
-    feeding the single-CTA GEMM (OQ_GEMM_PAIR=0), and 4-bit activation codes decoded inside
-    the CTA-pair GEMM (OQ_LINEAR_PATH=fused) or the single-CTA one (both variables).  In each,
+    feeding the single-CTA GEMM (OQ_GEMM_PAIR=0), 4-bit activation codes decoded inside the
+    CTA-pair GEMM (OQ_LINEAR_PATH=fused) or the single-CTA one (both variables), and 4-bit
+    weight codes decoded inside the CTA-pair GEMM (OQ_LINEAR_PATH=wcodes; with
+    OQ_GEMM_PAIR=0 that form does not apply and the prepass serves the weights).  In each,
     oq_quantized_linear takes the same form and equals the two calls bit for bit, and the
     attention workload's y is identical across all forms (same fp16 operands, same MMA
     order)."""
@@ -387,12 +389,14 @@ def test_linear_path_selection(oq):
     import sys
     child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_linear_path_child.py")
     hashes = {}
-    for path in ("default", "fused", "single", "fused_single"):
+    for path in ("default", "fused", "single", "fused_single", "wcodes", "wcodes_single"):
         env = dict(os.environ)
         env.pop("OQ_LINEAR_PATH", None)
         env.pop("OQ_GEMM_PAIR", None)
         if path.startswith("fused"):
             env["OQ_LINEAR_PATH"] = "fused"
+        if path.startswith("wcodes"):
+            env["OQ_LINEAR_PATH"] = "wcodes"
         if path.endswith("single"):
             env["OQ_GEMM_PAIR"] = "0"
         r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
