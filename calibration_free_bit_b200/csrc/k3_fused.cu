@@ -801,6 +801,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     }
 }
 
+// Zeroes the fused step's progress counters once the stream's earlier work is done, as a
+// programmatic-launch kernel: it can be resident beside the previous kernel's tail, and the
+// fused kernel launched after it sets up while it runs (a memset node would break the chain).
+__global__ void __launch_bounds__(256) k3_zero_counters(unsigned *ctr, int n) {
+    pdl_trigger();
+    pdl_wait();
+    for (int i = (int)threadIdx.x; i < n; i += (int)blockDim.x)
+        ctr[i] = 0u;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------
@@ -860,6 +870,10 @@ cudaError_t launch_t(const CUtensorMap &ma, const CUtensorMap &mb, const CUtenso
 bool fused_step_supported(int d, int h, int bits, bool bf16_in) {
     return bf16_in && (d == 1024 || d == 2048 || d == 3072 || d == 4096) &&
            (h == 64 || h == 128 || h == 256) && (bits == 2 || bits == 4 || bits == 8);
+}
+
+cudaError_t launch_zero_counters(unsigned *ctr, int n, cudaStream_t st) {
+    return launch_pdl(k3_zero_counters, dim3(1), dim3(256), 0, st, ctr, n);
 }
 
 size_t fused_step_counter_words(int T, int N) {

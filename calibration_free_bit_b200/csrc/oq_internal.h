@@ -188,6 +188,8 @@ struct FusedStepParams {
 };
 bool fused_step_supported(int d, int h, int bits, bool bf16_in);
 size_t fused_step_counter_words(int T, int N);
+// Zero n counter words on the stream (a programmatic-launch kernel, see k3_fused.cu).
+cudaError_t launch_zero_counters(unsigned *ctr, int n, cudaStream_t st);
 cudaError_t launch_fused_step(const FusedStepParams &p, int bits, int h, bool y_bf16,
                               const uint16_t *B16, void *y, cudaStream_t st, std::string *why);
 cudaError_t read_and_clear_k3_error(unsigned *out, cudaStream_t st);
