@@ -540,7 +540,10 @@ def run_ours(args, p, rank, world, dev):
         "config": workload_config(p, world),
         "api": ("oq_quantized_linear (one call; x_codes stay on chip)" if args.api == "forward"
                 else "oq_quantize_act + oq_linear"),
-        "kernels_ms_mean": ({"fused_step": gemm_ms, "decode": dec_ms} if fused_step else
+        "kernels_ms_mean": ({"fused_step": gemm_ms, "decode": dec_ms,
+                             "counter_reset": (statistics.mean(per_kernel["aux"])
+                                               if "aux" in per_kernel else None)}
+                            if fused_step else
                             {"quantize": quant_ms, "decode": dec_ms, "gemm": gemm_ms}),
         "gemm_a_operand": ("4-bit codes, decoded in the GEMM's shared memory" if acodes else
                            "fp16 centroids written by the quantizer" if direct else

@@ -785,7 +785,10 @@ int fused_step(const oq_rpbh *r, const oq_codebook *ca, const oq_codebook *cw, c
         p.wdec_words = (long long)out_features * d * cw->bits / 32;
         p.wdec_bits = cw->bits;
     }
-    e = oq::launch_zero_counters(ctr, (int)oq::fused_step_counter_words(T, out_features), st);
+    e = timed(OQ_KERNEL_AUX, st, [&] {
+        return oq::launch_zero_counters(ctr, (int)oq::fused_step_counter_words(T, out_features),
+                                        st);
+    });
     if (e == cudaSuccess && !wdec_in)
         e = timed(OQ_KERNEL_DECODE, st, [&] {
             return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,

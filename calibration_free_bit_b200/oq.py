@@ -275,8 +275,9 @@ def oq_check(stream=None):
     _check(lib().oq_check(_stream(stream)))
 
 
-KERNEL_NAMES = {1: "quantize", 2: "decode", 3: "gemm", 4: "fused"}
+KERNEL_NAMES = {1: "quantize", 2: "decode", 3: "gemm", 4: "fused", 5: "aux"}
 OQ_KERNEL_QUANTIZE, OQ_KERNEL_DECODE, OQ_KERNEL_GEMM, OQ_KERNEL_FUSED = 1, 2, 3, 4
+OQ_KERNEL_AUX = 5
 
 
 def oq_debug_arm_wait_timeout(kernel: int, limit_cycles: int):

@@ -269,6 +269,7 @@ void oq_free_codebook(oq_codebook *cb);
 #define OQ_KERNEL_DECODE 2     /* codes -> fp16 centroid prepass of oq_linear */
 #define OQ_KERNEL_GEMM 3       /* tcgen05 codebook GEMM of oq_linear */
 #define OQ_KERNEL_FUSED 4      /* quantize stage and GEMM in one kernel (OQ_FUSED_STEP=1) */
+#define OQ_KERNEL_AUX 5        /* auxiliary launch: the fused step's counter reset */
 typedef struct {
     int kernel;
     float ms;
