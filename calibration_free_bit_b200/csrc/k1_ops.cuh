@@ -136,12 +136,23 @@ __device__ __forceinline__ void decode_store(const uint32_t *dect, const uint32_
                      "r"(o[8 * k + 7]) : "memory");
 }
 
-// GELU in its exact (erf) form, x * Phi(x), in fp32, with Phi(x) = erfc(-x / sqrt 2) / 2
-// (CUDA's erfcf): no cancellation of 1 + erf(x / sqrt 2) for negative x, so the left tail
-// keeps its relative accuracy (the erf form loses it below about x = -4).
-__device__ __forceinline__ float gelu_erf(float x) {
-    return 0.5f * x * erfcf(x * -0.70710678118654752f);
+// GELU(x) = x * Phi(x) of a bf16 x (given as fp32 bits, the bf16 in the top half).  For
+// 2^-16 <= |x| < 16 every bf16 value has its own entry in the shared-memory table at tab_smem
+// (kGeluTableWords fp32 values, each GELU(x) computed in fp64 and rounded to nearest on the
+// host): with v = the bf16 bits without the sign (biased exponent and 7-bit mantissa), entry
+// sign * 2560 + v - kGeluV0, kGeluV0 = the bits of 2^-16.  Below 2^-16, GELU(x) = x/2 to
+// within 2^-17 relative; from 16 up it is x (Phi(16) = 1 - 6e-58), from -16 down 0 (below
+// the smallest fp32).
+constexpr int kGeluTableWords = 5120;
+constexpr uint32_t kGeluV0 = (127u - 16u) << 7;          // 2^-16
+constexpr uint32_t kGeluV1 = kGeluV0 + 2559u;            // largest bf16 below 16
+__device__ __forceinline__ float gelu_lookup(uint32_t xb, uint32_t tab_smem) {
+    const float x = __uint_as_float(xb);
+    const uint32_t v = (xb >> 16) & 0x7fffu;
+    const uint32_t sgn = xb >> 31;
+    const uint32_t vc = min(max(v, kGeluV0), kGeluV1);
+    const float t = __uint_as_float(lds32(tab_smem + 4u * (sgn * 2560u + vc - kGeluV0)));
+    return v < kGeluV0 ? 0.5f * x : (v > kGeluV1 ? (sgn ? 0.0f : x) : t);
 }
-
 }  // namespace k1ops
 }  // namespace oq

@@ -175,7 +175,8 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     uint32_t *gent = table + p.tbl_words;
     uint32_t *dect = gent + p.ent_words;             // A16 only (dec_words = 0 otherwise)
     uint32_t *wdect = dect + p.dec_words;            // fused 2-bit weight decode table
-    float2 *red = reinterpret_cast<float2 *>(wdect + p.wdec_words);
+    const float *gtab = reinterpret_cast<const float *>(wdect + p.wdec_words);   // GELU only
+    float2 *red = reinterpret_cast<float2 *>(wdect + p.wdec_words + p.gelu_words);
     unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + 2 * NG * kMaxSeg);
     // [0] next pair, [1 + grp] a group's next pair, [16] next decode chunk, [17 + grp] a
     // group's decode chunk
@@ -198,14 +199,16 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
     __syncthreads();
     if (tid == 0) {
         // host-built table, entry and decode images: bulk copies
-        mbar_expect_tx(setup_bar,
-                       4u * (p.tbl_words + p.ent_words + p.dec_words + p.wdec_words));
+        mbar_expect_tx(setup_bar, 4u * (p.tbl_words + p.ent_words + p.dec_words +
+                                        p.wdec_words + p.gelu_words));
         bulk_copy(smem_u32(table), p.tbl_img, 4u * p.tbl_words, setup_bar);
         bulk_copy(smem_u32(gent), p.ent_img, 4u * p.ent_words, setup_bar);
         if (p.dec_words > 0)
             bulk_copy(smem_u32(dect), p.dec_img, 4u * p.dec_words, setup_bar);
         if (p.wdec_words > 0)
             bulk_copy(smem_u32(wdect), p.wdec_img, 4u * p.wdec_words, setup_bar);
+        if (p.gelu_words > 0)
+            bulk_copy(smem_u32(gtab), p.gelu_img, 4u * p.gelu_words, setup_bar);
     }
 
     // this thread's 32 rotated positions: pos0 + e with pos0 = g * 32; r = its index inside
@@ -325,8 +328,8 @@ __global__ void __maxnreg__(96) k1_rotquant(const K1Params p) {
                     const uint32_t off = en & 0x7fffffffu;
                     if constexpr (GELU) {
                         const uint32_t w = lds32(base0 + off);
-                        const float a = gelu_erf(__uint_as_float(w << 16));
-                        const float b = gelu_erf(__uint_as_float(w & 0xffff0000u));
+                        const float a = gelu_lookup(w << 16, smem_u32(gtab));
+                        const float b = gelu_lookup(w & 0xffff0000u, smem_u32(gtab));
                         v[e].x = __uint_as_float(__float_as_uint(a) ^ sg);
                         v[e].y = __uint_as_float(__float_as_uint(b) ^ sg);
                     } else if constexpr (!IN_F32) {
@@ -615,7 +618,8 @@ cudaError_t launch_h(const K1Params &p, int h, long long ctas_needed, int thread
 
 size_t k1_smem(const K1Params &p, int in_f32, int NG, int stages) {
     const size_t row_in = (size_t)p.d * (in_f32 ? 4 : 2);
-    size_t b = 4 * (size_t)(p.tbl_words + p.ent_words + p.dec_words + p.wdec_words);
+    size_t b = 4 * (size_t)(p.tbl_words + p.ent_words + p.dec_words + p.wdec_words +
+                            p.gelu_words);
     b += sizeof(float2) * 2 * NG * kMaxSeg;                // norm partials, two buffers
     b += 8 * (size_t)(2 * NG + 2);                         // mbarriers
     b += 4 * 32;                                           // pair and decode scheduling words

@@ -412,6 +412,7 @@ struct DeviceInfo {
     cudaMemPool_t pool = nullptr;
     cudaStream_t side = nullptr;      // oq_quantized_linear: weight decode beside K1
     cudaEvent_t fork = nullptr, join = nullptr;
+    uint32_t *gelu_tab = nullptr;     // the fused GELU's table (oq::gelu_table_image)
 };
 DeviceInfo g_dev[oq::kMaxDevices];
 std::mutex g_dev_mu;
@@ -579,6 +580,14 @@ int quantize_rows(const oq_rpbh *r, const oq_codebook *cb, const void *x, int dt
     p.G = cb->G;
     p.F = cb->F;
     p.gelu = gelu ? 1 : 0;
+    if (gelu) {
+        static std::mutex gelu_mu;
+        static const std::vector<uint32_t> gelu_img = oq::gelu_table_image();
+        if ((rc = upload(gelu_mu, &di->gelu_tab, gelu_img, "upload GELU table")) != OQ_OK)
+            return rc;
+        p.gelu_img = di->gelu_tab;
+        p.gelu_words = (int)gelu_img.size();
+    }
     p.test_wait_cycles = take_armed(OQ_KERNEL_QUANTIZE);
     if (a16) {
         if (!oq::k1_a16_supported(cb->bits, r->h, dtype == OQ_BF16))
@@ -828,6 +837,26 @@ int fused_step(const oq_rpbh *r, const oq_codebook *ca, const oq_codebook *cw, c
 }
 
 }  // namespace
+
+namespace oq {
+
+// GELU(x) = x Phi(x) = x erfc(-x / sqrt 2) / 2 in fp64, rounded to fp32, for every bf16 x with
+// 2^-16 <= |x| < 16: entry sign * 2560 + (e + 16) * 128 + m holds |x| = (1 + m/128) 2^e.
+std::vector<uint32_t> gelu_table_image() {
+    std::vector<uint32_t> img(5120);
+    for (int sgn = 0; sgn < 2; ++sgn)
+        for (int e = -16; e <= 3; ++e)
+            for (int m = 0; m < 128; ++m) {
+                const double x = (sgn ? -1.0 : 1.0) * std::ldexp(1.0 + m / 128.0, e);
+                const float g = (float)(0.5 * x * std::erfc(-x / std::sqrt(2.0)));
+                uint32_t u;
+                std::memcpy(&u, &g, 4);
+                img[(size_t)sgn * 2560 + (size_t)(e + 16) * 128 + m] = u;
+            }
+    return img;
+}
+
+}  // namespace oq
 
 // ---------------------------------------------------------------------------------------
 // C ABI.

@@ -94,7 +94,12 @@ struct K1Params {
     const uint32_t *wdec_img;     // 2-bit: byte -> four fp16 centroids (256 x 8 bytes)
     int wdec_words;               // its size in words (0 for 4-bit)
     long long test_wait_cycles;   // > 0: the armed test wait (oq_debug_arm_wait_timeout)
+    const uint32_t *gelu_img;     // gelu: the GELU table of the bf16 values (k1_ops.cuh)
+    int gelu_words;               // its size in words (0 without gelu)
 };
+// GELU(x) for every bf16 x with 2^-16 <= |x| < 16 (layout in k1_ops.cuh, gelu_lookup), in fp64
+// rounded to fp32: the host image K1 copies into shared memory for its fused GELU.
+std::vector<uint32_t> gelu_table_image();
 // True when K1 can write fp16 centroids itself (launch_k1 with p.a16 set).
 inline bool k1_a16_supported(int bits, int h, bool bf16_in) {
     return bf16_in && h >= 32 && h <= 256 && (bits == 2 || bits == 4 || bits == 8);
