@@ -484,6 +484,33 @@ def test_k1_fused_gelu(oq, bits, h, d, T):
     np.testing.assert_allclose(s.cpu().numpy(), os_, rtol=NORM_RTOL)
 
 
+@pytest.mark.parametrize("h", [64, 256])
+def test_k1_fused_gelu_edge_values(oq, h):
+    """The fused GELU at the values where its evaluation changes form: zero, values below and
+    at the low end of its table (2^-16), inside it, at its top end (the largest bf16 below 16)
+    and beyond (16 and up, both signs), mixed with N(0, 1) values so that the rows have
+    ordinary norms.  Codes under the boundary-distance rule (such rows put many rotated values
+    near a few points, as the small-block GELU case does) and norms against the oracle."""
+    T, d, bits = 64, 1024, 4
+    special = np.array([0.0, 1e-6, 2.0 ** -17, 2.0 ** -16, 1.5 * 2.0 ** -16, 0.004, 0.75,
+                        1.0, 3.5, 15.9375, 16.0, 17.0, 100.0, 1e4])
+    special = np.concatenate([special, -special])
+    rng = np.random.default_rng(h)
+    x = rng.standard_normal((T, d))
+    mask = rng.random((T, d)) < 0.5
+    x[mask] = rng.choice(special, size=int(mask.sum()))
+    u = torch.from_numpy(x).float().to(torch.bfloat16)
+    r = oq.oq_build_rpbh(d, h, 0)
+    cb = oq.oq_lloyd_max(d, bits)
+    xc, s = oq.oq_quantize_act(r, cb, u.cuda(), gelu=True)
+    oq.oq_check()
+    perm, sign = O.build_rpbh(d, 0)
+    o, os_, _, ou = O.quantize_act(u.double().numpy(), h, perm, sign, bits, detail=True,
+                                   gelu_input=True)
+    check_codes(xc.cpu().numpy(), o, ou, d, bits, f"gelu edges h={h}", count_rule=False)
+    np.testing.assert_allclose(s.cpu().numpy(), os_, rtol=NORM_RTOL)
+
+
 def test_k1_fused_gelu_rejects_fp32(oq):
     r, cb = oq.oq_build_rpbh(256, 64, 0), oq.oq_lloyd_max(256, 4)
     with pytest.raises(oq.OQError):
