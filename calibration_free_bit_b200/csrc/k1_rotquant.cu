@@ -9,10 +9,11 @@
 // B200 design (one HBM-bound pass: read 2d bytes per bf16 row, write d*b/8 + 4):
 //   * Thread groups of d/32 threads; a group works on one token PAIR at a time, whose two
 //     rows stream into shared memory with bulk copies (completing on an mbarrier) one pair
-//     ahead of the compute.  bf16 rows whose groups are whole warps: one CTA per SM, an
-//     equal contiguous share of the pairs per CTA, each group on its own named barrier
-//     taking its next pair from a shared counter.  Otherwise several smaller CTAs per SM
-//     step through the pairs in lockstep rounds.
+//     ahead of the compute.  bf16 rows whose groups are whole warps, or can be padded to
+//     whole warps with at most one lane in eight idle: one CTA per SM, an equal contiguous
+//     share of the pairs per CTA, each group on its own named barrier taking its next pair
+//     from a shared counter.  Otherwise several smaller CTAs per SM step through the pairs in
+//     lockstep rounds.
 //   * bf16 rows are interleaved into 32-bit words (x_t0[j], x_t1[j]), so one 4-byte gather
 //     load serves both tokens and the butterfly runs on packed fp32x2 (add/sub/fma .f32x2,
 //     new on sm_100).  Each half of an 8-element chunk goes to a 16-byte slot the host
@@ -31,8 +32,11 @@
 //     cell's base code and its boundary, so the decision is exact in the fixed-point q grid
 //     (2^-23 of the grid span, < 1.2e-6 sigma).  Bit widths 2/3/4/6/8 pack LSB-first.
 //   * fp16 output (the one-call path): each code's fp16 unit centroid instead of the packed
-//     codes (the GEMM's A operand); with it, the groups that run out of pairs can decode the
-//     layer's 2- or 4-bit weight codes into the GEMM's B operand (each CTA an equal share).
+//     codes (the GEMM's A operand, 32-byte stores); with it, the groups that run out of pairs
+//     can decode the layer's 2- or 4-bit weight codes into the GEMM's B operand (each CTA an
+//     equal share).
+//   * Fused GELU (bf16 rows): GELU of each gathered element from a shared table of all bf16
+//     values (k1_ops.cuh, gelu_lookup).
 //   * Every mbarrier wait is bounded (about 2 s of SM clock); a wait that gives up sets a bit
 //     in the device error word (read by oq_check) and the round's outputs are not written.
 #include <cuda_bf16.h>
@@ -124,9 +128,9 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // to each gathered element before its sign flip (it is elementwise, so it commutes with P).
 // A16 (bf16 input, BITS = 2, 4, 8): instead of the packed codes, the kernel writes each code's
 // fp16 unit centroid to p.a16 [T, d] (the GEMM's A operand; the codes stay on chip).
-// NAMED (bf16 input, groups of whole warps): each group synchronises on its own named barrier
-// and takes pairs from a shared counter; the kernel then reserves all 16 barriers of the SM's
-// CTA slot, so it is launched one CTA per SM.  Otherwise the CTA synchronises as a whole and
+// NAMED (bf16 input, groups of whole warps, padded to them where k1_named allows): each group
+// synchronises on its own named barrier and takes pairs from a shared counter; the kernel then
+// reserves all 16 barriers of the SM's CTA slot, so it is launched one CTA per SM.  Otherwise the CTA synchronises as a whole and
 // its groups step through the CTA's pairs in lockstep.
 // H = kSmallH stands for every block size below 32 (2, 4, 8, 16): a thread's 32 positions
 // then hold 32/h whole blocks, the butterfly stops after log2(h) in-register stages (h read

@@ -13,10 +13,10 @@
 //     TMA ring, two TMEM accumulators, TMA-store epilogue), with tiles taken in row-block order
 //     from a global counter by the pair's leader and passed to both CTAs through a small ring
 //     of tile ids in shared memory;
-//   * warps 6..: one group of d/32 threads running the quantize stage of k1_rotquant.cu on
-//     token pairs taken from a global counter, writing each code's fp16 unit centroid into
-//     the GEMM's A operand and the norms s, and publishing, per block of 256 rows, how many
-//     rows are done (release add at GPU scope after a proxy fence);
+//   * warps 6..: one or two groups of d/32 threads running the quantize stage of
+//     k1_rotquant.cu on token pairs taken from a global counter, writing each code's fp16
+//     unit centroid into the GEMM's A operand and the norms s, and publishing, per block of
+//     256 rows, how many rows are done (release add at GPU scope after a proxy fence);
 //   * first of all, the GEMM warps decode the 2- or 4-bit weight codes into the fp16 B operand
 //     (a static share a warp, one proxy fence and one count a warp; the producers wait for the
 //     count once), and then, as ramp groups of d/32 threads with their buffers in the stage

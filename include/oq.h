@@ -141,8 +141,9 @@ int oq_quantize_act(const oq_rpbh *r, const oq_codebook *ca, const void *x, int 
 
 /* oq_quantize_act applied to GELU(x) = x Phi(x) = x (1 + erf(x/sqrt 2)) / 2, computed inside
  * the kernel: the quantized input of an MLP's down projection straight from the up
- * projection's pre-activation, with no GELU pass over memory.  GELU is evaluated in fp32
- * on each bf16 element (CUDA's erff); s = ||R GELU(x)||.  x must be OQ_BF16.  Same layouts and
+ * projection's pre-activation, with no GELU pass over memory.  GELU of each bf16 element is
+ * its fp64 value rounded to fp32 (a table over 2^-16 <= |x| < 16; x/2 below, x or 0 beyond
+ * +-16); s = ||R GELU(x)||.  x must be OQ_BF16.  Same layouts and
  * errors as oq_quantize_act, plus OQ_EINVAL for fp32 input.  The pages' models (FLUX, Wan)
  * feed their MLP down projections through GELU; this is the fused form of that step. */
 int oq_quantize_act_gelu(const oq_rpbh *r, const oq_codebook *ca, const void *x, int dtype,
@@ -186,8 +187,9 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * codes, the rotate+quantize kernel writes the packed codes instead and the GEMM decodes them
  * in shared memory (as oq_linear does under that variable); with OQ_LINEAR_PATH=wcodes and
  * 4-bit weight codes the GEMM decodes the weight codes itself (no weight decode launch and no
- * [out_features, d] fp16 buffer).  Otherwise, with 2- or 4-bit weight codes, d
- * a multiple of 1024 up to 5120, bf16 x and out_features <= T, the rotate+quantize kernel
+ * [out_features, d] fp16 buffer).  Otherwise, with 2- or 4-bit weight codes, d up to 5120
+ * whose d/32 threads a token pair fill whole warps (or nearly: d a multiple of 1024, or
+ * 896, 3968, ...), bf16 x and out_features <= T, the rotate+quantize kernel
  * also decodes the weight codes into the GEMM's B operand once it runs out of tokens;
  * otherwise the weight codes are decoded on a library-owned side stream of the device while x
  * is quantized.  With OQ_FUSED_STEP=1 (read once per process), bf16 x without GELU, 2/4/8-bit
