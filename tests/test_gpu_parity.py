@@ -406,6 +406,29 @@ def test_linear_path_selection(oq):
     assert len(set(hashes.values())) == 1, hashes
 
 
+def test_outputs_stay_inside_their_buffers(oq):
+    """Guard bytes around every output buffer (the stand-in for a bounds sanitizer): each
+    public call, on ragged shapes, writes only inside its outputs and writes all of them,
+    under every form the environment selects (child processes; the variables are read once
+    per process)."""
+    import os
+    import subprocess
+    import sys
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_canary_child.py")
+    forms = {"default": {}, "acodes": {"OQ_LINEAR_PATH": "fused"},
+             "wcodes": {"OQ_LINEAR_PATH": "wcodes"}, "single": {"OQ_GEMM_PAIR": "0"},
+             "fused_step": {"OQ_FUSED_STEP": "1"}, "k1_tc": {"OQ_K1_PATH": "tc"}}
+    for name, extra in forms.items():
+        env = dict(os.environ)
+        for k in ("OQ_LINEAR_PATH", "OQ_GEMM_PAIR", "OQ_FUSED_STEP", "OQ_K1_PATH",
+                  "OQ_FUSED_RAMP"):
+            env.pop(k, None)
+        env.update(extra)
+        r = subprocess.run([sys.executable, child], env=env, capture_output=True, text=True,
+                           timeout=600)
+        assert r.returncode == 0, name + ": " + r.stdout + r.stderr
+
+
 def test_fused_step_matches_the_two_calls(oq):
     """OQ_FUSED_STEP=1: oq_quantized_linear as one persistent kernel (the rotate+quantize stage
     and the CTA-pair GEMM side by side, rows handed over per 256-row block) equals
