@@ -24,6 +24,12 @@ struct DecodeParams {
     long long groups;           // rows * d / 8
     uint32_t L0, L1, H0, H1;    // decode8 sources (symmetric 4-bit path only)
     uint16_t lut[256];
+    // symmetric 4-bit path only: a second tensor decoded by the same launch (groups2 = 0:
+    // none), groups g >= groups being its groups g - groups, with its own decode8 sources
+    const uint8_t *codes2;
+    uint16_t *out2;
+    long long groups2;
+    uint32_t L0b, L1b, H0b, H1b;
 };
 
 constexpr int kDecThreads = 256;
@@ -100,22 +106,32 @@ __global__ void __launch_bounds__(kDecThreads) k2_decode(const __grid_constant__
     const uint32_t *tab32 = reinterpret_cast<const uint32_t *>(tab);
     const long long stride = (long long)gridDim.x * blockDim.x;
     uint4 *out = reinterpret_cast<uint4 *>(p.out);
-    for (long long g0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; g0 < p.groups;
+    uint4 *out2 = reinterpret_cast<uint4 *>(p.out2);
+    const long long total = p.groups + (SYM ? p.groups2 : 0);
+    for (long long g0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; g0 < total;
          g0 += kDecUnroll * stride) {
         uint64_t v[kDecUnroll];
 #pragma unroll
         for (int j = 0; j < kDecUnroll; ++j) {
             const long long g = g0 + j * stride;
-            v[j] = g < p.groups ? load_group<BITS>(p.codes, g) : 0;
+            if (SYM && g >= p.groups)
+                v[j] = g < total ? load_group<BITS>(p.codes2, g - p.groups) : 0;
+            else
+                v[j] = g < p.groups ? load_group<BITS>(p.codes, g) : 0;
         }
 #pragma unroll
         for (int j = 0; j < kDecUnroll; ++j) {
             const long long g = g0 + j * stride;
-            if (g < p.groups) {
+            if (g < total) {
                 if constexpr (SYM) {
                     uint32_t o[4];
-                    decode8((uint32_t)v[j], p.L0, p.L1, p.H0, p.H1, o);
-                    out[g] = make_uint4(o[0], o[1], o[2], o[3]);
+                    if (g < p.groups) {
+                        decode8((uint32_t)v[j], p.L0, p.L1, p.H0, p.H1, o);
+                        out[g] = make_uint4(o[0], o[1], o[2], o[3]);
+                    } else {
+                        decode8((uint32_t)v[j], p.L0b, p.L1b, p.H0b, p.H1b, o);
+                        out2[g - p.groups] = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
                 } else {
                     out[g] = decode_group<BITS>(tab32, v[j]);
                 }
@@ -126,7 +142,7 @@ __global__ void __launch_bounds__(kDecThreads) k2_decode(const __grid_constant__
 
 template <int BITS, bool SYM>
 cudaError_t decode(const DecodeParams &dp, cudaStream_t st, int num_sms) {
-    long long blocks = (dp.groups + kDecThreads - 1) / kDecThreads;
+    long long blocks = (dp.groups + (SYM ? dp.groups2 : 0) + kDecThreads - 1) / kDecThreads;
     const long long cap = (long long)num_sms * (2048 / kDecThreads);   // one resident wave
     if (blocks > cap)
         blocks = cap;
@@ -143,6 +159,10 @@ cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long lo
     dp.codes = codes;
     dp.out = out;
     dp.groups = rows * (d / 8);
+    dp.codes2 = nullptr;
+    dp.out2 = nullptr;
+    dp.groups2 = 0;
+    dp.L0b = dp.L1b = dp.H0b = dp.H1b = 0;
     for (int i = 0; i < 256; ++i)
         dp.lut[i] = lut[i];
     dp.L0 = dp.L1 = dp.H0 = dp.H1 = 0;
@@ -162,6 +182,29 @@ cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long lo
     if (e != cudaSuccess)
         *why = "decode launch";
     return e;
+}
+
+bool launch_decode_pair(int bits_a, const uint8_t *codes_a, uint16_t *out_a, long long rows_a,
+                        const uint16_t *lut_a, int bits_b, const uint8_t *codes_b,
+                        uint16_t *out_b, long long rows_b, const uint16_t *lut_b, int d,
+                        cudaStream_t st, int num_sms, cudaError_t *err, std::string *why) {
+    DecodeParams dp;
+    if (bits_a != 4 || bits_b != 4 ||
+        !decode8_sources(lut_a, &dp.L0, &dp.L1, &dp.H0, &dp.H1) ||
+        !decode8_sources(lut_b, &dp.L0b, &dp.L1b, &dp.H0b, &dp.H1b))
+        return false;
+    dp.codes = codes_a;
+    dp.out = out_a;
+    dp.groups = rows_a * (d / 8);
+    dp.codes2 = codes_b;
+    dp.out2 = out_b;
+    dp.groups2 = rows_b * (d / 8);
+    for (int i = 0; i < 256; ++i)
+        dp.lut[i] = 0;
+    *err = decode<4, true>(dp, st, num_sms);
+    if (*err != cudaSuccess)
+        *why = "decode launch";
+    return true;
 }
 
 }  // namespace oq

@@ -1191,16 +1191,30 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     uint16_t *A16 = nullptr, *B16 = static_cast<uint16_t *>(ws);
     if (wcodes)
         B16 = nullptr;
+    // both operands' 4-bit codes of odd-symmetric codebooks: one decode launch for the two
+    uint32_t src_a[4], src_w[4];
+    const bool both = !fused && !wcodes && ca->bits == 4 && cw->bits == 4 &&
+                      oq::decode8_sources(ca->lut, &src_a[0], &src_a[1], &src_a[2], &src_a[3]) &&
+                      oq::decode8_sources(cw->lut, &src_w[0], &src_w[1], &src_w[2], &src_w[3]);
     if (!fused) {
         A16 = static_cast<uint16_t *>(ws);
         if (!wcodes)
             B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
                                                oq::linear_workspace_b_offset(T, d));
-        e = timed(OQ_KERNEL_DECODE, st, [&] {
-            return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
-        });
+        if (both)
+            e = timed(OQ_KERNEL_DECODE, st, [&] {
+                cudaError_t err = cudaErrorInvalidValue;
+                oq::launch_decode_pair(ca->bits, x_codes, A16, T, ca->lut, cw->bits, W_codes,
+                                       B16, out_features, cw->lut, d, st, di->sms, &err, &why);
+                return err;
+            });
+        else
+            e = timed(OQ_KERNEL_DECODE, st, [&] {
+                return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms,
+                                         &why);
+            });
     }
-    if (e == cudaSuccess && !wcodes)
+    if (e == cudaSuccess && !wcodes && !both)
         e = timed(OQ_KERNEL_DECODE, st, [&] {
             return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
                                      di->sms, &why);
@@ -1265,14 +1279,27 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
     uint16_t *B16 = reinterpret_cast<uint16_t *>(static_cast<unsigned char *>(ws) +
                                                  oq::linear_workspace_b_offset(T, d));
     std::string why;
-    e = timed(OQ_KERNEL_DECODE, st, [&] {
-        return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
-    });
-    if (e == cudaSuccess)
+    uint32_t src_a[4], src_w[4];
+    const bool both = ca->bits == 4 && cw->bits == 4 &&
+                      oq::decode8_sources(ca->lut, &src_a[0], &src_a[1], &src_a[2], &src_a[3]) &&
+                      oq::decode8_sources(cw->lut, &src_w[0], &src_w[1], &src_w[2], &src_w[3]);
+    if (both) {
         e = timed(OQ_KERNEL_DECODE, st, [&] {
-            return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
-                                     di->sms, &why);
+            cudaError_t err = cudaErrorInvalidValue;
+            oq::launch_decode_pair(ca->bits, x_codes, A16, T, ca->lut, cw->bits, W_codes, B16,
+                                   out_features, cw->lut, d, st, di->sms, &err, &why);
+            return err;
         });
+    } else {
+        e = timed(OQ_KERNEL_DECODE, st, [&] {
+            return oq::launch_decode(ca->bits, x_codes, A16, T, d, ca->lut, st, di->sms, &why);
+        });
+        if (e == cudaSuccess)
+            e = timed(OQ_KERNEL_DECODE, st, [&] {
+                return oq::launch_decode(cw->bits, W_codes, B16, out_features, d, cw->lut, st,
+                                         di->sms, &why);
+            });
+    }
     if (e == cudaSuccess)
         e = timed(OQ_KERNEL_GEMM, st, [&] {
             return oq::launch_gemm(A16, nullptr, nullptr, B16, nullptr, nullptr, s, row_norms,

@@ -146,6 +146,12 @@ size_t linear_workspace_b_offset(int T, int d);
 
 cudaError_t launch_decode(int bits, const uint8_t *codes, uint16_t *out, long long rows, int d,
                           const uint16_t *lut, cudaStream_t st, int num_sms, std::string *why);
+// Both operands' codes in one decode launch when both are 4-bit codes of odd-symmetric
+// codebooks (byte-permute decode); false (nothing launched) otherwise.  *err: the launch.
+bool launch_decode_pair(int bits_a, const uint8_t *codes_a, uint16_t *out_a, long long rows_a,
+                        const uint16_t *lut_a, int bits_b, const uint8_t *codes_b,
+                        uint16_t *out_b, long long rows_b, const uint16_t *lut_b, int d,
+                        cudaStream_t st, int num_sms, cudaError_t *err, std::string *why);
 
 // y[T, N] = (s_t rn_o / d) * A[T, d] . B[N, d]^T   (fp16 x fp16 -> fp32 in TMEM)
 // A is A16 (fp16 centroids from the prepass) or, when A16 is null, x_codes4: 4-bit codes of
