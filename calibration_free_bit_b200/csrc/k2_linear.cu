@@ -37,7 +37,11 @@ __device__ unsigned int g_k2_err;
 // process exits.  Host code must not use the symbol as an address (it is a host-side stand-in);
 // noalloc_workspace() looks the device address up once per device.
 constexpr size_t kNoAllocWorkspaceBytes = 64ull << 20;
-static __device__ __align__(256) unsigned char g_noalloc_workspace[kNoAllocWorkspaceBytes];
+// beyond the operands: the split-K partials of a small-T call (at most 74 work units of one
+// 256 x 256 fp32 tile each, 18.5 MiB)
+constexpr size_t kNoAllocSplitBytes = 20ull << 20;
+static __device__ __align__(256) unsigned char
+    g_noalloc_workspace[kNoAllocWorkspaceBytes + kNoAllocSplitBytes];
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_STAGE_BYTES = BM * BK * 2;               // 16 KB
@@ -67,6 +71,10 @@ struct GemmParams {
     int M, N, K;
     float inv_d;
     long long test_wait_cycles; // > 0: the armed test wait (oq_debug_arm_wait_timeout)
+    int ksplit;                 // pair kernel: k-ranges per tile (1: none), kb_per k-blocks
+    int kb_per;                 // each; partials in rows part * m_pad + row of tmP
+    int m_pad;
+    void *y;                    // k2_splitk_reduce: the output
 };
 
 // The armed test of the bounded waits: after all of the kernel's work, one thread waits on a
@@ -424,7 +432,8 @@ static_assert(gemm_pair_smem<false>() <= 227 * 1024 && gemm_pair_smem<true>() <=
 template <bool BF16, int CODES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES != 0>(), 1)
     k2_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmY, const GemmParams p) {
+                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmP,
+                 const GemmParams p) {
     constexpr bool ACODES = CODES != 0;             // one operand arrives as codes
     constexpr int S = pair_stages<ACODES>();
     constexpr int kBarSets = ACODES ? 4 : 2;
@@ -454,6 +463,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
     const int n_tiles = (p.N + P_BN - 1) / P_BN;
     const int num_tiles = ((p.M + P_BM - 1) / P_BM) * n_tiles;
     const int num_kb = p.K / BK;
+    // work units: a tile, or with ksplit > 1 (the plain form, few tiles) one of its ksplit
+    // k-ranges of kb_per blocks, whose fp32 partial goes to tmP for k2_splitk_reduce
+    const int ksplit = p.ksplit;
+    const int num_units = num_tiles * ksplit;
+    auto unit_range = [&](int unit, int &tile, int &part, int &kb0, int &kb1) {
+        tile = unit / ksplit;
+        part = unit - tile * ksplit;
+        kb0 = part * p.kb_per;
+        kb1 = min(num_kb, kb0 + p.kb_per);
+    };
 
     pdl_trigger();
     if (threadIdx.x == 0) {
@@ -494,10 +513,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
         // ---------------- TMA producer (both CTAs) ----------------
         if (lane == 0) {
             uint32_t it = 0;
-            for (int tile = pair0; tile < num_tiles && !aborted(); tile += npair) {
+            for (int unit = pair0; unit < num_units && !aborted(); unit += npair) {
+                int tile, part, kb0, kb1;
+                unit_range(unit, tile, part, kb0, kb1);
                 const int m0 = (tile / n_tiles) * P_BM + (int)rank * 128;
                 const int n0 = (tile % n_tiles) * P_BN + (int)rank * 128;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (it >= S && !mbar_wait(empty_bar(s), ((it / S) & 1) ^ 1)) {
                         give_up(ERR_WAIT_EMPTY);
@@ -542,7 +563,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
         if (lane == 0 && rank == 0) {
             uint32_t it = 0;
             int i = 0;
-            for (int tile = pair0; tile < num_tiles && !aborted(); tile += npair, ++i) {
+            for (int unit = pair0; unit < num_units && !aborted(); unit += npair, ++i) {
+                int tile, part, kb0, kb1;
+                unit_range(unit, tile, part, kb0, kb1);
                 const int acc = i & 1;
                 if (i >= 2 && !mbar_wait(tempty_bar(acc), ((i >> 1) & 1) ^ 1)) {
                     give_up(ERR_WAIT_EMPTY);
@@ -551,7 +574,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * kAccCols);
                 bool ok = true;
-                for (int kb = 0; kb < num_kb; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % S;
                     if (!mbar_wait(full_bar(s), (it / S) & 1) ||
                         (ACODES && !mbar_wait(afull_bar(s), (it / S) & 1))) {
@@ -564,7 +587,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
                     const uint64_t db = sw128_desc(sB + s * P_B_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        mma_ss_pair(d_tmem, da + 2 * kk, db + 2 * kk, kIdescPair, (kb | kk) != 0);
+                        mma_ss_pair(d_tmem, da + 2 * kk, db + 2 * kk, kIdescPair,
+                                    (kb != kb0) || (kk != 0));
                     mma_commit_pair_mc(empty_bar(s), 0x3);
                 }
                 if (!ok)
@@ -583,7 +607,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
         unsigned char *out0p = basep + (out0 - base);
         uint32_t u = 0;
         int i = 0;
-        for (int tile = pair0; tile < num_tiles; tile += npair, ++i) {
+        for (int unit = pair0; unit < num_units; unit += npair, ++i) {
+            int tile, part, kb0, kb1;
+            unit_range(unit, tile, part, kb0, kb1);
             const int acc = i & 1;
             const int m0 = (tile / n_tiles) * P_BM + (int)rank * 128;
             const int n0 = (tile % n_tiles) * P_BN;
@@ -614,6 +640,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
                     tmem_ld32(t_base + (uint32_t)(c * kCW + 32), r1);
                 if (!rows_in || n0 + c * kCW >= p.N)
                     continue;
+                if (ksplit > 1) {
+                    // the unscaled fp32 partial of this k-range: rows part * m_pad + row of
+                    // tmP (x 1 x 1 in store_chunk is exact); bf16 y: two 32-column chunks
+#pragma unroll
+                    for (int h = 0; h < kCW / 32; ++h) {
+                        const uint32_t b = u & 1;
+                        if (lane == 0)
+                            bulk_wait_read<1>();
+                        __syncwarp();
+                        rn_w[lane] = 1.0f;
+                        __syncwarp();
+                        store_chunk(&tmP, out0p + b * kStageOut, out0 + b * kStageOut,
+                                    h == 0 ? r0 : r1, 1.0f, rn_w, lane, n0 + c * kCW + 32 * h,
+                                    part * p.m_pad + m0 + q * 32);
+                        ++u;
+                    }
+                    continue;
+                }
                 const uint32_t b = u & 1;
                 if (lane == 0)
                     bulk_wait_read<1>();
@@ -654,8 +698,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
         const uint32_t ready = rank == 0 ? 0u : 1u;
         uint32_t it = 0;
         bool stop = false;
-        for (int tile = pair0; tile < num_tiles && !stop; tile += npair) {
-            for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        for (int unit = pair0; unit < num_units && !stop; unit += npair) {
+            int tile, part, kb0, kb1;
+            unit_range(unit, tile, part, kb0, kb1);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 const int s = it % S;
                 const bool ok = mbar_wait(cfull_bar(s), (it / S) & 1);
                 if (!__all_sync(0xffffffffu, ok)) {
@@ -700,6 +746,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_threads<CODES !
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
                      ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+// The epilogue of a K-split pair GEMM: y = (the ksplit fp32 partials summed in order) *
+// (s[row] / d) * rn[col], the same expression as the one-pass epilogue, fp32 or bf16 (round to
+// nearest even).  One thread per 4 consecutive columns of a row; partial k of row r at
+// part + (k * m_pad + r) * N.
+template <bool BF16>
+__global__ void __launch_bounds__(256) k2_splitk_reduce(const float *part, int ksplit,
+                                                        const GemmParams p) {
+    pdl_trigger();
+    pdl_wait();
+    const int n4 = p.N / 4;
+    const long long total = (long long)p.M * n4;
+    const size_t part_stride = (size_t)p.m_pad * p.N;
+    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int row = (int)(idx / n4), c4 = (int)(idx - (long long)row * n4);
+        const float *src = part + (size_t)row * p.N + 4 * (size_t)c4;
+        float4 a = *reinterpret_cast<const float4 *>(src);
+        for (int k = 1; k < ksplit; ++k) {
+            const float4 b = *reinterpret_cast<const float4 *>(src + k * part_stride);
+            a.x += b.x;
+            a.y += b.y;
+            a.z += b.z;
+            a.w += b.w;
+        }
+        const float srow = p.s[row] * p.inv_d;
+        const float *rn = p.rn + 4 * (size_t)c4;
+        const float o0 = a.x * srow * rn[0], o1 = a.y * srow * rn[1];
+        const float o2 = a.z * srow * rn[2], o3 = a.w * srow * rn[3];
+        const size_t off = (size_t)row * p.N + 4 * (size_t)c4;
+        if constexpr (BF16) {
+            const __nv_bfloat162 h0 = __floats2bfloat162_rn(o0, o1);
+            const __nv_bfloat162 h1 = __floats2bfloat162_rn(o2, o3);
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.y) + off) =
+                make_uint2(*reinterpret_cast<const uint32_t *>(&h0),
+                           *reinterpret_cast<const uint32_t *>(&h1));
+        } else {
+            *reinterpret_cast<float4 *>(static_cast<float *>(p.y) + off) =
+                make_float4(o0, o1, o2, o3);
+        }
     }
 }
 
@@ -893,12 +981,13 @@ int gemm_pair_slots() {
 
 template <bool BF16, int CODES>
 cudaError_t launch_gemm_pair_t(const CUtensorMap &ma, const CUtensorMap &mb,
-                               const CUtensorMap &my, const GemmParams &gp, int pairs,
-                               cudaStream_t st, std::string *why) {
+                               const CUtensorMap &my, const CUtensorMap &mp,
+                               const GemmParams &gp, int pairs, cudaStream_t st,
+                               std::string *why) {
     constexpr bool ACODES = CODES != kCodesNone;
     const cudaError_t e =
         launch_pdl(k2_gemm_pair<BF16, CODES>, dim3(2 * pairs), dim3(pair_threads<ACODES>()),
-                   gemm_pair_smem<ACODES>(), st, ma, mb, my, gp);
+                   gemm_pair_smem<ACODES>(), st, ma, mb, my, mp, gp);
     if (e != cudaSuccess)
         *why = "k2_gemm_pair launch";
     return e;
@@ -920,7 +1009,7 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
                         const uint16_t *B16, const uint8_t *w_codes4, const uint16_t *lut_w,
                         const float *s, const float *rn, void *y, bool y_bf16, int T, int N,
                         int d, cudaStream_t st, int num_sms, std::string *why,
-                        long long test_wait_cycles) {
+                        long long test_wait_cycles, void *split_ws, size_t split_ws_bytes) {
     const bool acodes = A16 == nullptr, wcodes = B16 == nullptr;
     GemmParams gp;
     gp.test_wait_cycles = test_wait_cycles;
@@ -931,6 +1020,10 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
     gp.N = N;
     gp.K = d;
     gp.inv_d = 1.0f / (float)d;
+    gp.ksplit = 1;
+    gp.kb_per = d / BK;
+    gp.m_pad = 0;
+    gp.y = y;
     if (acodes && wcodes) {
         *why = "k2_gemm: at most one operand can arrive as codes";
         return cudaErrorInvalidValue;
@@ -962,17 +1055,84 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
                 *why = "cuTensorMapEncodeTiled failed";
                 return cudaErrorInvalidValue;
             }
-            const int tiles = ((N + P_BN - 1) / P_BN) * ((T + P_BM - 1) / P_BM);
-            const int pairs = tiles < slots ? tiles : slots;
-            if (acodes)
-                return y_bf16 ? launch_gemm_pair_t<true, kCodesA>(ma, mb, my, gp, pairs, st, why)
-                              : launch_gemm_pair_t<false, kCodesA>(ma, mb, my, gp, pairs, st, why);
-            if (wcodes)
-                return y_bf16 ? launch_gemm_pair_t<true, kCodesB>(ma, mb, my, gp, pairs, st, why)
-                              : launch_gemm_pair_t<false, kCodesB>(ma, mb, my, gp, pairs, st, why);
-            return y_bf16
-                       ? launch_gemm_pair_t<true, kCodesNone>(ma, mb, my, gp, pairs, st, why)
-                       : launch_gemm_pair_t<false, kCodesNone>(ma, mb, my, gp, pairs, st, why);
+            const int m_tiles = (T + P_BM - 1) / P_BM;
+            const int tiles = ((N + P_BN - 1) / P_BN) * m_tiles;
+            // Few tiles (small T): split each tile's K loop over ksplit work units, so that
+            // more CTA pairs work; their fp32 partials are summed by k2_splitk_reduce.
+            // (decided on the plain kernel's pair count, so that every operand form splits the
+            // same way and gives the same bits)
+            const int num_kb = d / BK;
+            const int plain = y_bf16 ? gemm_pair_slots<true, kCodesNone>()
+                                     : gemm_pair_slots<false, kCodesNone>();
+            int ksplit = 1;
+            if (plain > 0 && tiles * 2 <= plain && num_kb >= 8) {
+                ksplit = std::min(std::min(plain / tiles, num_kb / 4), 8);
+                if (ksplit >= 2) {
+                    gp.kb_per = (num_kb + ksplit - 1) / ksplit;
+                    ksplit = (num_kb + gp.kb_per - 1) / gp.kb_per;
+                }
+            }
+            auto go = [&](const CUtensorMap &mp, int pairs) -> cudaError_t {
+                if (acodes)
+                    return y_bf16 ? launch_gemm_pair_t<true, kCodesA>(ma, mb, my, mp, gp, pairs,
+                                                                      st, why)
+                                  : launch_gemm_pair_t<false, kCodesA>(ma, mb, my, mp, gp,
+                                                                       pairs, st, why);
+                if (wcodes)
+                    return y_bf16 ? launch_gemm_pair_t<true, kCodesB>(ma, mb, my, mp, gp, pairs,
+                                                                      st, why)
+                                  : launch_gemm_pair_t<false, kCodesB>(ma, mb, my, mp, gp,
+                                                                       pairs, st, why);
+                return y_bf16 ? launch_gemm_pair_t<true, kCodesNone>(ma, mb, my, mp, gp, pairs,
+                                                                     st, why)
+                              : launch_gemm_pair_t<false, kCodesNone>(ma, mb, my, mp, gp, pairs,
+                                                                      st, why);
+            };
+            if (ksplit < 2) {
+                gp.kb_per = num_kb;
+                return go(my, tiles < slots ? tiles : slots);
+            }
+            gp.ksplit = ksplit;
+            gp.m_pad = m_tiles * P_BM;
+            const size_t part_bytes = (size_t)ksplit * gp.m_pad * N * 4;
+            void *part = split_ws;
+            cudaError_t e = cudaSuccess;
+            if (split_ws) {
+                if (part_bytes > split_ws_bytes) {
+                    *why = "k2_gemm: split-K partials exceed the given workspace";
+                    return cudaErrorInvalidValue;
+                }
+            } else {
+                e = cudaMallocAsync(&part, part_bytes, st);
+                if (e != cudaSuccess) {
+                    *why = "k2_gemm: split-K partial buffer";
+                    return e;
+                }
+            }
+            CUtensorMap mp;
+            if (!make_out_map(&mp, part, ksplit * gp.m_pad, N, false)) {
+                if (!split_ws)
+                    cudaFreeAsync(part, st);
+                *why = "cuTensorMapEncodeTiled failed";
+                return cudaErrorInvalidValue;
+            }
+            const int units = tiles * ksplit;
+            e = go(mp, units < slots ? units : slots);
+            if (e == cudaSuccess) {
+                const long long work = (long long)T * (N / 4);
+                long long blocks = (work + 255) / 256;
+                if (blocks > (long long)num_sms * 8)
+                    blocks = (long long)num_sms * 8;
+                e = y_bf16 ? launch_pdl(k2_splitk_reduce<true>, dim3((unsigned)blocks), dim3(256),
+                                        0, st, static_cast<const float *>(part), ksplit, gp)
+                           : launch_pdl(k2_splitk_reduce<false>, dim3((unsigned)blocks),
+                                        dim3(256), 0, st, static_cast<const float *>(part),
+                                        ksplit, gp);
+                if (e != cudaSuccess)
+                    *why = "k2_splitk_reduce launch";
+            }
+            const cudaError_t e2 = split_ws ? cudaSuccess : cudaFreeAsync(part, st);
+            return e != cudaSuccess ? e : e2;
         }
     }
     if (wcodes) {
@@ -993,11 +1153,23 @@ cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint
                   : launch_gemm_t<false, false>(ma, mb, my, gp, grid, st, why);
 }
 
+bool gemm_splits_k(int T, int N, int d, bool y_bf16) {
+    if (!gemm_pair_enabled())
+        return false;
+    const int plain = y_bf16 ? gemm_pair_slots<true, kCodesNone>()
+                             : gemm_pair_slots<false, kCodesNone>();
+    const int tiles = ((N + P_BN - 1) / P_BN) * ((T + P_BM - 1) / P_BM);
+    const int num_kb = d / BK;
+    return plain > 0 && tiles * 2 <= plain && num_kb >= 8 &&
+           std::min(std::min(plain / tiles, num_kb / 4), 8) >= 2;
+}
+
 bool make_operand_map(CUtensorMap *map, const void *ptr, long long rows, int K) {
     return make_map(map, ptr, rows, K, 128);
 }
 
 size_t noalloc_workspace_bytes() { return kNoAllocWorkspaceBytes; }
+size_t noalloc_split_bytes() { return kNoAllocSplitBytes; }
 
 cudaError_t noalloc_workspace(void **out) {
     static std::mutex mu;

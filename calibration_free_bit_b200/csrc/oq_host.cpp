@@ -700,11 +700,16 @@ int linear_path() {
 }
 bool fused_requested() { return linear_path() == 1; }
 
-// The weight operand of this codebook decoded inside the GEMM (OQ_LINEAR_PATH=wcodes, 4-bit
-// odd-symmetric codebook, CTA-pair GEMM).
-bool wcodes_applies(const oq_codebook *cw) {
+// The weight operand of this codebook decoded inside the GEMM: 4-bit codes of an
+// odd-symmetric codebook and the CTA-pair GEMM, with OQ_LINEAR_PATH=wcodes, or by default when
+// T <= 256 (one 256-row tile: each weight row is decoded once either way, and the call saves
+// the decode launch and the [N, d] fp16 buffer; measured 19.8-22.8 against 24.6-28.0 us per
+// one-call step at d = N = 3072).
+bool wcodes_applies(const oq_codebook *cw, int T) {
     uint32_t src[4];
-    return linear_path() == 2 && cw->bits == 4 && oq::gemm_pair_enabled() &&
+    const int path = linear_path();
+    return (path == 2 || (path == 0 && T <= 256)) && cw->bits == 4 &&
+           oq::gemm_pair_enabled() &&
            oq::decode8_sources(cw->lut, &src[0], &src[1], &src[2], &src[3]);
 }
 
@@ -1178,7 +1183,7 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
     // OQ_LINEAR_PATH=fused, 4-bit activation codes are decoded inside the GEMM kernel and only
     // the weight codes get the prepass.
     const bool fused = ca->bits == 4 && fused_requested();
-    const bool wcodes = wcodes_applies(cw);
+    const bool wcodes = !fused && wcodes_applies(cw, T);
     const size_t ws_bytes = fused    ? (size_t)out_features * d * 2
                             : wcodes ? (size_t)T * d * 2
                                      : oq::linear_workspace_bytes(T, d, out_features);
@@ -1304,7 +1309,9 @@ int oq_linear_noalloc(const oq_codebook *ca, const oq_codebook *cw, const uint8_
         e = timed(OQ_KERNEL_GEMM, st, [&] {
             return oq::launch_gemm(A16, nullptr, nullptr, B16, nullptr, nullptr, s, row_norms,
                                    y, out_dtype == OQ_BF16, T, out_features, d, st, di->sms,
-                                   &why, take_armed(OQ_KERNEL_GEMM));
+                                   &why, take_armed(OQ_KERNEL_GEMM),
+                                   static_cast<unsigned char *>(ws) + have,
+                                   oq::noalloc_split_bytes());
         });
     if (e != cudaSuccess)
         return fail_cuda(e, why.c_str());
@@ -1356,8 +1363,11 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
     if (!side)
         return rc;
     // The whole step as one persistent kernel where it applies (OQ_FUSED_STEP=1)
+    // (not where the GEMM would split its K loop: few tiles leave the persistent kernel
+    // nothing to overlap, and the split form's summation order is the one to match)
     if (fused_step_requested() && !gelu && !tc_k1_requested() &&
-        oq::fused_step_supported(d, r->h, ca->bits, dtype == OQ_BF16))
+        oq::fused_step_supported(d, r->h, ca->bits, dtype == OQ_BF16) &&
+        !oq::gemm_splits_k(T, out_features, d, out_dtype == OQ_BF16))
         return fused_step(r, ca, cw, x, W_codes, row_norms, T, d, out_features, y, out_dtype, s,
                           (cudaStream_t)stream, dev, di, pool, who);
     // The activation operand takes one of three forms:
@@ -1375,7 +1385,7 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
                         oq::decode8_sources(ca->lut, &src_probe[0], &src_probe[1],
                                             &src_probe[2], &src_probe[3]);
     const bool direct = !acodes && oq::k1_a16_supported(ca->bits, r->h, dtype == OQ_BF16);
-    const bool wcodes = wcodes_applies(cw);
+    const bool wcodes = !acodes && wcodes_applies(cw, T);
     const size_t a_bytes = acodes ? 0 : align_up((size_t)T * d * 2, 1024);
     const size_t b_bytes = wcodes ? 0 : align_up((size_t)out_features * d * 2, 1024);
     const size_t s_bytes = s ? 0 : align_up((size_t)T * 4, 1024);

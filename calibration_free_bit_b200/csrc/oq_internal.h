@@ -159,12 +159,16 @@ bool launch_decode_pair(int bits_a, const uint8_t *codes_a, uint16_t *out_a, lon
 // B likewise: B16, or (B16 null; CTA-pair kernel only) w_codes4 with lut_w.  At most one
 // operand as codes.  y is fp32, or bf16 (round to nearest even of the fp32 epilogue value)
 // when y_bf16.  test_wait_cycles > 0 arms the kernel's test of its bounded waits
-// (oq_debug_arm_wait_timeout).
+// (oq_debug_arm_wait_timeout).  With few output tiles (fp16 operands, CTA-pair kernel) the
+// K loop is split over more CTA pairs and a reduce kernel sums their fp32 partials, in
+// split_ws (split_ws_bytes; an error if too small) or, when it is null, a stream-ordered
+// temporary buffer.
 cudaError_t launch_gemm(const uint16_t *A16, const uint8_t *x_codes4, const uint16_t *lut_a,
                         const uint16_t *B16, const uint8_t *w_codes4, const uint16_t *lut_w,
                         const float *s, const float *rn, void *y, bool y_bf16, int T, int N,
                         int d, cudaStream_t st, int num_sms, std::string *why,
-                        long long test_wait_cycles = 0);
+                        long long test_wait_cycles = 0, void *split_ws = nullptr,
+                        size_t split_ws_bytes = 0);
 
 // The online step in one persistent kernel (k3_fused.cu): the quantize stage and the CTA-pair
 // GEMM side by side on every SM, rows handed over through per-block counters.
@@ -209,10 +213,14 @@ bool make_operand_map(CUtensorMap *map, const void *ptr, long long rows, int K);
 
 // False when OQ_GEMM_PAIR=0 asks for the single-CTA GEMM (read once per process).
 bool gemm_pair_enabled();
+// True when launch_gemm splits the K loop of a [T, d] x [N, d] product (few output tiles).
+bool gemm_splits_k(int T, int N, int d, bool y_bf16);
 
 // Fixed device workspace of oq_linear_noalloc (a static __device__ array in k2_linear.cu):
 // its size, and its address on the current device (looked up once per device).
 size_t noalloc_workspace_bytes();
+// its region past the operands for split-K partials (noalloc_workspace + the size above)
+size_t noalloc_split_bytes();
 cudaError_t noalloc_workspace(void **out);
 
 // Device error words written by the kernels (bounded waits that gave up etc.):

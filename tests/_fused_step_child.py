@@ -1,7 +1,8 @@
 """Child process for the fused-step test: OQ_FUSED_STEP is read once per process, so the
 one-call path's persistent kernel (the quantize stage and the CTA-pair GEMM side by side) is
 exercised in a process of its own.  Every case must equal oq_quantize_act + oq_linear bit for
-bit (y and s); shapes outside the kernel's range must take the other forms, still identical.
+bit (y and s); shapes outside the kernel's range, or with so few output tiles that the GEMM
+splits its K loop, must take the other forms, still identical.
 Exits non-zero on any failure."""
 import os
 import sys
@@ -41,7 +42,7 @@ def armed_wait():
     """The fused kernel's armed test wait: the call does its work, the wait runs out after its
     short limit and oq_check reports bit 0x10 of the fused kernel's error word; the outputs
     equal an unarmed call's and the next call is clean."""
-    d, T, N = 1024, 300, 272
+    d, T, N = 1024, 2310, 784                  # enough tiles that the GEMM does not split K
     p = synth.sweep_projection(d, 128, 4, T)
     x = synth.activations(p).cuda()
     W = (torch.randn(N, d, generator=torch.Generator().manual_seed(3)) / d ** 0.5).cuda()
@@ -72,12 +73,13 @@ def main():
     cases = [
         (3072, 128, 4, 4, 4608, 3072, torch.float32, True),    # the attention projection
         (3072, 128, 4, 4, 4608, 3072, torch.bfloat16, True),
-        (1024, 64, 2, 4, 777, 272, torch.float32, False),      # ragged T (odd) and N
-        (2048, 256, 8, 2, 513, 528, torch.float32, False),
-        (4096, 128, 4, 8, 300, 1040, torch.bfloat16, False),
+        (1024, 64, 2, 4, 4099, 784, torch.float32, False),     # ragged T (odd) and N
+        (2048, 256, 8, 2, 4353, 528, torch.float32, False),
+        (4096, 128, 4, 8, 2310, 1040, torch.bfloat16, False),  # 8-bit weights: decode launch
+        # few tiles (the GEMM splits its K loop) or outside the kernel: the other forms
         (3072, 128, 4, 4, 1, 16, torch.float32, False),        # one token
-        (3072, 128, 4, 4, 2, 4096, torch.float32, False),      # more tiles than token blocks
-        (5120, 128, 4, 4, 64, 256, torch.float32, False),      # outside the kernel: other forms
+        (3072, 128, 4, 4, 2, 4096, torch.float32, False),
+        (5120, 128, 4, 4, 64, 256, torch.float32, False),
     ]
     ok = True
     for d, h, ba, bw, T, N, out, attn in cases:
