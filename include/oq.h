@@ -167,6 +167,12 @@ int oq_quantize_act_gelu(const oq_rpbh *r, const oq_codebook *ca, const void *x,
  * weight codes and OQ_LINEAR_PATH=wcodes, the weight codes are the ones decoded inside the
  * (CTA-pair) GEMM, each weight row once per 256-row tile of y, and only the activation codes
  * get an fp16 buffer (again the same y; with OQ_GEMM_PAIR=0 the variable has no effect).
+ * Without OQ_LINEAR_PATH, 4-bit weight codes of an odd-symmetric codebook take that form
+ * when T <= 256 (one row of tiles: each weight row is decoded once either way).  When the
+ * product has few 256 x 256 output tiles (small T), the GEMM splits its K loop over more CTA
+ * pairs and a second kernel sums their fp32 partials in a fixed order (a stream-ordered
+ * temporary buffer of at most ~19 MB): y then differs from the unsplit product by fp32
+ * summation order only, and every form of the call splits the same way.
  * Either way the temporary device memory is stream-ordered, from a library-owned
  * pool.  The fp16 operands meet in a tcgen05 GEMM on pairs of CTAs (256 x 256 output tiles);
  * the environment variable OQ_GEMM_PAIR=0 (read once per process) selects the single-CTA
@@ -214,8 +220,9 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
 
 /* oq_linear for callers that cannot allocate device memory.  The paper has no counterpart;
  * this is a deployment variant of the same computation, with the same arguments and errors as
- * oq_linear.  It always runs the decode prepass into fp16 operands followed by the GEMM (the
- * default form of oq_linear, bit-identical to it); it ignores OQ_LINEAR_PATH, so in a process
+ * oq_linear.  It always runs the decode prepass into fp16 operands followed by the GEMM,
+ * bit-identical to oq_linear's default forms (which feed the GEMM the same fp16 values, and
+ * split its K loop the same way at small T); it ignores OQ_LINEAR_PATH, so in a process
  * that set OQ_LINEAR_PATH=fused the two calls may differ in the last bits (both are within the
  * linear layer's parity bound).  oq_timing_* records its kernels like oq_linear's.
  * Who needs it: code that runs inside a host framework which owns all device memory and gives
@@ -223,8 +230,9 @@ int oq_quantized_linear(const oq_rpbh *r, const oq_codebook *ca, const oq_codebo
  * memory cap), and latency-critical serving loops that forbid allocation on the request path
  * because cudaMalloc/cudaFree can synchronise the device and stall other streams.
  * How: the two fp16 operand buffers live in a fixed array compiled into the library
- * (OQ_NOALLOC_WORKSPACE_BYTES = 64 MiB), which every GPU that loads the library holds until
- * the process exits.  The call allocates and frees nothing.
+ * (OQ_NOALLOC_WORKSPACE_BYTES = 64 MiB, plus 20 MiB for the split-K partials of small-T
+ * calls), which every GPU that loads the library holds until the process exits.  The call
+ * allocates and frees nothing.
  * Limit: 2*(T*d + out_features*d) bytes, each part rounded up to 1 KiB, must fit in
  * OQ_NOALLOC_WORKSPACE_BYTES (e.g. T = 4608, d = out_features = 3072 needs 47 MB); larger
  * calls return OQ_EINVAL with the sizes in oq_last_error(), before touching the device.
