@@ -191,9 +191,10 @@ int oq_linear(const oq_codebook *ca, const oq_codebook *cw, const uint8_t *x_cod
  * ba in {2, 4, 8}, 32 <= h <= 256; otherwise codes and the decode prepass are used inside the
  * call).  With OQ_LINEAR_PATH=fused (read once per process), bf16 x and 4-bit activation
  * codes, the rotate+quantize kernel writes the packed codes instead and the GEMM decodes them
- * in shared memory (as oq_linear does under that variable); with OQ_LINEAR_PATH=wcodes and
- * 4-bit weight codes the GEMM decodes the weight codes itself (no weight decode launch and no
- * [out_features, d] fp16 buffer).  Otherwise, with 2- or 4-bit weight codes, d up to 5120
+ * in shared memory (as oq_linear does under that variable); with OQ_LINEAR_PATH=wcodes, or
+ * by default when T <= 256, 4-bit weight codes of an odd-symmetric codebook are decoded by the
+ * GEMM itself (no weight decode launch and no [out_features, d] fp16 buffer); with few output
+ * tiles the GEMM splits its K loop as oq_linear does.  Otherwise, with 2- or 4-bit weight codes, d up to 5120
  * whose d/32 threads a token pair fill whole warps (or nearly: d a multiple of 1024, or
  * 896, 3968, ...), bf16 x and out_features <= T, the rotate+quantize kernel
  * also decodes the weight codes into the GEMM's B operand once it runs out of tokens;
