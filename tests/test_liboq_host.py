@@ -33,6 +33,25 @@ def test_library_exports_every_header_symbol():
     assert oq.version().startswith("liboq")
 
 
+def test_binding_constants_match_the_header():
+    """Every OQ_* constant the Python binding defines has the value of the header's #define
+    (status codes, element types, flags, kernel ids), and every kernel id has a name."""
+    import os
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    hdr = open(os.path.join(root, "include", "oq.h")).read()
+    defs = {}
+    for name, val in re.findall(r"^#define (OQ_[A-Z0-9_]+)\s+\(?(-?\d+)u?\)?", hdr, re.M):
+        defs[name] = int(val)
+    bound = {k: getattr(oq, k) for k in dir(oq) if k.startswith("OQ_") and
+             isinstance(getattr(oq, k), int)}
+    assert bound, "no constants in the binding"
+    for k, v in bound.items():
+        assert k in defs and defs[k] == v, (k, v, defs.get(k))
+    kernel_ids = {v for k, v in defs.items() if k.startswith("OQ_KERNEL_")}
+    assert kernel_ids == set(oq.KERNEL_NAMES), (kernel_ids, oq.KERNEL_NAMES)
+
+
 @pytest.mark.parametrize("d,h,seed", [(256, 64, 0), (3072, 128, 0), (13824, 128, 7),
                                       (16384, 256, 12345), (1024, 32, 2**63 + 5)])
 def test_rpbh_tables_bit_exact_vs_oracle(d, h, seed):
