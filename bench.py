@@ -1,10 +1,14 @@
 #!/usr/bin/env python
 """Benchmark: OrbitQuant online quantized-linear path on B200.
 
-One step = the whole hot path on one batch: oq_quantize_act (fused RPBH rotate + norm +
-Lloyd-Max codes of the activations) followed by oq_linear (codebook GEMM against weight codes
-quantized offline, before timing).  Default workload: the FLUX-like attention projection
-(T = 4608 tokens, d = 3072 -> 3072, bf16 inputs, h = 128, W4A4).
+One step = the whole hot path on one batch: by default one oq_quantized_linear call (fused
+RPBH rotate + norm + Lloyd-Max quantize of the activations, whose fp16 centroids go straight to
+the codebook GEMM against weight codes quantized offline, before timing); with --api calls,
+oq_quantize_act followed by oq_linear.  Default workload: the FLUX-like attention projection
+(T = 4608 tokens, d = 3072 -> 3072, bf16 inputs, h = 128, W4A4).  The JSON line carries the
+step rate (CUDA-graph replays), the end-to-end rate from pinned host memory (e2e), the
+rooflines of the GEMM (roofline) and of the quantize kernel (roofline_quantize, plus the
+codes-only launch as context), the oracle's CPU rate (cpu_baseline), clocks and launches.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
